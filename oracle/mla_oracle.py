@@ -1,0 +1,263 @@
+"""CPU oracle for the absorbed sparse-MLA decode step (float64, numpy).
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the package entry point's smoke
+check and the bench's CPU-baseline leg may import this module.  The CUDA
+library never calls it, and it shares no code with the CUDA path.
+
+Every function is a plain restatement of what the DeepSeek-V3.2-Exp pages
+define, in float64, with no blocking, fusion or reordering beyond the stated
+equations.  Library primitives (numpy matmul/einsum, exp, sqrt) serve as
+single steps.  All functions are shape-generic (head count, latent width,
+rotary width and head dims are taken from the arguments) so that tests can
+run them on hand-sized problems.
+
+Sources (page title, section):
+  * "Mix and project" (decode branch, model.py 590-606): absorbed decode --
+    fold W_UK into q_nope, score against the cached latent plus the shared
+    rotary key over the indexer's selected positions, scale, softmax, mix
+    the latent, apply W_UV per head.
+  * "Key heads" (equations k^C = c^KV W_UK, K_i = [K^C_i ; k^R]; prefill
+    listing, model.py 574-589): the materialised path used as a cross-check.
+  * "KV compression" (model.py 565-568) and "Rotated shared key"
+    (apply_rotary_emb, model.py 405-425): cache write and rotary embedding.
+
+Readings taken where the pages are silent (also listed in the design doc):
+  * index semantics follow the decode mask built by scatter of 0 into a -inf
+    row over [0, end_pos): a position counts once however often it is
+    listed; -1 is padding; any other index outside [0, end_pos) is ignored
+    and counted as invalid;
+  * a row whose selection is empty gives O = 0 (the reference softmax would
+    produce NaN);
+  * RMSNorm is y = x / sqrt(mean(x^2) + eps) * w;
+  * end_pos is given per batch row.
+
+Parity status: every function here is pinned by tests/test_oracle_pins.py
+(equivalences, closed forms, invariants, brute force and the pages' printed
+parameter counts); there is no printed numeric output on the pages to match.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+# ---------------------------------------------------------------------------
+# selection
+# ---------------------------------------------------------------------------
+
+
+def selected_positions(topk_row, end_pos: int, T: int):
+    """Valid distinct positions of one row, in first-occurrence order, and the
+    number of invalid entries (neither -1 padding nor in [0, min(end_pos, T)))."""
+    seen = set()
+    keep = []
+    invalid = 0
+    lim = min(int(end_pos), int(T))
+    for v in np.asarray(topk_row).tolist():
+        v = int(v)
+        if v == -1:
+            continue
+        if v < 0 or v >= lim:
+            invalid += 1
+            continue
+        if v not in seen:
+            seen.add(v)
+            keep.append(v)
+    return keep, invalid
+
+
+def index_mask(topk, end_pos, T: int):
+    """mask[b, t] = 1 iff t is listed in topk[b] and 0 <= t < end_pos[b].
+
+    Mirrors the decode mask ("Mix and project", decode listing): a -inf row
+    over [0, end_pos) into which the indexer's positions are scattered as 0.
+    Returns (uint8 mask [B, T], total count of invalid entries)."""
+    topk = np.asarray(topk)
+    B = topk.shape[0]
+    mask = np.zeros((B, T), dtype=np.uint8)
+    bad = 0
+    for b in range(B):
+        keep, inv = selected_positions(topk[b], int(end_pos[b]), T)
+        mask[b, keep] = 1
+        bad += inv
+    return mask, bad
+
+
+# ---------------------------------------------------------------------------
+# absorbed decode, step by step ("Mix and project", decode branch)
+# ---------------------------------------------------------------------------
+
+
+def fold_wuk(q_nope, wkv_b):
+    """q~[b,h,c] = sum_d q_nope[b,h,d] * W_UK[h,d,c], W_UK = wkv_b[:, :Dn, :]."""
+    Dn = q_nope.shape[-1]
+    w_uk = wkv_b[:, :Dn, :]
+    return np.einsum("bhd,hdc->bhc", q_nope, w_uk)
+
+
+def scores(q_tilde_bh, q_pe_bh, c_rows, pe_rows, scale):
+    """s[h,t] = (q~[h]·c_KV[t] + q_pe[h]·k_pe[t]) * softmax_scale."""
+    return (q_tilde_bh @ c_rows.T + q_pe_bh @ pe_rows.T) * scale
+
+
+def softmax_rows(s):
+    """Row softmax with the row maximum subtracted."""
+    m = s.max(axis=-1, keepdims=True)
+    e = np.exp(s - m)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def mix_latent(A, c_rows):
+    """O~[h,c] = sum_t A[h,t] * c_KV[t,c]."""
+    return A @ c_rows
+
+
+def apply_wuv(o_tilde, wkv_b, Dv):
+    """O[h,d] = sum_c O~[h,c] * W_UV[h,d,c], W_UV = wkv_b[:, -Dv:, :]."""
+    w_uv = wkv_b[:, -Dv:, :]
+    return np.einsum("hc,hdc->hd", o_tilde, w_uv)
+
+
+def decode_absorbed(q_nope, q_pe, wkv_b, c_kv, k_pe, topk, end_pos, scale,
+                    return_weights=False):
+    """Absorbed sparse decode for one query per batch row.
+
+    q_nope [B,H,Dn], q_pe [B,H,Rr], wkv_b [H, Dn+Dv, C], c_kv [B,T,C],
+    k_pe [B,T,Rr], topk [B,k] int, end_pos [B] int -> O [B,H,Dv] float64.
+    With return_weights the per-row attention weights and selected positions
+    are returned as well."""
+    q_nope = np.asarray(q_nope, dtype=np.float64)
+    q_pe = np.asarray(q_pe, dtype=np.float64)
+    wkv_b = np.asarray(wkv_b, dtype=np.float64)
+    B, Hh, Dn = q_nope.shape
+    Dv = wkv_b.shape[1] - Dn
+    T = c_kv.shape[1]
+    q_tilde = fold_wuk(q_nope, wkv_b)
+    out = np.zeros((B, Hh, Dv))
+    weights = []
+    for b in range(B):
+        keep, _ = selected_positions(topk[b], int(end_pos[b]), T)
+        if not keep:
+            weights.append((np.zeros((Hh, 0)), keep))
+            continue
+        c_rows = np.asarray(c_kv[b, keep], dtype=np.float64)
+        pe_rows = np.asarray(k_pe[b, keep], dtype=np.float64)
+        s = scores(q_tilde[b], q_pe[b], c_rows, pe_rows, scale)
+        A = softmax_rows(s)
+        out[b] = apply_wuv(mix_latent(A, c_rows), wkv_b, Dv)
+        weights.append((A, keep))
+    if return_weights:
+        return out, weights
+    return out
+
+
+# ---------------------------------------------------------------------------
+# materialised path ("Key heads": K_i = [c^KV W_UK,i ; k^R], V_i = c^KV W_UV,i)
+# ---------------------------------------------------------------------------
+
+
+def decode_materialised(q_nope, q_pe, wkv_b, c_kv, k_pe, topk, end_pos, scale):
+    """Per-head keys and values are expanded from the latent, every position
+    in [0, end_pos) is scored, the index mask (-inf everywhere, 0 at the
+    listed positions) is added, then softmax and the value mix -- the shape
+    of the prefill branch, specialised to one query."""
+    q_nope = np.asarray(q_nope, dtype=np.float64)
+    q_pe = np.asarray(q_pe, dtype=np.float64)
+    wkv_b = np.asarray(wkv_b, dtype=np.float64)
+    B, Hh, Dn = q_nope.shape
+    Dv = wkv_b.shape[1] - Dn
+    T = c_kv.shape[1]
+    out = np.zeros((B, Hh, Dv))
+    for b in range(B):
+        e = min(int(end_pos[b]), T)
+        c = np.asarray(c_kv[b, :e], dtype=np.float64)          # [e, C]
+        kv = np.einsum("tc,hjc->thj", c, wkv_b)                # [e, H, Dn+Dv]
+        k_nope, v = kv[:, :, :Dn], kv[:, :, Dn:]
+        pe = np.asarray(k_pe[b, :e], dtype=np.float64)         # [e, Rr]
+        k = np.concatenate([k_nope, np.broadcast_to(pe[:, None, :], (e, Hh, pe.shape[1]))], -1)
+        q = np.concatenate([q_nope[b], q_pe[b]], -1)           # [H, Dn+Rr]
+        s = np.einsum("hd,thd->ht", q, k) * scale
+        mask = np.full(e, -np.inf)
+        for v_idx in np.asarray(topk[b]).tolist():
+            if 0 <= v_idx < e:
+                mask[v_idx] = 0.0
+        s = s + mask[None, :]
+        if not np.isfinite(mask).any():
+            continue
+        m = s.max(-1, keepdims=True)
+        p = np.exp(s - m)
+        p = p / p.sum(-1, keepdims=True)
+        out[b] = np.einsum("ht,thd->hd", p, v)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# rotary embedding ("Rotated shared key", apply_rotary_emb)
+# ---------------------------------------------------------------------------
+
+
+def rope(x, R, interleaved=True):
+    """Rotate feature pairs of x [..., S, Hx, Rr] by R [S, Rr/2] (complex).
+
+    interleaved: pair j is (x[2j], x[2j+1]) and the result goes back to
+    (2j, 2j+1).  Otherwise pair j is (x[j], x[j+Rr/2]) and the result is laid
+    out as all real parts, then all imaginary parts."""
+    x = np.asarray(x, dtype=np.float64)
+    half = x.shape[-1] // 2
+    if interleaved:
+        z = x[..., 0::2] + 1j * x[..., 1::2]
+    else:
+        z = x[..., :half] + 1j * x[..., half:]
+    y = z * R[:, None, :]
+    out = np.empty_like(x)
+    if interleaved:
+        out[..., 0::2] = y.real
+        out[..., 1::2] = y.imag
+    else:
+        out[..., :half] = y.real
+        out[..., half:] = y.imag
+    return out
+
+
+# ---------------------------------------------------------------------------
+# cache write ("KV compression", model.py 565-568)
+# ---------------------------------------------------------------------------
+
+
+def rmsnorm(x, w, eps):
+    x = np.asarray(x, dtype=np.float64)
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps) * np.asarray(w, dtype=np.float64)
+
+
+def cache_write(x, w_kva, norm_w, eps, R_pos, C, interleaved=True):
+    """kv = x W_KVa, split [C latent, rotary]; latent -> RMSNorm; rotary ->
+    RoPE at the row's position.  x [rows, dim], w_kva [dim, C+Rr] (x·W form),
+    R_pos complex [rows, Rr/2] (the rotary coefficients of each row's
+    position).  Returns (latent [rows, C], rotary key [rows, Rr]) in float64."""
+    kv = np.asarray(x, dtype=np.float64) @ np.asarray(w_kva, dtype=np.float64)
+    lat, pe = kv[:, :C], kv[:, C:]
+    lat = rmsnorm(lat, norm_w, eps)
+    pe = rope(pe[:, None, :], R_pos, interleaved)[:, 0, :]
+    return lat, pe
+
+
+# ---------------------------------------------------------------------------
+# parameter counts (printed on the "Key heads", "KV compression", "Mix and
+# project" and "Query rotary up-projection" pages)
+# ---------------------------------------------------------------------------
+
+
+def parameter_counts(n_heads=128, kv_lora_rank=512, qk_nope=128, qk_rope=64,
+                     v_head=128, dim=7168, q_lora_rank=1536):
+    return {
+        "W_UK": kv_lora_rank * n_heads * qk_nope,
+        "W_KR": dim * qk_rope,
+        "key_heads_total": kv_lora_rank * n_heads * qk_nope + dim * qk_rope,
+        "wkv_a_latent": dim * kv_lora_rank,
+        "kv_norm": kv_lora_rank,
+        "kv_compression_total": dim * kv_lora_rank + kv_lora_rank,
+        "wkv_a_plus_norm": dim * (kv_lora_rank + qk_rope) + kv_lora_rank,
+        "W_O": n_heads * v_head * dim,
+        "W_QR": q_lora_rank * n_heads * qk_rope,
+        "wkv_b": kv_lora_rank * n_heads * (qk_nope + v_head),
+        "cache_per_position": kv_lora_rank + qk_rope,
+        "full_kv_per_position": n_heads * ((qk_nope + qk_rope) + v_head),
+    }

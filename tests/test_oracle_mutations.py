@@ -1,0 +1,160 @@
+"""Planted mistakes in the oracle (on the CPU) must each trip a pin.
+
+Each mutant replaces one step of the oracle with a plausible slip -- a
+dropped term, a wrong sign, a wrong weight slice, a transposed operand, a
+missing normalisation -- and the test asserts that at least one of the pins
+in test_oracle_pins.py fails under it.  This shows the pins can see such
+mistakes anywhere in the oracle.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import oracle.mla_oracle as om
+import test_oracle_pins as pins
+
+DECODE_PINS = [
+    lambda: pins.test_absorbed_equals_materialised_small_dims(0),
+    pins.test_all_selected_equals_unmasked_dense,
+    pins.test_softmax_rows_sum_to_one_and_nonnegative,
+    pins.test_duplicates_padding_and_invalid_entries,
+    pins.test_materialised_matches_with_duplicates,
+    pins.test_empty_selection_gives_zero,
+    pins.test_single_key_closed_form,
+    pins.test_zero_query_gives_uniform_mean,
+    pins.test_two_keys_closed_form,
+    pins.test_brute_force_scalar_loops,
+    pins.test_index_mask_brute_force,
+]
+ROPE_PINS = [
+    pins.test_rope_position_zero_is_identity,
+    pins.test_rope_unit_vector_closed_form,
+    pins.test_rope_preserves_pair_norms_and_relative_positions,
+    pins.test_rope_noninterleaved_is_permuted_interleaved,
+    pins.test_cache_write_with_selection_weights,
+]
+NORM_PINS = [pins.test_rmsnorm_unit_rms, pins.test_cache_write_with_selection_weights]
+
+
+def _fold_wrong_rows(q_nope, wkv_b):
+    Dn = q_nope.shape[-1]
+    return np.einsum("bhd,hdc->bhc", q_nope, wkv_b[:, -Dn:, :])
+
+
+def _fold_wrong_head(q_nope, wkv_b):
+    Dn = q_nope.shape[-1]
+    return np.einsum("bhd,hdc->bhc", q_nope, np.roll(wkv_b, 1, axis=0)[:, :Dn, :])
+
+
+def _scores_no_rope(qt, qpe, c, pe, scale):
+    return (qt @ c.T) * scale
+
+
+def _scores_rope_sign(qt, qpe, c, pe, scale):
+    return (qt @ c.T - qpe @ pe.T) * scale
+
+
+def _scores_no_scale(qt, qpe, c, pe, scale):
+    return qt @ c.T + qpe @ pe.T
+
+
+def _softmax_wrong_axis(s):
+    e = np.exp(s - s.max(axis=0, keepdims=True))
+    return e / e.sum(axis=0, keepdims=True)
+
+
+def _softmax_unnormalised(s):
+    return np.exp(s - s.max(axis=-1, keepdims=True))
+
+
+def _mix_transposed(A, c):
+    return (A / A.shape[1]) @ np.roll(c, 1, axis=0)
+
+
+def _wuv_wrong_rows(o_t, wkv_b, Dv):
+    return np.einsum("hc,hdc->hd", o_t, wkv_b[:, :Dv, :])
+
+
+def _wuv_transposed_head(o_t, wkv_b, Dv):
+    return np.einsum("hc,hdc->hd", o_t, np.roll(wkv_b, 1, axis=0)[:, -Dv:, :])
+
+
+def _select_no_dedup(row, end_pos, T):
+    keep, invalid = [], 0
+    for v in np.asarray(row).tolist():
+        if v == -1:
+            continue
+        if not (0 <= v < min(end_pos, T)):
+            invalid += 1
+            continue
+        keep.append(int(v))
+    return keep, invalid
+
+
+def _select_off_by_one(row, end_pos, T):
+    keep, invalid, seen = [], 0, set()
+    for v in np.asarray(row).tolist():
+        if v == -1:
+            continue
+        if not (0 <= v <= min(end_pos, T)) or v >= T:
+            invalid += 1
+            continue
+        if v not in seen:
+            seen.add(v)
+            keep.append(int(v))
+    return keep, invalid
+
+
+def _rope_conjugate(x, R, interleaved=True):
+    return _orig_rope(x, np.conj(R), interleaved)
+
+
+def _rope_swapped_pairs(x, R, interleaved=True):
+    x = np.asarray(x, dtype=np.float64)
+    return _orig_rope(x, R, not interleaved)
+
+
+def _rmsnorm_no_sqrt(x, w, eps):
+    x = np.asarray(x, dtype=np.float64)
+    return x / (np.mean(x * x, axis=-1, keepdims=True) + eps) * np.asarray(w)
+
+
+def _rmsnorm_sum_not_mean(x, w, eps):
+    x = np.asarray(x, dtype=np.float64)
+    return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps) * np.asarray(w)
+
+
+_orig_rope = om.rope
+
+MUTANTS = [
+    ("fold_wuk", _fold_wrong_rows, DECODE_PINS),
+    ("fold_wuk", _fold_wrong_head, DECODE_PINS),
+    ("scores", _scores_no_rope, DECODE_PINS),
+    ("scores", _scores_rope_sign, DECODE_PINS),
+    ("scores", _scores_no_scale, DECODE_PINS),
+    ("softmax_rows", _softmax_wrong_axis, DECODE_PINS),
+    ("softmax_rows", _softmax_unnormalised, DECODE_PINS),
+    ("mix_latent", _mix_transposed, DECODE_PINS),
+    ("apply_wuv", _wuv_wrong_rows, DECODE_PINS),
+    ("apply_wuv", _wuv_transposed_head, DECODE_PINS),
+    ("selected_positions", _select_no_dedup, DECODE_PINS),
+    ("selected_positions", _select_off_by_one, DECODE_PINS),
+    ("rope", _rope_conjugate, ROPE_PINS),
+    ("rope", _rope_swapped_pairs, ROPE_PINS),
+    ("rmsnorm", _rmsnorm_no_sqrt, NORM_PINS),
+    ("rmsnorm", _rmsnorm_sum_not_mean, NORM_PINS),
+]
+
+
+@pytest.mark.parametrize("name,mutant,checks", MUTANTS,
+                         ids=[f"{n}:{m.__name__}" for n, m, _ in MUTANTS])
+def test_planted_mistake_is_caught(monkeypatch, name, mutant, checks):
+    monkeypatch.setattr(om, name, mutant)
+    monkeypatch.setattr(oracle, name, mutant, raising=False)
+    caught = 0
+    for check in checks:
+        try:
+            check()
+        except (AssertionError, ValueError, IndexError):
+            caught += 1
+    assert caught >= 1, f"no pin caught the planted mistake in {name}"

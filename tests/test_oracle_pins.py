@@ -1,0 +1,426 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+No test here re-types the oracle's own formula: each compares it with an
+independent route (the materialised per-head key/value path, dense masked
+attention, scalar brute force, closed forms of special cases, invariants)
+or with numbers printed on the pages.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import mla_inputs as mi
+import oracle as orc
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand_problem(rng, B=2, H=4, Dn=8, Dv=6, C=16, Rr=4, T=40, k=17, scale=0.3):
+    q_nope = rng.standard_normal((B, H, Dn))
+    q_pe = rng.standard_normal((B, H, Rr))
+    wkv_b = rng.standard_normal((H, Dn + Dv, C)) / math.sqrt(C)
+    c_kv = rng.standard_normal((B, T, C))
+    k_pe = rng.standard_normal((B, T, Rr))
+    end_pos = np.array([T - 3 * b for b in range(B)])
+    k = min(k, int(end_pos.min()))
+    topk = np.stack([rng.permutation(int(end_pos[b]))[:k] for b in range(B)])
+    return q_nope, q_pe, wkv_b, c_kv, k_pe, topk, end_pos, scale
+
+
+def _rel(a, b):
+    return np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300)
+
+
+# ---------------------------------------------------------------------------
+# absorbed == materialised ("Key heads": folding W_UK into the queries gives
+# the same scores; "Mix and project": O_i = O~_i W_UV,i)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_absorbed_equals_materialised_small_dims(seed):
+    rng = np.random.default_rng(seed)
+    p = _rand_problem(rng)
+    a = orc.decode_absorbed(*p)
+    m = orc.decode_materialised(*p)
+    assert _rel(a, m) < 1e-12
+
+
+def test_absorbed_equals_materialised_model_dims():
+    wl = mi.make_small(B=2, T=70, k=33, seed=3, end_pos=[70, 51])
+    args = (mi.f64(wl.q_nope), mi.f64(wl.q_pe), mi.f64(wl.wkv_b),
+            mi.f64(wl.cache[..., :mi.C]), mi.f64(wl.cache[..., mi.C:]),
+            wl.topk.numpy(), wl.end_pos.numpy(), wl.scale)
+    a = orc.decode_absorbed(*args)
+    m = orc.decode_materialised(*args)
+    assert a.shape == (2, 128, 128)
+    assert _rel(a, m) < 1e-12
+
+
+def test_all_selected_equals_unmasked_dense():
+    """Selecting every position reproduces dense attention (no mask at all),
+    computed here from per-head keys/values built from the latent."""
+    rng = np.random.default_rng(7)
+    q_nope, q_pe, wkv_b, c_kv, k_pe, _, _, scale = _rand_problem(rng, B=1, T=12, k=12)
+    T = 12
+    topk = rng.permutation(T)[None, :]
+    end_pos = np.array([T])
+    a = orc.decode_absorbed(q_nope, q_pe, wkv_b, c_kv, k_pe, topk, end_pos, scale)
+    Dn = q_nope.shape[-1]
+    out = np.zeros_like(a)
+    for h in range(q_nope.shape[1]):
+        K = np.concatenate([c_kv[0] @ wkv_b[h, :Dn].T, k_pe[0]], 1)     # [T, Dn+Rr]
+        V = c_kv[0] @ wkv_b[h, Dn:].T                                   # [T, Dv]
+        q = np.concatenate([q_nope[0, h], q_pe[0, h]])
+        s = K @ q * scale
+        w = np.exp(s - s.max())
+        out[0, h] = (w / w.sum()) @ V
+    assert _rel(a, out) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# softmax / selection invariants
+# ---------------------------------------------------------------------------
+
+def test_softmax_rows_sum_to_one_and_nonnegative():
+    rng = np.random.default_rng(11)
+    p = _rand_problem(rng, k=25)
+    _, ws = orc.decode_absorbed(*p, return_weights=True)
+    for A, keep in ws:
+        assert A.shape[1] == len(keep) == 25
+        assert np.all(A >= 0)
+        assert np.max(np.abs(A.sum(1) - 1.0)) < 1e-12
+
+
+def test_permuting_the_selection_changes_nothing():
+    rng = np.random.default_rng(12)
+    p = list(_rand_problem(rng))
+    a = orc.decode_absorbed(*p)
+    p[5] = np.stack([row[rng.permutation(len(row))] for row in p[5]])
+    b = orc.decode_absorbed(*p)
+    assert _rel(b, a) < 1e-13
+
+
+def test_duplicates_padding_and_invalid_entries():
+    """Listed twice counts once (scatter of 0 is idempotent); -1 is padding;
+    other out-of-range entries are ignored and counted."""
+    rng = np.random.default_rng(13)
+    p = list(_rand_problem(rng, B=2, T=30, k=10))
+    base = orc.decode_absorbed(*p)
+    end_pos = p[6]
+    extra = np.array([[p[5][0, 0], -1, -1, int(end_pos[0]), -5],
+                      [p[5][1, 3], p[5][1, 3], -1, 10_000, int(end_pos[1]) + 2]])
+    p2 = list(p)
+    p2[5] = np.concatenate([p[5], extra], 1)
+    got = orc.decode_absorbed(*p2)
+    assert _rel(got, base) < 1e-13
+    mask, bad = orc.index_mask(p2[5], end_pos, 30)
+    assert bad == 2 + 2
+    mask0, bad0 = orc.index_mask(p[5], end_pos, 30)
+    assert bad0 == 0 and np.array_equal(mask, mask0)
+
+
+def test_materialised_matches_with_duplicates():
+    rng = np.random.default_rng(14)
+    p = list(_rand_problem(rng, B=1, T=20, k=6))
+    p[5] = np.concatenate([p[5], p[5][:, :3], -np.ones((1, 2), int)], 1)
+    assert _rel(orc.decode_absorbed(*p), orc.decode_materialised(*p)) < 1e-12
+
+
+def test_empty_selection_gives_zero():
+    rng = np.random.default_rng(15)
+    p = list(_rand_problem(rng, B=2, T=20, k=4))
+    p[5] = p[5].copy()
+    p[5][1] = -1
+    out = orc.decode_absorbed(*p)
+    assert np.all(out[1] == 0)
+    assert np.any(out[0] != 0)
+
+
+def test_index_mask_brute_force():
+    rng = np.random.default_rng(16)
+    T = 50
+    topk = rng.integers(-3, 60, size=(4, 30))
+    end_pos = np.array([50, 10, 33, 1])
+    mask, bad = orc.index_mask(topk, end_pos, T)
+    exp_bad = 0
+    for b in range(4):
+        for t in range(T):
+            listed = any(int(v) == t for v in topk[b])
+            assert mask[b, t] == (1 if listed and t < end_pos[b] else 0)
+        for v in topk[b]:
+            if v != -1 and not (0 <= v < end_pos[b]):
+                exp_bad += 1
+    assert bad == exp_bad
+
+
+# ---------------------------------------------------------------------------
+# closed forms
+# ---------------------------------------------------------------------------
+
+def test_single_key_closed_form():
+    """One selected position: the softmax weight is 1, so O_h = W_UV,h c_t."""
+    rng = np.random.default_rng(21)
+    q_nope, q_pe, wkv_b, c_kv, k_pe, _, _, scale = _rand_problem(rng, B=2, T=9)
+    topk = np.array([[4], [8]])
+    end_pos = np.array([9, 9])
+    out = orc.decode_absorbed(q_nope, q_pe, wkv_b, c_kv, k_pe, topk, end_pos, scale)
+    Dn = q_nope.shape[-1]
+    for b, t in ((0, 4), (1, 8)):
+        for h in range(q_nope.shape[1]):
+            assert np.allclose(out[b, h], wkv_b[h, Dn:] @ c_kv[b, t], rtol=0, atol=1e-13)
+
+
+def test_zero_query_gives_uniform_mean():
+    """q = 0: all scores are 0, weights are 1/n, O_h = W_UV,h mean(c_sel)."""
+    rng = np.random.default_rng(22)
+    q_nope, q_pe, wkv_b, c_kv, k_pe, topk, end_pos, scale = _rand_problem(rng)
+    q_nope[:] = 0
+    q_pe[:] = 0
+    out = orc.decode_absorbed(q_nope, q_pe, wkv_b, c_kv, k_pe, topk, end_pos, scale)
+    Dn = q_nope.shape[-1]
+    for b in range(out.shape[0]):
+        mean = c_kv[b, topk[b]].mean(0)
+        for h in range(out.shape[1]):
+            assert np.allclose(out[b, h], wkv_b[h, Dn:] @ mean, atol=1e-13)
+
+
+def test_shared_rotary_key_shift_invariance():
+    """If every selected position has the same rotary key, the rotary term
+    adds the same constant to each score of a head and cancels in the
+    softmax: the result does not depend on q_pe."""
+    rng = np.random.default_rng(23)
+    q_nope, q_pe, wkv_b, c_kv, k_pe, topk, end_pos, scale = _rand_problem(rng)
+    k_pe[:] = rng.standard_normal(k_pe.shape[-1])
+    a = orc.decode_absorbed(q_nope, q_pe, wkv_b, c_kv, k_pe, topk, end_pos, scale)
+    b = orc.decode_absorbed(q_nope, 5 * rng.standard_normal(q_pe.shape), wkv_b, c_kv,
+                            k_pe, topk, end_pos, scale)
+    assert _rel(a, b) < 1e-12
+
+
+def test_two_keys_closed_form():
+    """Two positions: weight of the first is the logistic of the score gap."""
+    rng = np.random.default_rng(24)
+    q_nope, q_pe, wkv_b, c_kv, k_pe, _, _, scale = _rand_problem(rng, B=1, T=5)
+    Dn = q_nope.shape[-1]
+    topk = np.array([[1, 3]])
+    out = orc.decode_absorbed(q_nope, q_pe, wkv_b, c_kv, k_pe, topk, np.array([5]), scale)
+    for h in range(q_nope.shape[1]):
+        K1 = np.concatenate([wkv_b[h, :Dn] @ c_kv[0, 1], k_pe[0, 1]])
+        K3 = np.concatenate([wkv_b[h, :Dn] @ c_kv[0, 3], k_pe[0, 3]])
+        q = np.concatenate([q_nope[0, h], q_pe[0, h]])
+        w1 = 1.0 / (1.0 + math.exp(-(q @ K1 - q @ K3) * scale))
+        expect = wkv_b[h, Dn:] @ (w1 * c_kv[0, 1] + (1 - w1) * c_kv[0, 3])
+        assert np.allclose(out[0, h], expect, atol=1e-13)
+
+
+def test_brute_force_scalar_loops():
+    """Hand-sized problem, every sum written as a scalar loop over the
+    materialised definitions (K_i = [c W_UK,i^T ; k^R], V_i = c W_UV,i^T)."""
+    rng = np.random.default_rng(25)
+    H, Dn, Dv, C, Rr, T = 2, 2, 3, 3, 2, 4
+    q_nope = rng.standard_normal((1, H, Dn))
+    q_pe = rng.standard_normal((1, H, Rr))
+    wkv_b = rng.standard_normal((H, Dn + Dv, C))
+    c_kv = rng.standard_normal((1, T, C))
+    k_pe = rng.standard_normal((1, T, Rr))
+    topk = np.array([[2, 0, 3]])
+    scale = 0.7
+    out = orc.decode_absorbed(q_nope, q_pe, wkv_b, c_kv, k_pe, topk, np.array([T]), scale)
+    for h in range(H):
+        s = {}
+        for t in (2, 0, 3):
+            acc = 0.0
+            for d in range(Dn):
+                kc = 0.0
+                for c in range(C):
+                    kc += c_kv[0, t, c] * wkv_b[h, d, c]
+                acc += q_nope[0, h, d] * kc
+            for r in range(Rr):
+                acc += q_pe[0, h, r] * k_pe[0, t, r]
+            s[t] = acc * scale
+        mx = max(s.values())
+        z = sum(math.exp(v - mx) for v in s.values())
+        for d in range(Dv):
+            o = 0.0
+            for t in (2, 0, 3):
+                v = 0.0
+                for c in range(C):
+                    v += c_kv[0, t, c] * wkv_b[h, Dn + d, c]
+                o += math.exp(s[t] - mx) / z * v
+            assert abs(out[0, h, d] - o) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# rotary embedding ("Rotated shared key", apply_rotary_emb)
+# ---------------------------------------------------------------------------
+
+def _angles(T, theta=1e4, Rr=64):
+    j = np.arange(Rr // 2)
+    return np.outer(np.arange(T), theta ** (-2.0 * j / Rr))
+
+
+def test_rope_table_matches_definition():
+    """R[t, j] = exp(i t theta^(-2j/64)) up to fp32 rounding of the angle."""
+    T = 4096
+    R = mi.rope_complex(mi.rope_table(T))
+    ang = _angles(T)
+    err = np.abs(R - np.exp(1j * ang))
+    # the fp32 product t*freq carries up to ~T * 2^-24 rad of rounding
+    assert err.max() < T * 2.0 ** -23 + 1e-6
+    assert np.all(R[0] == 1.0)
+
+
+def test_rope_position_zero_is_identity():
+    x = np.random.default_rng(1).standard_normal((2, 1, 3, 64))
+    R = np.ones((1, 32), dtype=complex)
+    assert np.array_equal(orc.rope(x, R, True), x)
+    assert np.array_equal(orc.rope(x, R, False), x)
+
+
+def test_rope_unit_vector_closed_form():
+    """Pair (1, 0) rotated by angle a becomes (cos a, sin a)."""
+    ang = _angles(7)
+    R = np.exp(1j * ang)
+    x = np.zeros((1, 7, 1, 64))
+    x[..., 0::2] = 1.0
+    y = orc.rope(x, R, True)
+    assert np.allclose(y[0, :, 0, 0::2], np.cos(ang), atol=1e-15)
+    assert np.allclose(y[0, :, 0, 1::2], np.sin(ang), atol=1e-15)
+    x2 = np.zeros((1, 7, 1, 64))
+    x2[..., :32] = 1.0
+    y2 = orc.rope(x2, R, False)
+    assert np.allclose(y2[0, :, 0, :32], np.cos(ang), atol=1e-15)
+    assert np.allclose(y2[0, :, 0, 32:], np.sin(ang), atol=1e-15)
+
+
+def test_rope_preserves_pair_norms_and_relative_positions():
+    rng = np.random.default_rng(3)
+    T = 40
+    R = np.exp(1j * _angles(T))
+    q = rng.standard_normal(64)
+    k = rng.standard_normal(64)
+    xq = np.broadcast_to(q, (1, T, 1, 64)).copy()
+    xk = np.broadcast_to(k, (1, T, 1, 64)).copy()
+    rq = orc.rope(xq, R, True)[0, :, 0]
+    rk = orc.rope(xk, R, True)[0, :, 0]
+    pn = lambda v: v[..., 0::2] ** 2 + v[..., 1::2] ** 2  # noqa: E731
+    assert np.allclose(pn(rq), pn(xq[0, :, 0]), atol=1e-12)
+    # <RoPE(q, t1), RoPE(k, t2)> depends only on t1 - t2
+    for d in (0, 3, 11):
+        vals = [rq[t + d] @ rk[t] for t in range(0, T - d)]
+        assert np.ptp(vals) < 1e-10
+
+
+def test_rope_noninterleaved_is_permuted_interleaved():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((2, 5, 3, 64))
+    R = np.exp(1j * _angles(5))
+    perm = np.empty(64, dtype=int)
+    perm[0::2] = np.arange(32)
+    perm[1::2] = np.arange(32, 64)
+    inter = orc.rope(x[..., perm], R, True)
+    non = orc.rope(x, R, False)
+    assert np.allclose(non, inter[..., np.argsort(perm)], atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# RMSNorm and cache write ("KV compression")
+# ---------------------------------------------------------------------------
+
+def test_rmsnorm_unit_rms():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((6, 512)) * 3.0
+    eps = 1e-6
+    y = orc.rmsnorm(x, np.ones(512), eps)
+    ms = np.mean(x * x, -1)
+    assert np.allclose(np.sqrt(np.mean(y * y, -1)), np.sqrt(ms / (ms + eps)), rtol=1e-14)
+    # positive homogeneity: y(a x) = y(x) when eps = 0
+    assert np.allclose(orc.rmsnorm(7 * x, np.ones(512), 0.0), orc.rmsnorm(x, np.ones(512), 0.0),
+                       rtol=1e-14)
+    w = rng.standard_normal(512)
+    assert np.allclose(orc.rmsnorm(x, w, eps), y * w, rtol=1e-14)
+
+
+def test_cache_write_with_selection_weights():
+    """With W_KVa a 0/1 selection matrix, kv is a column pick of x: the latent
+    is RMSNorm of the picked columns, the rotary key is their rotation."""
+    rng = np.random.default_rng(6)
+    dim, C, Rr, rows = 40, 16, 4, 3
+    x = rng.standard_normal((rows, dim))
+    cols = rng.permutation(dim)[:C + Rr]
+    W = np.zeros((dim, C + Rr))
+    W[cols, np.arange(C + Rr)] = 1.0
+    ang = rng.uniform(-3, 3, size=(rows, Rr // 2))
+    Rp = np.exp(1j * ang)
+    lat, pe = orc.cache_write(x, W, np.ones(C), 1e-6, Rp, C)
+    pick = x[:, cols]
+    ms = np.mean(pick[:, :C] ** 2, -1, keepdims=True)
+    assert np.allclose(lat, pick[:, :C] / np.sqrt(ms + 1e-6), rtol=1e-14)
+    a, b = pick[:, C::2], pick[:, C + 1::2]
+    assert np.allclose(pe[:, 0::2], a * np.cos(ang) - b * np.sin(ang), atol=1e-14)
+    assert np.allclose(pe[:, 1::2], a * np.sin(ang) + b * np.cos(ang), atol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# numbers printed on the pages
+# ---------------------------------------------------------------------------
+
+def test_parameter_counts_match_the_pages():
+    gold = json.load(open(os.path.join(GOLD, "param_counts.json")))
+    pc = orc.parameter_counts()
+    for key in ("W_UK", "W_KR", "key_heads_total", "wkv_a_latent", "kv_norm",
+                "kv_compression_total", "W_O", "W_QR", "cache_per_position",
+                "full_kv_per_position"):
+        assert pc[key] == gold[key]["value"], key
+    assert pc["key_heads_total"] * 58 == gold["key_heads_x58"]["value"]
+    assert pc["W_O"] * 58 == gold["W_O_x58"]["value"]
+    assert pc["W_QR"] * 58 == gold["W_QR_x58"]["value"]
+    assert pc["kv_compression_total"] * 58 == gold["kv_compression_x58"]["value"]
+    # wkv_a + kv_norm = 7168 x 576 + 512 = latent part + rotary part + norm
+    assert pc["wkv_a_plus_norm"] == gold["wkv_a_latent"]["value"] + gold["W_KR"]["value"] \
+        + gold["kv_norm"]["value"]
+    # wkv_b = W_UK + W_UV, each 512 x 16,384
+    assert pc["wkv_b"] == 2 * gold["W_UK"]["value"]
+
+
+def test_decode_example_shape_from_the_pages():
+    """'Mix and project' at position 1000: A is [B, 128 heads, 1 query, 1001
+    keys] and c^KV is [B, 1001, 512].  The all-selected tiny workload has
+    exactly this shape."""
+    wl = mi.make_config(0)
+    assert tuple(wl.cache.shape) == (1, 1001, 576)
+    assert int(wl.end_pos[0]) == 1001 and wl.k == 1001
+    rows = mi.f64(wl.cache)
+    _, ws = orc.decode_absorbed(mi.f64(wl.q_nope), mi.f64(wl.q_pe), mi.f64(wl.wkv_b),
+                                rows[..., :512], rows[..., 512:], wl.topk.numpy(),
+                                wl.end_pos.numpy(), wl.scale, return_weights=True)
+    A, keep = ws[0]
+    assert A.shape == (128, 1001) and sorted(keep) == list(range(1001))
+
+
+def test_score_scale_is_unit_variance_for_the_workloads():
+    """With the workload distributions, scaled scores have variance ~1
+    (128*512*(1/512) + 64 = 192, times 1/192): a non-degenerate softmax."""
+    wl = mi.make_small(B=2, T=300, k=200, seed=9)
+    q_t = orc.fold_wuk(mi.f64(wl.q_nope), mi.f64(wl.wkv_b))
+    rows = mi.f64(wl.cache[0, :200])
+    s = orc.scores(q_t[0], mi.f64(wl.q_pe[0]), rows[:, :512], rows[:, 512:], wl.scale)
+    assert 0.8 < s.var() < 1.25
+
+
+def test_inputs_are_seeded_and_shapes_match():
+    a = mi.make_small(seed=1)
+    b = mi.make_small(seed=1)
+    assert torch.equal(a.cache, b.cache) and torch.equal(a.topk, b.topk)
+    for b_ in range(a.B):
+        row = a.topk[b_].tolist()
+        valid = [v for v in row if 0 <= v < int(a.end_pos[b_])]
+        assert len(set(valid)) == len(valid)
+    w3 = mi.make_config(1)
+    assert tuple(w3.topk.shape) == (8, 2048)
+    for b_ in range(8):
+        assert len(set(w3.topk[b_].tolist())) == 2048
