@@ -1,0 +1,453 @@
+#!/usr/bin/env python
+"""Benchmark of the absorbed sparse-MLA decode step (DeepSeek-V3.2-Exp sparse
+latent attention, decode branch) on B200.
+
+Workload (default): B=128 decode rows, per-row end_pos uniform in
+[4096, 131072], top-k = 2048 positions per row (half from the last 4096
+positions, half from the rest), bf16 cache [128, 131072, 576] (19.3 GB),
+128 heads.  One step = one ``mla_decode`` call over the batch: fold of W_UK,
+gather + scores + softmax + latent mix, split merge + W_UV.
+
+Metric: head*keys/s = (rows x selected keys x 128 heads) per second, summed
+over ranks; also microseconds per step.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Under torchrun each rank runs the same per-GPU workload (weak scaling, no
+data-path collective); the timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+HEADS = 128
+ROW_BYTES = 576 * 2
+METRIC = "sparse MLA decode head*keys/s"
+UNIT = "head*keys/s"
+L2_FLUSH_BYTES = 256 << 20
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "core_kernel_config3_traffic.txt")
+
+
+# ---------------------------------------------------------------------------
+# host-side helpers (importable without a GPU; covered by CPU tests)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def algorithmic_work(B: int, k: int):
+    """Bytes and flops the method itself must move / compute per step:
+    gathered rows + queries + indices + output + wkv_b read once; fold and
+    W_UV GEMMs + the two score/mix contractions over the selected keys."""
+    bytes_ = B * k * ROW_BYTES + B * (HEADS * 128 * 2 + HEADS * 64 * 2 + 4 * k + HEADS * 128 * 2) \
+        + 128 * 256 * 512 * 2
+    flops = B * (2 * 2 * HEADS * 128 * 512 + k * 2 * HEADS * (576 + 512))
+    return bytes_, flops
+
+
+def core_kernel_work(B: int, k: int):
+    """Algorithmic bytes / flops of the attend kernel alone: each selected
+    row (1152 B) and its index (4 B) once; 2*128*(576+512) flops per key."""
+    return B * k * (ROW_BYTES + 4), B * k * 2 * HEADS * (576 + 512)
+
+
+def load_peaks(path=os.path.join(ROOT, "MEASURED_PEAKS.json")):
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for rel in ("sparse_head_latent_absorbed_b200/csrc/decode.cu",
+                "sparse_head_latent_absorbed_b200/csrc/common.cuh"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic():
+    """Per-launch DRAM bytes of the attend kernel from the committed ncu
+    summary, or None when that summary is missing or was taken on other
+    kernel sources."""
+    try:
+        kv = {}
+        with open(PROFILE_TRAFFIC) as f:
+            for line in f:
+                if ":" in line:
+                    a, b = line.split(":", 1)
+                    kv[a.strip()] = b.strip()
+        if kv.get("source_sha256") != kernel_source_sha():
+            return None
+        return float(kv["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max over ranks (a timing reduction, not part of the data path)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the float64 oracle on the host cores
+# ---------------------------------------------------------------------------
+
+def oracle_sample_rate(wl, rows, repeats=1):
+    """Time the oracle (as it stands) on the compacted selected rows of the
+    given batch rows; returns (head*keys/s, seconds, threads)."""
+    import numpy as np
+
+    import mla_inputs as mi
+    import oracle as orc
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    prepared = []
+    for b in rows:
+        r, keep = mi.compact_rows(wl, b)
+        r = mi.f64(r)
+        n = len(keep)
+        prepared.append((mi.f64(wl.q_nope[b:b + 1]), mi.f64(wl.q_pe[b:b + 1]), r[None, :, :512],
+                         r[None, :, 512:], np.arange(n)[None], np.array([n])))
+    wkv = mi.f64(wl.wkv_b)
+    keys = 0
+    t0 = time.perf_counter()
+    for _ in range(repeats):
+        for qn, qp, c, pe, idx, ep in prepared:
+            orc.decode_absorbed(qn, qp, wkv, c, pe, idx, ep, wl.scale)
+            keys += idx.shape[1]
+    dt = time.perf_counter() - t0
+    return keys * HEADS / dt, dt, threads
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import torch
+
+    import mla_inputs as mi
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    wl = mi.make_config(args.config, device=dev,
+                        batch=slice(0, min(8, {0: 1, 1: 8, 2: 64, 3: 128, 4: 32}[args.config])))
+    rows = list(range(wl.B))
+    for _ in range(args.warmup):
+        oracle_sample_rate(wl, rows[:1])
+    rates, secs, threads = [], 0.0, 1
+    for _ in range(args.steps):
+        r, dt, threads = oracle_sample_rate(wl, rows)
+        rates.append(r)
+        secs += dt
+    value = len(rates) * len(rows) * wl.k * HEADS / secs
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(args.config, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{len(rows)} batch rows of the workload per step "
+                                   f"(selected rows only), float64 numpy oracle"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(cid: int, world: int):
+    desc = {
+        0: ("tiny dense decode B=1 end_pos=1001 all 1001 selected", 1, 1001),
+        1: ("decode B=8 end_pos=4096 top-k=2048", 8, 2048),
+        2: ("decode B=64 end_pos=32768 top-k=2048", 64, 2048),
+        3: ("decode B=128 end_pos~U[4096,131072] top-k=2048 (1024 recent + 1024 older), "
+            "bf16 cache [128,131072,576]", 128, 2048),
+        4: ("cache-write B=32 at 65535 + decode top-k=2048 over 65536", 32, 2048),
+    }[cid]
+    return {"workload": desc[0], "batch_per_gpu": desc[1], "global_batch": desc[1] * world,
+            "top_k": desc[2], "heads": HEADS, "latent": 512, "rope": 64,
+            "l2": "flushed between steps (256 MiB write)", "parallelism": f"replicas x{world}"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    import mla_inputs as mi
+    import sparse_head_latent_absorbed_b200 as shla
+
+    wl = mi.make_config(args.config, device=dev)
+    B, k = wl.B, wl.k
+    ws = torch.empty(shla.mla_decode_workspace_bytes(B, k), dtype=torch.uint8, device=dev)
+    out = torch.empty(B, HEADS, 128, dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(2, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    write = args.config == 4
+    cw_ws = None
+    if write:
+        cw_ws = torch.empty(shla.mla_cache_write_workspace_bytes(B), dtype=torch.uint8, device=dev)
+        tab = wl.rope[wl.write_pos:wl.write_pos + 1].contiguous()
+
+    def step():
+        if write:
+            shla.mla_cache_write(wl.x, wl.w_kva, wl.norm_w, wl.eps, tab, wl.write_pos, wl.cache,
+                                 ws=cw_ws)
+        shla.mla_decode(wl.q_nope, wl.q_pe, wl.wkv_b, wl.cache, wl.topk, wl.end_pos, wl.scale,
+                        out=out, ws=ws, status=status)
+
+    launches_per_step = 3 + (2 if write else 0)
+    smi_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local
+
+    # ---- device-timed steps ----
+    with ClockSampler(smi_index) as clk:
+        for _ in range(args.warmup):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
+        barrier(world)
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    clocks = clk.summary()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = reduce_max(sum(step_ms), world, dev)
+    ms_per_step = total_ms / args.steps
+    if int(status[0]) != 0:
+        raise RuntimeError(f"kernel status word reports a timeout: {status.tolist()}")
+
+    # ---- the attend kernel alone (roofline of the dominant kernel) ----
+    phase_ms = {1: [], 2: [], 3: []}
+    if not write:
+        n_rep = max(3, min(args.steps, 200))
+        for i in range(n_rep + 3):
+            flush.zero_()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            ev[0].record(stream)
+            for ph in (1, 2, 3):
+                shla.mla_decode_phase(ph, wl.q_nope, wl.q_pe, wl.wkv_b, wl.cache, wl.topk,
+                                      wl.end_pos, wl.scale, out, ws, status)
+                ev[ph].record(stream)
+            torch.cuda.synchronize()
+            if i >= 3:
+                for ph in (1, 2, 3):
+                    phase_ms[ph].append(ev[ph - 1].elapsed_time(ev[ph]))
+    peaks = load_peaks()
+    roofline = None
+    if phase_ms[2]:
+        core_ms = reduce_max(statistics.mean(phase_ms[2]), world, dev)
+        cb, cf = core_kernel_work(B, k)
+        achieved = cb / (core_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": achieved / peaks["hbm_gbs"], "traffic": profiled_traffic(),
+                    "kernel": "core_kernel (gather + QK^T + softmax + PV)",
+                    "kernel_us": core_ms * 1e3,
+                    "tensor_tflops": cf / (core_ms * 1e-3) / 1e12,
+                    "tensor_frac_of_bf16_peak": cf / (core_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                    "peak_source": peaks["source"] + " (burst copy)",
+                    "phase_us": {"fold": 1e3 * statistics.mean(phase_ms[1]),
+                                 "attend": 1e3 * statistics.mean(phase_ms[2]),
+                                 "merge_uv": 1e3 * statistics.mean(phase_ms[3])}}
+
+    # ---- end to end through the public API with host buffers ----
+    h_qn = wl.q_nope.cpu().pin_memory()
+    h_qp = wl.q_pe.cpu().pin_memory()
+    h_ix = wl.topk.cpu().pin_memory()
+    h_ep = wl.end_pos.cpu().pin_memory()
+    h_out = torch.empty(B, HEADS, 128, dtype=torch.bfloat16).pin_memory()
+    d_qn, d_qp = torch.empty_like(wl.q_nope), torch.empty_like(wl.q_pe)
+    d_ix, d_ep = torch.empty_like(wl.topk), torch.empty_like(wl.end_pos)
+    h2d = sum(t.numel() * t.element_size() for t in (h_qn, h_qp, h_ix, h_ep))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        d_qn.copy_(h_qn, non_blocking=True)
+        d_qp.copy_(h_qp, non_blocking=True)
+        d_ix.copy_(h_ix, non_blocking=True)
+        d_ep.copy_(h_ep, non_blocking=True)
+        if write:
+            shla.mla_cache_write(wl.x, wl.w_kva, wl.norm_w, wl.eps, tab, wl.write_pos, wl.cache,
+                                 ws=cw_ws)
+        shla.mla_decode(d_qn, d_qp, wl.wkv_b, wl.cache, d_ix, d_ep, wl.scale, out=out, ws=ws)
+        h_out.copy_(out, non_blocking=True)
+
+    n_e2e = max(3, min(args.steps, 200))
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e_ms = 0.0
+    for _ in range(n_e2e):
+        flush.zero_()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_step()
+        b_.record(stream)
+        torch.cuda.synchronize()
+        e_ms += a.elapsed_time(b_)
+    e_ms = reduce_max(e_ms / n_e2e, world, dev)
+
+    units = B * k * HEADS
+    value = world * units / (ms_per_step * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "us_per_step": ms_per_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded, distributions of the workload; no public dataset involved)",
+        "config": workload_config(args.config, world),
+        "roofline": roofline,
+        "e2e": {"value": world * units / (e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
+                "what": "H2D of q_nope, q_pe, top-k, end_pos from pinned host memory, "
+                        "mla_decode, D2H of O; cache and weights resident"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "algorithmic": dict(zip(("bytes_per_step", "flops_per_step"), algorithmic_work(B, k))),
+    }
+    # ---- CPU baseline: the oracle on a bounded sample, rank 0 at N=1 ----
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        rows = list(range(min(args.cpu_rows, B)))
+        rate, dt, threads = oracle_sample_rate(wl, rows)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": f"{len(rows)} of {B} batch rows (their selected rows "
+                                          f"only), one pass, {dt:.1f} s"}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", type=int, default=3, choices=[0, 1, 2, 3, 4])
+    ap.add_argument("--cpu-rows", type=int, default=128)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

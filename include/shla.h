@@ -1,0 +1,200 @@
+/*
+ * libshla -- absorbed sparse multi-head latent attention decode for B200
+ * (sm_100a): the decode step of DeepSeek-V3.2-Exp's sparse latent attention,
+ * with W_UK folded into the queries and W_UV applied after the latent mix.
+ *
+ * C ABI.  All tensor arguments are DEVICE pointers owned by the caller; the
+ * library never allocates, frees or keeps per-call state, and it keeps no
+ * pointer after a call returns.  Every compute entry point only enqueues work
+ * on the given CUDA stream (``stream`` is a cudaStream_t; NULL = legacy
+ * default stream) and returns at once.
+ *
+ * Element types:
+ *   bf16  = 16-bit brain float, passed as raw bits (mla_bf16_t)
+ *   fp32  = IEEE float
+ *   int32 = int32_t
+ * All arrays are row-major.  Unless a stride argument says otherwise, they are
+ * contiguous.  Base pointers and row strides of every bf16/fp32 array must be
+ * 16-byte aligned (MLA_ERR_ALIGN otherwise).
+ *
+ * Model dimensions are fixed ("Key heads" page, MLA init listing; "KV
+ * compression" page):
+ *   H  = 128 heads
+ *   C  = 512 latent width (kv_lora_rank)
+ *   R  = 64 shared rotary key width (qk_rope_head_dim)
+ *   Dn = 128 non-rotary query/key width, Dv = 128 value width
+ *   DIM = 7168 model width
+ *
+ * Return value: MLA_OK (0), or a negative MLA_ERR_* code for a synchronous
+ * error found before anything was enqueued.  Asynchronous conditions go into
+ * an optional caller-owned device int32 status[2]:
+ *   status[0] |= MLA_STATUS_TIMEOUT  if a kernel gave up a bounded wait (the
+ *                                    output is then undefined);
+ *   status[1] += count of top-k entries that are neither -1 nor inside
+ *                [0, min(end_pos[b], T)) (they are ignored).
+ * The library never clears the status word.
+ */
+#ifndef SHLA_H_
+#define SHLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t mla_bf16_t;
+
+enum {
+  MLA_OK = 0,
+  MLA_ERR_NULL = -1,        /* a required pointer is NULL */
+  MLA_ERR_SHAPE = -2,       /* a size or stride is out of range */
+  MLA_ERR_ALIGN = -3,       /* a pointer or stride breaks 16-byte alignment */
+  MLA_ERR_WORKSPACE = -4,   /* workspace pointer NULL or too small */
+  MLA_ERR_UNSUPPORTED = -5, /* device is not sm_100 */
+  MLA_ERR_CUDA = -6         /* a CUDA launch or attribute call failed */
+};
+
+#define MLA_STATUS_TIMEOUT 1
+
+#define MLA_HEADS 128
+#define MLA_LATENT 512
+#define MLA_ROPE 64
+#define MLA_NOPE 128
+#define MLA_VDIM 128
+#define MLA_ROW 576
+#define MLA_DIM 7168
+
+/* Human-readable text for a return code.  Static storage; never NULL. */
+const char* mla_status_string(int code);
+
+/*
+ * Rotary embedding of feature pairs ("Rotated shared key" page,
+ * apply_rotary_emb, model.py 405-425).
+ *   x    bf16  [B, S, Hx, 64]
+ *   rope fp32  [S, 32, 2]: (cos, sin) of the angle for sequence slot s and
+ *              pair j; slot s of x uses row s (the caller offsets the table to
+ *              the first position)
+ *   interleaved != 0: pair j = (x[2j], x[2j+1]); result written back to
+ *              (2j, 2j+1).  interleaved == 0: pair j = (x[j], x[j+32]); result
+ *              written as all real parts then all imaginary parts.
+ *   y    bf16  [B, S, Hx, 64]; may equal x (in place)
+ * Rotation in fp32, one rounding to bf16.
+ */
+int mla_rope(const mla_bf16_t* x, const float* rope, int B, int S, int Hx, int interleaved,
+             mla_bf16_t* y, void* stream);
+
+/*
+ * Cache write for new positions ("KV compression" page, model.py 565-568,
+ * and the cache write of 576 values per position, model.py 572-573):
+ *   kv = x W_KVa (fp32 accumulation); latent = RMSNorm(kv[0:512]) * norm_w
+ *   (y = v / sqrt(mean(v^2) + eps) * w, fp32); k_pe = interleaved RoPE of
+ *   kv[512:576] at the row's position; both stored as bf16.
+ *   x       bf16 [B, S, 7168]
+ *   w_kva   bf16 [7168, 576]   (x W form: row i holds input feature i)
+ *   norm_w  bf16 [512]
+ *   rope    fp32 [S, 32, 2]    coefficients of positions start_pos .. start_pos+S-1
+ *   c_kv    bf16 latent cache: element (b, t, c) at c_kv[b*ckv_bstride + t*ckv_rstride + c]
+ *   k_pe    bf16 rotary cache: element (b, t, r) at k_pe[b*kpe_bstride + t*kpe_rstride + r]
+ *           (fused [B, T, 576] rows: k_pe = c_kv + 512, both rstrides 576)
+ *   T       cache capacity; requires 0 <= start_pos, start_pos + S <= T
+ *   ws      device workspace of at least mla_cache_write_workspace_bytes(B*S)
+ *           bytes, 256-byte aligned; contents need not be initialised
+ * Requires 1 <= B*S <= 4096.
+ */
+size_t mla_cache_write_workspace_bytes(int rows);
+int mla_cache_write(const mla_bf16_t* x, const mla_bf16_t* w_kva, const mla_bf16_t* norm_w,
+                    float eps, const float* rope, int B, int S, int start_pos,
+                    mla_bf16_t* c_kv, int64_t ckv_bstride, int ckv_rstride,
+                    mla_bf16_t* k_pe, int64_t kpe_bstride, int kpe_rstride, int T,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Absorbed sparse decode, one query per batch row ("Mix and project" page,
+ * decode branch, model.py 590-606):
+ *   q~[b,h,:]  = q_nope[b,h,:] W_UK[h]            W_UK[h] = wkv_b[h, 0:128, :]
+ *   s[b,h,t]   = (q~[b,h,:].c_KV[b,t,:] + q_pe[b,h,:].k_pe[b,t,:]) * scale
+ *                for t in the selected set of row b
+ *   A          = softmax_t(s)
+ *   O~[b,h,:]  = sum_t A[b,h,t] c_KV[b,t,:]
+ *   O[b,h,:]   = W_UV[h] O~[b,h,:]                W_UV[h] = wkv_b[h, 128:256, :]
+ * The selected set of row b is the set of distinct entries of topk[b, :]
+ * inside [0, min(end_pos[b], T)); -1 entries are padding.  Other entries are
+ * ignored and counted in status[1].  A row with an empty set gets O = 0.
+ *   q_nope  bf16 [B, 128, 128]
+ *   q_pe    bf16 [B, 128, 64]   (already rotated)
+ *   wkv_b   bf16 [128, 256, 512] ([out, in] storage of the 512 -> 128*256 projection)
+ *   c_kv, k_pe, strides, T: cache as in mla_cache_write (read only)
+ *   topk    int32 [B, k]   entries of a row must be distinct (besides -1)
+ *   end_pos int32 [B]
+ *   scale   softmax scale (192^-0.5 * mscale^2 in the model)
+ *   O       bf16 [B, 128, 128]
+ *   ws      device workspace of at least mla_decode_workspace_bytes(B, k) bytes,
+ *           256-byte aligned; contents need not be initialised
+ *   status  optional int32[2] (see top of file), may be NULL
+ * Requires 1 <= B <= 65535 and 1 <= k <= 65536; scores, softmax and
+ * accumulations are fp32; q~, the softmax weights and per-split partial
+ * outputs are rounded to bf16 as tensor-core operands.
+ */
+size_t mla_decode_workspace_bytes(int B, int k);
+int mla_decode(const mla_bf16_t* q_nope, const mla_bf16_t* q_pe, const mla_bf16_t* wkv_b,
+               const mla_bf16_t* c_kv, int64_t ckv_bstride, int ckv_rstride,
+               const mla_bf16_t* k_pe, int64_t kpe_bstride, int kpe_rstride, int T,
+               const int32_t* topk, int k, const int32_t* end_pos, int B, float scale,
+               mla_bf16_t* O, void* ws, size_t ws_bytes, int32_t* status, void* stream);
+
+/*
+ * The same call split into its three launches, for timing one of them alone:
+ *   phase 1: fold of W_UK into the queries (writes q~ into ws)
+ *   phase 2: gather + scores + softmax + latent mix per key split (reads q~,
+ *            writes the per-split partial outputs into ws)
+ *   phase 3: merge of the splits and W_UV (reads ws, writes O)
+ *   phase 0: all three (identical to mla_decode)
+ * Phases must run in order on one stream with the same arguments and
+ * workspace; each phase alone leaves O undefined until phase 3 has run.
+ */
+int mla_decode_phase(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_pe,
+                     const mla_bf16_t* wkv_b, const mla_bf16_t* c_kv, int64_t ckv_bstride,
+                     int ckv_rstride, const mla_bf16_t* k_pe, int64_t kpe_bstride,
+                     int kpe_rstride, int T, const int32_t* topk, int k, const int32_t* end_pos,
+                     int B, float scale, mla_bf16_t* O, void* ws, size_t ws_bytes,
+                     int32_t* status, void* stream);
+
+/*
+ * Fold of W_UK into the queries, the first step of mla_decode ("Mix and
+ * project" page, decode branch: einsum bshd,hdc->bshc):
+ *   q_tilde[b,h,c] = sum_d q_nope[b,h,d] wkv_b[h,d,c]     bf16 [B, 128, 512]
+ * fp32 accumulation, one rounding to bf16.  Requires 1 <= B <= 65535.
+ */
+int mla_fold_wuk(const mla_bf16_t* q_nope, const mla_bf16_t* wkv_b, int B,
+                 mla_bf16_t* q_tilde, void* stream);
+
+/*
+ * Test hook: the decode index mask ("Mix and project" page, decode branch:
+ * a -inf row over [0, end_pos) with the indexer's positions scattered to 0).
+ *   mask uint8 [B, T]: 1 where t is listed in topk[b] and t < end_pos[b], else 0.
+ * Invalid entries are counted in status[1] (status may be NULL).
+ */
+int mla_index_mask(const int32_t* topk, int B, int k, const int32_t* end_pos, int T,
+                   uint8_t* mask, int32_t* status, void* stream);
+
+/*
+ * Test hook: the row gather of mla_decode.  rows[b, j, :] = the 576 cached
+ * values (latent then rotary key) of position topk[b, j], or zeros when the
+ * entry is -1 or invalid (invalid ones are counted in status[1]).
+ *   rows bf16 [B, k, 576]
+ */
+int mla_gather_rows(const mla_bf16_t* c_kv, int64_t ckv_bstride, int ckv_rstride,
+                    const mla_bf16_t* k_pe, int64_t kpe_bstride, int kpe_rstride, int T,
+                    const int32_t* topk, int B, int k, const int32_t* end_pos,
+                    mla_bf16_t* rows, int32_t* status, void* stream);
+
+/* Number of key splits mla_decode uses for (B, k) on the current device. */
+int mla_decode_num_splits(int B, int k);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SHLA_H_ */

@@ -1,0 +1,279 @@
+"""CUDA path (through the C ABI) against the float64 oracle on identical
+seeded inputs.
+
+Tolerances: decode output O (bf16) -- relative L2 error <= 1e-2 and max-abs
+error <= 2e-2; index masks and gathered rows -- bit-exact; rope and cache
+write -- every element within one bf16 rounding of the exact value (plus a
+tiny fp32 allowance).
+"""
+import numpy as np
+import pytest
+import torch
+
+import mla_inputs as mi
+import oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 1e-2
+MAX_ABS = 2e-2
+
+
+@pytest.fixture(scope="module")
+def shla():
+    import sparse_head_latent_absorbed_b200 as m
+    return m
+
+
+def _rel(a, b):
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def _check_O(gpu, ref, what=""):
+    g = gpu.float().cpu().numpy().astype(np.float64)
+    assert np.isfinite(g).all(), what
+    rel = _rel(g, ref)
+    mx = float(np.abs(g - ref).max())
+    assert rel <= REL_L2, f"{what} rel-L2 {rel:.3e}"
+    assert mx <= MAX_ABS, f"{what} max-abs {mx:.3e}"
+    return rel, mx
+
+
+def _oracle_decode(wl, rows=None):
+    rows = range(wl.B) if rows is None else rows
+    rows = list(rows)
+    cache = mi.f64(wl.cache[rows])
+    return orc.decode_absorbed(mi.f64(wl.q_nope[rows]), mi.f64(wl.q_pe[rows]), mi.f64(wl.wkv_b),
+                               cache[..., :512], cache[..., 512:],
+                               wl.topk[rows].cpu().numpy(), wl.end_pos[rows].cpu().numpy(),
+                               wl.scale)
+
+
+def _oracle_decode_compact(wl, b, override=None):
+    """Oracle on the selected rows of batch row b only (the cache itself is
+    too large for the host at the biggest workloads).  ``override`` maps a
+    position to a replacement row (float64 [576])."""
+    rows, keep = mi.compact_rows(wl, b)
+    r = mi.f64(rows)
+    if override:
+        for i, t in enumerate(keep):
+            if t in override:
+                r[i] = override[t]
+    n = len(keep)
+    return orc.decode_absorbed(mi.f64(wl.q_nope[b:b + 1]), mi.f64(wl.q_pe[b:b + 1]),
+                               mi.f64(wl.wkv_b), r[None, :, :512], r[None, :, 512:],
+                               np.arange(n)[None, :], np.array([n]), wl.scale)[0]
+
+
+# ---------------------------------------------------------------------------
+# boundary ops
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("interleaved", [True, False])
+@pytest.mark.parametrize("Hx", [1, 128])
+def test_rope(shla, interleaved, Hx):
+    x = mi.make_rope_input(B=3, S=7, Hx=Hx, seed=Hx, device="cuda")
+    tab = mi.rope_table(4096)[4000:4007].contiguous().cuda()
+    y = shla.mla_rope(x, tab, interleaved)
+    ref = orc.rope(mi.f64(x), mi.rope_complex(tab), interleaved)
+    g = mi.f64(y)
+    err = np.abs(g - ref)
+    assert np.all(err <= np.abs(ref) * 2.0 ** -8 + 1e-6 * np.abs(mi.f64(x)).max()), err.max()
+    # in place gives the same bits
+    x2 = x.clone()
+    shla.mla_rope(x2, tab, interleaved, out=x2)
+    assert torch.equal(x2, y)
+
+
+def test_rope_position_zero_is_identity(shla):
+    x = mi.make_rope_input(B=2, S=1, Hx=128, seed=5, device="cuda")
+    tab = mi.rope_table(1).cuda()
+    assert torch.equal(shla.mla_rope(x, tab, True), x)
+
+
+def test_index_mask_bit_exact(shla):
+    wl = mi.make_small(B=4, T=257, k=150, seed=1, n_pad=5, n_invalid=4, dup=3, device="cuda")
+    status = torch.zeros(2, dtype=torch.int32, device="cuda")
+    mask = shla.mla_index_mask(wl.topk, wl.end_pos, wl.T, status=status)
+    ref, bad = orc.index_mask(wl.topk.cpu().numpy(), wl.end_pos.cpu().numpy(), wl.T)
+    assert np.array_equal(mask.cpu().numpy(), ref)
+    assert int(status[1]) == bad and int(status[0]) == 0
+
+
+def test_gather_rows_bit_exact(shla):
+    wl = mi.make_small(B=3, T=200, k=90, seed=2, n_pad=3, n_invalid=2, device="cuda")
+    status = torch.zeros(2, dtype=torch.int32, device="cuda")
+    rows = shla.mla_gather_rows(wl.cache, wl.topk, wl.end_pos, status=status).cpu()
+    cache = wl.cache.cpu()
+    bad = 0
+    for b in range(wl.B):
+        ep = int(wl.end_pos[b])
+        for j, v in enumerate(wl.topk[b].tolist()):
+            if 0 <= v < min(ep, wl.T):
+                assert torch.equal(rows[b, j], cache[b, v])
+            else:
+                assert torch.all(rows[b, j] == 0)
+                bad += v != -1
+    assert int(status[1]) == bad
+
+
+@pytest.mark.parametrize("B", [1, 5, 40, 300])
+def test_fold_wuk(shla, B):
+    g = torch.Generator(device="cuda").manual_seed(B)
+    q = torch.randn(B, 128, 128, generator=g, device="cuda").bfloat16()
+    w = (torch.randn(128, 256, 512, generator=g, device="cuda") / 512 ** 0.5).bfloat16()
+    out = shla.mla_fold_wuk(q, w)
+    ref = orc.fold_wuk(mi.f64(q), mi.f64(w))
+    g64 = mi.f64(out)
+    assert _rel(g64, ref) < 4e-3
+    assert np.all(np.abs(g64 - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-3)
+
+
+# ---------------------------------------------------------------------------
+# decode
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("B,T,k,seed", [
+    (1, 64, 1, 0), (1, 64, 63, 1), (2, 128, 64, 2), (2, 300, 65, 3),
+    (3, 300, 130, 4), (5, 1000, 333, 5), (2, 4096, 2048, 6), (17, 700, 450, 7),
+])
+def test_decode_small(shla, B, T, k, seed):
+    wl = mi.make_small(B=B, T=T, k=k, seed=seed, device="cuda")
+    status = torch.zeros(2, dtype=torch.int32, device="cuda")
+    out = shla.mla_decode(wl.q_nope, wl.q_pe, wl.wkv_b, wl.cache, wl.topk, wl.end_pos,
+                          wl.scale, status=status)
+    torch.cuda.synchronize()
+    assert int(status[0]) == 0
+    _check_O(out, _oracle_decode(wl), f"B={B} T={T} k={k}")
+
+
+def test_decode_padding_invalid_duplicate_free(shla):
+    wl = mi.make_small(B=4, T=500, k=200, seed=11, n_pad=17, n_invalid=9, device="cuda")
+    status = torch.zeros(2, dtype=torch.int32, device="cuda")
+    out = shla.mla_decode(wl.q_nope, wl.q_pe, wl.wkv_b, wl.cache, wl.topk, wl.end_pos,
+                          wl.scale, status=status)
+    _, bad = orc.index_mask(wl.topk.cpu().numpy(), wl.end_pos.cpu().numpy(), wl.T)
+    torch.cuda.synchronize()
+    assert int(status[0]) == 0 and int(status[1]) == bad
+    _check_O(out, _oracle_decode(wl))
+
+
+def test_decode_empty_selection_gives_zero(shla):
+    wl = mi.make_small(B=3, T=100, k=70, seed=12, device="cuda")
+    wl.topk[1] = -1
+    out = shla.mla_decode(wl.q_nope, wl.q_pe, wl.wkv_b, wl.cache, wl.topk, wl.end_pos, wl.scale)
+    assert torch.all(out[1] == 0)
+    _check_O(out, _oracle_decode(wl))
+
+
+def test_decode_zero_query_uniform(shla):
+    wl = mi.make_small(B=2, T=300, k=150, seed=13, q_zero=True, device="cuda")
+    out = shla.mla_decode(wl.q_nope, wl.q_pe, wl.wkv_b, wl.cache, wl.topk, wl.end_pos, wl.scale)
+    _check_O(out, _oracle_decode(wl))
+
+
+def test_decode_large_scores_trigger_rescaling(shla):
+    """A large softmax scale makes the running maximum grow across tiles."""
+    wl = mi.make_small(B=2, T=2000, k=1500, seed=14, device="cuda")
+    out = shla.mla_decode(wl.q_nope, wl.q_pe, wl.wkv_b, wl.cache, wl.topk, wl.end_pos, 0.4)
+    wl.scale = 0.4
+    _check_O(out, _oracle_decode(wl))
+
+
+def test_decode_deterministic_and_canaries(shla):
+    wl = mi.make_small(B=6, T=1500, k=777, seed=15, device="cuda")
+    B = wl.B
+    buf = torch.full((B + 2, 128, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    out = buf[1:B + 1]
+    first = None
+    for _ in range(20):
+        shla.mla_decode(wl.q_nope, wl.q_pe, wl.wkv_b, wl.cache, wl.topk, wl.end_pos, wl.scale,
+                        out=out)
+        if first is None:
+            first = out.clone()
+        else:
+            assert torch.equal(out, first)
+    assert torch.all(buf[0] == 7.0) and torch.all(buf[B + 1] == 7.0)
+
+
+def test_decode_strided_cache_view(shla):
+    """Cache rows padded to 640 elements (strides passed through the ABI)."""
+    wl = mi.make_small(B=2, T=256, k=100, seed=16, device="cuda")
+    big = torch.zeros(2, 256, 640, dtype=torch.bfloat16, device="cuda")
+    big[..., :576] = wl.cache
+    view = big[..., :576]
+    out = shla.mla_decode(wl.q_nope, wl.q_pe, wl.wkv_b, view, wl.topk, wl.end_pos, wl.scale)
+    _check_O(out, _oracle_decode(wl))
+
+
+# ---------------------------------------------------------------------------
+# the five workloads at full size (sampled rows where the oracle needs it)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("cid,sample", [(0, None), (1, None), (2, [0, 17, 40, 63]),
+                                        (3, [0, 31, 64, 101, 127])])
+def test_decode_workloads(shla, cid, sample):
+    wl = mi.make_config(cid, device="cuda")
+    status = torch.zeros(2, dtype=torch.int32, device="cuda")
+    out = shla.mla_decode(wl.q_nope, wl.q_pe, wl.wkv_b, wl.cache, wl.topk, wl.end_pos,
+                          wl.scale, status=status)
+    torch.cuda.synchronize()
+    assert int(status[0]) == 0 and int(status[1]) == 0
+    if sample is None:
+        _check_O(out, _oracle_decode(wl), f"config {cid}")
+    else:
+        for b in sample:
+            _check_O(out[b:b + 1], _oracle_decode_compact(wl, b)[None], f"config {cid} b={b}")
+    del wl
+    torch.cuda.empty_cache()
+
+
+def test_cache_write_then_decode_workload(shla):
+    """Cache write of 32 rows at position 65535, then top-k decode over 65536
+    positions that always include the fresh row."""
+    wl = mi.make_config(4, device="cuda")
+    wp = wl.write_pos
+    sample = [0, 9, 31]
+    before = {b: mi.compact_rows(wl, b) for b in sample}  # inputs, taken before the write
+    tab = wl.rope[wp:wp + 1].contiguous()
+    guard_prev = wl.cache[:, wp - 1].clone()
+    shla.mla_cache_write(wl.x, wl.w_kva, wl.norm_w, wl.eps, tab, wp, wl.cache)
+    out = shla.mla_decode(wl.q_nope, wl.q_pe, wl.wkv_b, wl.cache, wl.topk, wl.end_pos, wl.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(wl.cache[:, wp - 1], guard_prev)
+    lat, pe = orc.cache_write(mi.f64(wl.x), mi.f64(wl.w_kva), mi.f64(wl.norm_w), wl.eps,
+                              np.repeat(mi.rope_complex(tab), wl.B, 0), 512)
+    exact = np.concatenate([lat, pe], 1)
+    got = mi.f64(wl.cache[:, wp])
+    assert np.all(np.abs(got - exact) <= np.abs(exact) * 2.0 ** -7 + 1e-4)
+    stored = torch.from_numpy(exact).to(torch.bfloat16).double().numpy()  # the cache is bf16
+    for b in sample:
+        rows, keep = before[b]
+        r = mi.f64(rows)
+        r[keep.index(wp)] = stored[b]
+        n = len(keep)
+        ref = orc.decode_absorbed(mi.f64(wl.q_nope[b:b + 1]), mi.f64(wl.q_pe[b:b + 1]),
+                                  mi.f64(wl.wkv_b), r[None, :, :512], r[None, :, 512:],
+                                  np.arange(n)[None], np.array([n]), wl.scale)
+        _check_O(out[b:b + 1], ref, f"config 4 b={b}")
+
+
+@pytest.mark.parametrize("rows,S,norm_ones", [(1, 1, True), (32, 1, True), (5, 3, False),
+                                              (300, 1, False)])
+def test_cache_write(shla, rows, S, norm_ones):
+    B = rows
+    T = 40
+    x, w, nw, tab, _ = mi.make_cache_write(rows=B * S, T=T, seed=rows, device="cuda",
+                                           norm_w_ones=norm_ones)
+    x = x.view(B, S, -1)
+    cache = torch.full((B, T, 576), 3.0, dtype=torch.bfloat16, device="cuda")
+    start = 20
+    shla.mla_cache_write(x, w, nw, 1e-6, tab[start:start + S].contiguous(), start, cache)
+    R = mi.rope_complex(tab[start:start + S])
+    lat, pe = orc.cache_write(mi.f64(x.reshape(B * S, -1)), mi.f64(w), mi.f64(nw), 1e-6,
+                              np.tile(R, (B, 1)), 512)
+    exact = np.concatenate([lat, pe], 1).reshape(B, S, 576)
+    got = mi.f64(cache[:, start:start + S])
+    assert np.all(np.abs(got - exact) <= np.abs(exact) * 2.0 ** -7 + 1e-4)
+    untouched = torch.cat([cache[:, :start], cache[:, start + S:]], 1)
+    assert torch.all(untouched == 3.0)
