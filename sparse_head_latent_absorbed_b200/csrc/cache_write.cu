@@ -56,17 +56,18 @@ __global__ void __launch_bounds__(128) cw_gemm_kernel(const __nv_bfloat16* __res
   for (int q = tid; q < KCH * 16; q += 128) {
     const int i = q >> 4, ch = q & 15;
     const int o = mt * 128 + ch * 8;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (o < kOut) v = ld_global_nc_v4(w + (size_t)(kc * KCH + i) * kOut + o);
-    st_shared_v4(sA + (ch >> 3) * 32768 + sw128_off(i, ch & 7), v.x, v.y, v.z, v.w);
+    const bool in = o < kOut;
+    cp_async_16(sA + (ch >> 3) * 32768 + sw128_off(i, ch & 7),
+                w + (size_t)(kc * KCH + i) * kOut + (in ? o : 0), in ? 16u : 0u);
   }
   // B: x[r0 + n][kc*256 + 8*ch .. +8]
   for (int q = tid; q < NB * 32; q += 128) {
     const int n = q >> 5, ch = q & 31, r = r0 + n;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r < rows) v = ld_global_nc_v4(x + (size_t)r * kDim + kc * KCH + ch * 8);
-    st_shared_v4(sB + (ch >> 3) * (NB * 128) + sw128_off(n, ch & 7), v.x, v.y, v.z, v.w);
+    const bool in = r < rows;
+    cp_async_16(sB + (ch >> 3) * (NB * 128) + sw128_off(n, ch & 7),
+                x + (size_t)(in ? r : 0) * kDim + kc * KCH + ch * 8, in ? 16u : 0u);
   }
+  cp_async_wait_all();
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();

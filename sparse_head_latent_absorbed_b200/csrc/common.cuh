@@ -93,6 +93,26 @@ DEV bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// non-blocking test of a phase (acquire, CTA scope)
+DEV bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// one arrival that also raises the phase's expected transaction bytes
+DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
 // Bounded wait for the phase with the given parity to complete.  Returns
 // false (after flagging ``*abort`` and the status word) when the limit
 // expires or when another thread of the CTA has already aborted.
@@ -138,6 +158,16 @@ DEV uint32_t mapa_shared(uint32_t local_addr, uint32_t rank) {
   return r;
 }
 
+// 16-byte store into another CTA's shared memory that counts its bytes
+// against that CTA's mbarrier (complete_tx); no fence needed on either side
+DEV void st_async_v4(uint32_t addr, float a, float b, float c, float d, uint32_t remote_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::
+          "r"(addr),
+      "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
+      : "memory");
+}
+
 DEV void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
   asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
                "f"(c), "f"(d)
@@ -156,6 +186,13 @@ DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;
 DEV void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
                "r"(src_bytes)
+               : "memory");
+}
+DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// arrive on ``bar`` once all cp.async copies issued so far by this thread
+// have landed (counts as one of the barrier's expected arrivals)
+DEV void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
 }
 DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
@@ -269,6 +306,13 @@ DEV uint32_t sw128_off(uint32_t row, uint32_t chunk) {
 // 512-byte aligned).
 DEV uint32_t sw64_off(uint32_t row, uint32_t chunk) {
   return row * 64u + ((chunk ^ ((row >> 1) & 3u)) << 4);
+}
+
+// 2^x on the special-function unit (inputs are <= 0 or -inf here)
+DEV float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 DEV uint32_t pack_bf16x2(float lo, float hi) {

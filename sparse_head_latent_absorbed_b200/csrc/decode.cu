@@ -55,15 +55,16 @@ __global__ void __launch_bounds__(128) fold_kernel(const __nv_bfloat16* __restri
   }
   for (int q = tid; q < 128 * 16; q += 128) {
     const int d = q >> 4, ch = q & 15;
-    const uint4 v = ld_global_nc_v4(wkv_b + ((size_t)h * 256 + d) * kC + ct * 128 + ch * 8);
-    st_shared_v4(sA + (ch >> 3) * 16384 + sw128_off(d, ch & 7), v.x, v.y, v.z, v.w);
+    cp_async_16(sA + (ch >> 3) * 16384 + sw128_off(d, ch & 7),
+                wkv_b + ((size_t)h * 256 + d) * kC + ct * 128 + ch * 8, 16);
   }
   for (int q = tid; q < NB * 16; q += 128) {
     const int n = q >> 4, ch = q & 15, b = b0 + n;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (b < B) v = ld_global_nc_v4(q_nope + ((size_t)b * kH + h) * kDn + ch * 8);
-    st_shared_v4(sB + (ch >> 3) * (NB * 128) + sw128_off(n, ch & 7), v.x, v.y, v.z, v.w);
+    const bool in = b < B;
+    cp_async_16(sB + (ch >> 3) * (NB * 128) + sw128_off(n, ch & 7),
+                q_nope + ((size_t)(in ? b : 0) * kH + h) * kDn + ch * 8, in ? 16u : 0u);
   }
+  cp_async_wait_all();
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -108,23 +109,42 @@ __global__ void __launch_bounds__(128) fold_kernel(const __nv_bfloat16* __restri
 
 // ===========================================================================
 // K2: sparse attention core on a 2-CTA cluster
+//
+// Warp roles per CTA (288 threads):
+//   warps 0-3  softmax: one thread per head row (TMEM lane); exchange of the
+//              partial score tile with the peer CTA through DSMEM, running
+//              max / sum, P (bf16) into shared memory, O rescaling
+//   warps 4-7  gather: cp.async of this CTA's 288 columns of each selected
+//              cache row into a NST-deep ring of key tiles
+//   warp 8     TMEM owner and MMA issuer (one thread)
+// Per key tile j (KT keys):  S_j = Q~_half K_j_half^T (M=128, N=KT, K=288)
+// into one of two TMEM score buffers; after the softmax, O_half += P_j V_j_half
+// (M=128, N=256, K=KT) where V is the same shared-memory tile read MN-major.
 // ===========================================================================
 namespace core {
-constexpr int KT = 64;                       // keys per tile
-constexpr int NST = 2;                       // gather stages
-constexpr int NTHREADS = 288;                // warps 0-3 softmax, 4-7 gather, 8 MMA
+constexpr int KT = 32;                       // keys per tile
+constexpr int NST = 6;                       // gather ring depth
+constexpr int NTHREADS = 288;
 constexpr int OFF_QC = 0;                    // Q~ latent half: 4 atoms x 128 rows x 128 B
 constexpr int OFF_QR = 65536;                // q_pe half: 128 rows x 64 B (64 B swizzle)
-constexpr int OFF_ST = 73728;                // stages
-constexpr int ST_KR = 32768;                 // offset of the rotary part inside a stage
-constexpr int ST_BYTES = 36864;              // 4 x 64 x 128 + 64 x 64
-constexpr int OFF_P = OFF_ST + NST * ST_BYTES;   // P: 128 rows x 128 B
-constexpr int OFF_XS = OFF_P + 16384;            // exchanged partial scores
-constexpr int XS_STRIDE = 272;                   // 64 fp32 + 16 B pad per row
-constexpr int OFF_END = OFF_XS + 128 * XS_STRIDE;
+constexpr int OFF_ST = 73728;                // key tiles
+constexpr int ST_ATOM = KT * 128;            // one 64-column latent atom of a tile
+constexpr int ST_KR = 4 * ST_ATOM;           // rotary part of a tile (64 B swizzle)
+constexpr int ST_BYTES = ST_KR + KT * 64;
+constexpr int OFF_P = OFF_ST + NST * ST_BYTES;   // P: 128 rows x KT bf16 (64 B swizzle)
+constexpr int P_BYTES = 128 * KT * 2;
+constexpr int OFF_XS = OFF_P + P_BYTES;          // two buffers of exchanged partial scores
+constexpr int XS_STRIDE = KT * 4 + 16;           // padded fp32 row
+constexpr int XS_BYTES = 128 * XS_STRIDE;
+constexpr int OFF_END = OFF_XS + 2 * XS_BYTES;
+constexpr uint32_t XS_TX_BYTES = 128 * KT * 4;   // partial scores received per tile
 constexpr int SMEM_BYTES = OFF_END + 1024;       // + alignment slack
-constexpr uint32_t TMEM_COLS = 512;              // S0 @0, S1 @64, O half @256
+constexpr uint32_t TMEM_COLS = 512;              // S0 @0, S1 @KT, O half @256
 constexpr float kRescaleThreshold = 8.0f;        // log2 units
+constexpr int PER_PRODUCER = KT * 36 / 128;      // 16-byte chunks per gather thread per tile
+static_assert(KT * 36 % 128 == 0, "gather split");
+static_assert(ST_BYTES % 1024 == 0 && OFF_ST % 1024 == 0 && OFF_P % 512 == 0, "alignment");
+static_assert(SMEM_BYTES + 256 <= 232448, "shared memory budget");
 
 struct Params {
   const __nv_bfloat16* q_tilde;   // [B][128][512]
@@ -147,7 +167,8 @@ struct Params {
 };
 
 struct Bars {
-  uint64_t full[NST], empty[NST], s_full[2], s_empty[2], p_full, o_done, xs_full, xs_free, drain;
+  uint64_t full[NST], empty[NST], s_full[2], s_empty[2], p_full, o_done, xs_full[2], xs_free[2],
+      drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -174,6 +195,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
   const int lim = min(p.end_pos[b], p.T);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sbase = smem_u32(smem);
+  const int32_t* topk_b = p.topk + (size_t)b * p.k;
 
   if (warp == 8) {
     tmem_alloc(&bars.tmem_base, TMEM_COLS);
@@ -187,27 +209,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.s_full[i], 1);
       mbar_init(&bars.s_empty[i], 128);
+      mbar_init(&bars.xs_full[i], 1);    // own expect_tx arrival + the peer's st.async bytes
+      mbar_init(&bars.xs_free[i], 4);    // one arrival per softmax warp of the peer
     }
     mbar_init(&bars.p_full, 128);
     mbar_init(&bars.o_done, 1);
-    mbar_init(&bars.xs_full, 128);
-    mbar_init(&bars.xs_free, 128);
     mbar_init(&bars.drain, 1);
     bars.abort = 0;
     fence_mbarrier_init_cluster();
+    // first use of each exchange buffer: expect one tile of partial scores
+    mbar_arrive_expect_tx(&bars.xs_full[0], XS_TX_BYTES);
+    mbar_arrive_expect_tx(&bars.xs_full[1], XS_TX_BYTES);
   }
-  // this CTA's half of Q~ (latent) and of q_pe (rotary), 16-byte chunks
+  // this CTA's half of Q~ (latent) and of q_pe (rotary)
   for (int q = tid; q < 128 * 36; q += NTHREADS) {
     const int h = q / 36, ch = q - h * 36;
-    if (ch < 32) {
-      const uint4 v = ld_global_nc_v4(p.q_tilde + ((size_t)b * kH + h) * kC + rank * 256 + ch * 8);
-      st_shared_v4(sbase + OFF_QC + (ch >> 3) * 16384 + sw128_off(h, ch & 7), v.x, v.y, v.z, v.w);
-    } else {
-      const uint4 v =
-          ld_global_nc_v4(p.q_pe + ((size_t)b * kH + h) * kR + rank * 32 + (ch - 32) * 8);
-      st_shared_v4(sbase + OFF_QR + sw64_off(h, ch - 32), v.x, v.y, v.z, v.w);
-    }
+    if (ch < 32)
+      cp_async_16(sbase + OFF_QC + (ch >> 3) * 16384 + sw128_off(h, ch & 7),
+                  p.q_tilde + ((size_t)b * kH + h) * kC + rank * 256 + ch * 8, 16);
+    else
+      cp_async_16(sbase + OFF_QR + sw64_off(h, ch - 32),
+                  p.q_pe + ((size_t)b * kH + h) * kR + rank * 32 + (ch - 32) * 8, 16);
   }
+  cp_async_wait_all();
   fence_proxy_async_smem();
   tc_fence_before();
   cluster_sync_all();
@@ -215,65 +239,79 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
   const uint32_t tmem = bars.tmem_base;
 
   if (warp >= 4 && warp < 8) {
-    // ---------------- gather producers ----------------
+    // ---------------- gather ----------------
     const int pt = tid - 128;
     int bad = 0;
     const __nv_bfloat16* ckv_b = p.c_kv + (size_t)b * p.ckv_bs + rank * 256;
     const __nv_bfloat16* kpe_b = p.k_pe + (size_t)b * p.kpe_bs + rank * 32;
-    const int32_t* topk_b = p.topk + (size_t)b * p.k;
+    int key[PER_PRODUCER], ch[PER_PRODUCER], v[PER_PRODUCER];
+#pragma unroll
+    for (int i = 0; i < PER_PRODUCER; ++i) {
+      const int q = pt + 128 * i;
+      key[i] = q / 36;
+      ch[i] = q - key[i] * 36;
+      const int j = tile0 * KT + key[i];
+      v[i] = j < p.k ? topk_b[j] : -1;
+    }
 #pragma unroll 1
     for (int jj = 0; jj < nt; ++jj) {
       const int s = jj % NST;
       if (!mbar_wait(&bars.empty[s], ((jj / NST) & 1) ^ 1, abort, p.status)) break;
-      const int kb = (tile0 + jj) * KT;
       const uint32_t stage = sbase + OFF_ST + s * ST_BYTES;
-#pragma unroll 2
-      for (int i = 0; i < 18; ++i) {
-        const int q = pt + 128 * i;
-        const int key = q / 36, ch = q - key * 36;
-        const int j = kb + key;
-        const int v = j < p.k ? topk_b[j] : -1;
-        const bool ok = key_valid(v, lim);
-        if (rank == 0 && ch == 0 && !ok && v != -1) ++bad;
-        const long long vv = ok ? v : 0;
+#pragma unroll
+      for (int i = 0; i < PER_PRODUCER; ++i) {
+        const bool ok = key_valid(v[i], lim);
+        if (rank == 0 && ch[i] == 0 && !ok && v[i] != -1) ++bad;
+        const long long vv = ok ? v[i] : 0;
         const void* src;
         uint32_t dst;
-        if (ch < 32) {
-          src = ckv_b + vv * p.ckv_rs + ch * 8;
-          dst = stage + (ch >> 3) * 8192 + sw128_off(key, ch & 7);
+        if (ch[i] < 32) {
+          src = ckv_b + vv * p.ckv_rs + ch[i] * 8;
+          dst = stage + (ch[i] >> 3) * ST_ATOM + sw128_off(key[i], ch[i] & 7);
         } else {
-          src = kpe_b + vv * p.kpe_rs + (ch - 32) * 8;
-          dst = stage + ST_KR + sw64_off(key, ch - 32);
+          src = kpe_b + vv * p.kpe_rs + (ch[i] - 32) * 8;
+          dst = stage + ST_KR + sw64_off(key[i], ch[i] - 32);
         }
         cp_async_16(dst, src, ok ? 16u : 0u);
       }
-      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
-                       smem_u32(&bars.full[s]))
-                   : "memory");
+      cp_async_arrive_noinc(&bars.full[s]);
+      // indices of the next tile, loaded while this one is in flight
+      if (jj + 1 < nt) {
+#pragma unroll
+        for (int i = 0; i < PER_PRODUCER; ++i) {
+          const int j = (tile0 + jj + 1) * KT + key[i];
+          v[i] = j < p.k ? topk_b[j] : -1;
+        }
+      }
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
+    cp_async_wait_all();
     if (bad && p.status) atomicAdd(p.status + 1, bad);
   } else if (warp == 8) {
     // ---------------- MMA issuer ----------------
+    // Event loop: a score tile is computed as soon as its keys have landed
+    // and a score buffer is free (up to two tiles ahead of the softmax); a
+    // value product as soon as its P is in shared memory.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, KT, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, 0, 1);
       const uint32_t qc = sbase + OFF_QC, qr = sbase + OFF_QR, pb = sbase + OFF_P;
-      bool alive = true;
+      int qk = 0, pv = 0, idle = 0;
+      uint64_t t_last = globaltimer_ns();
 #pragma unroll 1
-      for (int jj = 0; jj <= nt && alive; ++jj) {
-        if (jj < nt) {
-          const int s = jj % NST, b2 = jj & 1;
-          if (!mbar_wait(&bars.full[s], (jj / NST) & 1, abort, p.status)) break;
-          if (!mbar_wait(&bars.s_empty[b2], ((jj >> 1) & 1) ^ 1, abort, p.status)) break;
+      while (pv < nt) {
+        bool did = false;
+        if (qk < nt && mbar_test(&bars.full[qk % NST], (qk / NST) & 1) &&
+            mbar_test(&bars.s_empty[qk & 1], ((qk >> 1) & 1) ^ 1)) {
           fence_proxy_async_smem();
           tc_fence_after();
-          const uint32_t st = sbase + OFF_ST + s * ST_BYTES;
-          const uint32_t d = tmem + b2 * KT;
+          const uint32_t st = sbase + OFF_ST + (qk % NST) * ST_BYTES;
+          const uint32_t d = tmem + (qk & 1) * KT;
 #pragma unroll
           for (int ks = 0; ks < 16; ++ks) {
-            const uint64_t ad = smem_desc(qc + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSwizzle128B);
-            const uint64_t bd = smem_desc(st + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSwizzle128B);
+            const uint64_t ad =
+                smem_desc(qc + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSwizzle128B);
+            const uint64_t bd =
+                smem_desc(st + (ks >> 2) * ST_ATOM + (ks & 3) * 32, 16, 1024, kSwizzle128B);
             tc_mma(d, ad, bd, idesc_qk, ks > 0);
           }
 #pragma unroll
@@ -282,22 +320,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
             const uint64_t bd = smem_desc(st + ST_KR + ks * 32, 16, 512, kSwizzle64B);
             tc_mma(d, ad, bd, idesc_qk, 1);
           }
-          tc_commit(&bars.s_full[b2]);
+          tc_commit(&bars.s_full[qk & 1]);
+          ++qk;
+          did = true;
         }
-        if (jj >= 1) {
-          const int j = jj - 1, s = j % NST;
-          if (!mbar_wait(&bars.p_full, j & 1, abort, p.status)) break;
+        if (pv < qk && mbar_test(&bars.p_full, pv & 1)) {
           tc_fence_after();
+          const int s = pv % NST;
           const uint32_t st = sbase + OFF_ST + s * ST_BYTES;
 #pragma unroll
           for (int ks = 0; ks < KT / 16; ++ks) {
-            const uint64_t ad = smem_desc(pb + ks * 32, 16, 1024, kSwizzle128B);
-            const uint64_t bd = smem_desc(st + ks * 2048, 8192, 1024, kSwizzle128B);
-            tc_mma(tmem + 256, ad, bd, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
+            const uint64_t ad = smem_desc(pb + ks * 32, 16, 512, kSwizzle64B);
+            const uint64_t bd = smem_desc(st + ks * 2048, ST_ATOM, 1024, kSwizzle128B);
+            tc_mma(tmem + 256, ad, bd, idesc_pv, (pv > 0 || ks > 0) ? 1u : 0u);
           }
           tc_commit(&bars.o_done);
           tc_commit(&bars.empty[s]);
+          ++pv;
+          did = true;
         }
+        if (did) {
+          idle = 0;
+        } else if (++idle >= 64) {
+          idle = 0;
+          const uint64_t now = globaltimer_ns();
+          if (*abort) break;
+          if (now - t_last > kWaitLimitNs) {
+            *abort = 1;
+            report_timeout(p.status);
+            break;
+          }
+        }
+        if (did) t_last = globaltimer_ns();
       }
       // everything issued so far has finished before TMEM is released
       tc_commit(&bars.drain);
@@ -308,27 +362,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     // ---------------- softmax (one thread per head row) ----------------
     const int h = tid;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t xs_row = sbase + OFF_XS + h * XS_STRIDE;
-    const uint32_t xs_peer_row = mapa_shared(xs_row, peer);
-    const uint32_t xs_full_peer = mapa_shared(smem_u32(&bars.xs_full), peer);
-    const uint32_t xs_free_peer = mapa_shared(smem_u32(&bars.xs_free), peer);
+    // exchange buffer / barrier i sits at +i*XS_BYTES / +i*8 from buffer 0 in
+    // both CTAs, so the peer addresses follow from one mapa each
+    const uint32_t xs_row0 = sbase + OFF_XS + h * XS_STRIDE;
+    const uint32_t xs_peer_row0 = mapa_shared(xs_row0, peer);
+    const uint32_t xs_full_peer0 = mapa_shared(smem_u32(&bars.xs_full[0]), peer);
+    // (each exchange buffer's xs_full phase expects XS_TX_BYTES from the peer)
+    const uint32_t xs_free_peer0 = mapa_shared(smem_u32(&bars.xs_free[0]), peer);
     const uint32_t prow = sbase + OFF_P;
-    const int32_t* topk_b = p.topk + (size_t)b * p.k;
     float m_used = -INFINITY, l = 0.f;
+    float sn[KT];  // own partial scores of the tile after the current one
     bool alive = true;
-#pragma unroll 1
-    for (int jj = 0; jj < nt; ++jj) {
-      const int kb = (tile0 + jj) * KT;
-      const int j0 = kb + lane, j1 = kb + 32 + lane;
-      const int v0 = j0 < p.k ? topk_b[j0] : -1;
-      const int v1 = j1 < p.k ? topk_b[j1] : -1;
-      const uint32_t mlo = __ballot_sync(0xffffffffu, key_valid(v0, lim));
-      const uint32_t mhi = __ballot_sync(0xffffffffu, key_valid(v1, lim));
 
-      const int b2 = jj & 1;
-      if (!warp_wait(&bars.s_full[b2], (jj >> 1) & 1, abort, p.status)) { alive = false; break; }
+    // own partial of tile t: TMEM -> registers -> peer's exchange buffer
+    auto fetch_send = [&](int t) -> bool {
+      const int b2 = t & 1;
+      if (!warp_wait(&bars.s_full[b2], (t >> 1) & 1, abort, p.status)) return false;
       tc_fence_after();
-      float s[KT];
       {
         uint32_t r[16];
 #pragma unroll
@@ -336,37 +386,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
           tmem_ld16(tmem + lane_base + b2 * KT + c, r);
           tc_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) s[c + i] = __uint_as_float(r[i]);
+          for (int i = 0; i < 16; ++i) sn[c + i] = __uint_as_float(r[i]);
         }
       }
       tc_fence_before();
       mbar_arrive(&bars.s_empty[b2]);
-
-      // exchange partial scores with the peer CTA (other latent half)
-      if (!warp_wait<true>(&bars.xs_free, (jj & 1) ^ 1, abort, p.status)) { alive = false; break; }
+      if (!warp_wait<true>(&bars.xs_free[b2], ((t >> 1) & 1) ^ 1, abort, p.status)) return false;
 #pragma unroll
-      for (int i = 0; i < KT; i += 4) st_cluster_v4(xs_peer_row + i * 4, s[i], s[i + 1], s[i + 2], s[i + 3]);
-      mbar_arrive_cluster(xs_full_peer);
-      if (!warp_wait<true>(&bars.xs_full, jj & 1, abort, p.status)) { alive = false; break; }
+      for (int i = 0; i < KT; i += 4)
+        st_async_v4(xs_peer_row0 + b2 * XS_BYTES + i * 4, sn[i], sn[i + 1], sn[i + 2], sn[i + 3],
+                    xs_full_peer0 + b2 * 8);
+      return true;
+    };
+
+    int vpre = (tile0 * KT + lane < p.k) ? topk_b[tile0 * KT + lane] : -1;
+    alive = fetch_send(0);
+#pragma unroll 1
+    for (int jj = 0; jj < nt && alive; ++jj) {
+      const uint32_t valid = __ballot_sync(0xffffffffu, key_valid(vpre, lim));
+      if (jj + 1 < nt) {
+        const int j = (tile0 + jj + 1) * KT + lane;
+        vpre = j < p.k ? topk_b[j] : -1;
+      }
+      float s[KT];
+#pragma unroll
+      for (int i = 0; i < KT; ++i) s[i] = sn[i];
+      if (jj + 1 < nt && !fetch_send(jj + 1)) { alive = false; break; }
+
+      // add the peer's partial scores (other latent half) of this tile
+      const int b2 = jj & 1;
+      if (!warp_wait<true>(&bars.xs_full[b2], (jj >> 1) & 1, abort, p.status)) { alive = false; break; }
 #pragma unroll
       for (int i = 0; i < KT; i += 4) {
         float4 o;
         asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                      : "=f"(o.x), "=f"(o.y), "=f"(o.z), "=f"(o.w)
-                     : "r"(xs_row + i * 4));
+                     : "r"(xs_row0 + b2 * XS_BYTES + i * 4));
         s[i] += o.x;
         s[i + 1] += o.y;
         s[i + 2] += o.z;
         s[i + 3] += o.w;
       }
-      mbar_arrive_cluster(xs_free_peer);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(xs_free_peer0 + b2 * 8);
+      // next use of this buffer (tile jj + 2): expect the peer's bytes again
+      if (tid == 0 && jj + 2 < nt) mbar_arrive_expect_tx(&bars.xs_full[b2], XS_TX_BYTES);
 
-      // scale, mask, running max
+      // scale, mask, running max (log2 domain)
       float mt = -INFINITY;
 #pragma unroll
       for (int i = 0; i < KT; ++i) {
-        const bool ok = ((i < 32 ? mlo >> i : mhi >> (i - 32)) & 1u) != 0;
-        s[i] = ok ? s[i] * p.scale_log2 : -INFINITY;
+        s[i] = ((valid >> i) & 1u) ? s[i] * p.scale_log2 : -INFINITY;
         mt = fmaxf(mt, s[i]);
       }
       const float m_new = fmaxf(m_used, mt);
@@ -375,39 +445,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
         if (!warp_wait(&bars.o_done, (jj - 1) & 1, abort, p.status)) { alive = false; break; }
         tc_fence_after();
       }
-      if (rescale) {
-        const float alpha = exp2f(m_used - m_new);
-        l *= alpha;
-        if (jj > 0) {
-          uint32_t r[16];
+      const float alpha = rescale ? fast_exp2(m_used - m_new) : 1.f;
+      l *= alpha;
+      if (jj > 0 && __any_sync(0xffffffffu, rescale)) {
+        // warp-collective: rows that keep their maximum scale by 1
+        uint32_t r[16];
 #pragma unroll 1
-          for (int c = 0; c < 256; c += 16) {
-            const uint32_t ta = tmem + lane_base + 256 + c;
-            tmem_ld16(ta, r);
-            tc_wait_ld();
+        for (int c = 0; c < 256; c += 16) {
+          const uint32_t ta = tmem + lane_base + 256 + c;
+          tmem_ld16(ta, r);
+          tc_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st16(ta, r);
-          }
-          tc_wait_st();
+          for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st16(ta, r);
         }
-        m_used = m_new;
+        tc_wait_st();
       }
-      // P = 2^(s - m) in bf16, summed as rounded
+      if (rescale) m_used = m_new;
+      // P = 2^(s - m) in bf16; the row sum adds the rounded values
       const bool live = m_used != -INFINITY;
       float psum = 0.f;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < KT / 8; ++c) {
         uint32_t w[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float e0 = live ? exp2f(s[c * 8 + 2 * i] - m_used) : 0.f;
-          const float e1 = live ? exp2f(s[c * 8 + 2 * i + 1] - m_used) : 0.f;
+          const float e0 = live ? fast_exp2(s[c * 8 + 2 * i] - m_used) : 0.f;
+          const float e1 = live ? fast_exp2(s[c * 8 + 2 * i + 1] - m_used) : 0.f;
           const __nv_bfloat162 pr = __floats2bfloat162_rn(e0, e1);
-          psum += __low2float(pr) + __high2float(pr);
+          const float2 back = __bfloat1622float2(pr);
+          psum += back.x + back.y;
           w[i] = *reinterpret_cast<const uint32_t*>(&pr);
         }
-        st_shared_v4(prow + sw128_off(h, c), w[0], w[1], w[2], w[3]);
+        st_shared_v4(prow + sw64_off(h, c), w[0], w[1], w[2], w[3]);
       }
       l += psum;
       fence_proxy_async_smem();
@@ -518,32 +588,54 @@ __global__ void __launch_bounds__(256) merge_uv_kernel(const __nv_bfloat16* __re
     }
     for (int q = tid; q < 128 * 16; q += 256) {
       const int d = q >> 4, ch = q & 15;
-      const uint4 v =
-          ld_global_nc_v4(wkv_b + ((size_t)h * 256 + kDn + d) * kC + kc * 128 + ch * 8);
-      st_shared_v4(sA + (ch >> 3) * 16384 + sw128_off(d, ch & 7), v.x, v.y, v.z, v.w);
+      cp_async_16(sA + (ch >> 3) * 16384 + sw128_off(d, ch & 7),
+                  wkv_b + ((size_t)h * 256 + kDn + d) * kC + kc * 128 + ch * 8, 16);
     }
-    for (int q = tid; q < NB * 16; q += 256) {
-      const int n = q >> 4, ch = q & 15, b = b0 + n;
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if (b < B) {
-        for (int s = 0; s < splits; ++s) {
-          const float w = wts[n * splits + s];
-          if (w == 0.f) continue;
-          const uint4 v = ld_global_nc_v4(opart + (((size_t)b * splits + s) * kH + h) * kC +
-                                          kc * 128 + ch * 8);
-          const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&v);
+    // merged O~ chunk: 4 independent 16-byte items per thread in flight
+#pragma unroll 1
+    for (int q0 = tid; q0 < NB * 16; q0 += 256 * 4) {
+      float acc[4][8];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
+#pragma unroll 1
+      for (int s = 0; s < splits; ++s) {
+        uint4 v[4];
+        float w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int q = q0 + 256 * u;
+          const int n = q >> 4, ch = q & 15, b = b0 + n;
+          w[u] = (q < NB * 16 && b < B) ? wts[n * splits + s] : 0.f;
+          v[u] = make_uint4(0, 0, 0, 0);
+          if (w[u] != 0.f)
+            v[u] = ld_global_nc_v4(opart + (((size_t)b * splits + s) * kH + h) * kC + kc * 128 +
+                                   ch * 8);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const float2 f = __bfloat1622float2(pv[i]);
-            acc[2 * i] += w * f.x;
-            acc[2 * i + 1] += w * f.y;
+            acc[u][2 * i] += w[u] * f.x;
+            acc[u][2 * i + 1] += w[u] * f.y;
           }
         }
       }
-      st_shared_v4(sB + (ch >> 3) * (NB * 128) + sw128_off(n, ch & 7), pack_bf16x2(acc[0], acc[1]),
-                   pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
-                   pack_bf16x2(acc[6], acc[7]));
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int q = q0 + 256 * u;
+        if (q < NB * 16) {
+          const int n = q >> 4, ch = q & 15;
+          st_shared_v4(sB + (ch >> 3) * (NB * 128) + sw128_off(n, ch & 7),
+                       pack_bf16x2(acc[u][0], acc[u][1]), pack_bf16x2(acc[u][2], acc[u][3]),
+                       pack_bf16x2(acc[u][4], acc[u][5]), pack_bf16x2(acc[u][6], acc[u][7]));
+        }
+      }
     }
+    cp_async_wait_all();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();

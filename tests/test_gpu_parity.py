@@ -173,11 +173,19 @@ def test_decode_zero_query_uniform(shla):
 
 
 def test_decode_large_scores_trigger_rescaling(shla):
-    """A large softmax scale makes the running maximum grow across tiles."""
+    """A large softmax scale (scores with std ~5.5 instead of ~1) makes the
+    running maximum grow across tiles, so the accumulator is rescaled at
+    different tiles in different rows.  The softmax is then nearly one-hot
+    and O takes values of order 1 instead of ~0.04, so the absolute bound of
+    the workload tolerance is scaled by max|O| (the bf16 output rounding alone
+    is up to 2^-9 |O|)."""
     wl = mi.make_small(B=2, T=2000, k=1500, seed=14, device="cuda")
     out = shla.mla_decode(wl.q_nope, wl.q_pe, wl.wkv_b, wl.cache, wl.topk, wl.end_pos, 0.4)
     wl.scale = 0.4
-    _check_O(out, _oracle_decode(wl))
+    ref = _oracle_decode(wl)
+    g = out.double().cpu().numpy()
+    assert _rel(g, ref) <= REL_L2
+    assert np.abs(g - ref).max() <= MAX_ABS * max(1.0, np.abs(ref).max())
 
 
 def test_decode_deterministic_and_canaries(shla):
