@@ -2,18 +2,38 @@
 // branch, model.py 590-606).  Three kernels on the caller's stream:
 //
 //   fold_kernel      q~ = q_nope W_UK per head (tcgen05, latent as M, batch as N)
-//   core_kernel      per (batch row, key split), a 2-CTA cluster: gather the
-//                    selected cache rows, S = Q~ K^T with the 128 heads as M,
-//                    fp32 online softmax, O~ += P V.  CTA r of the pair owns
-//                    latent columns [256r, 256r+256) and rotary columns
-//                    [32r, 32r+32); the two partial score tiles are summed
-//                    through distributed shared memory.
-//   merge_uv_kernel  log-sum-exp merge of the splits, then O = O~ W_UV^T per
-//                    head (tcgen05, value dim as M, batch as N)
+//   core_kernel      persistent 2-CTA clusters over equal ranges of the
+//                    (batch row, key tile) list: TMA gather of the selected
+//                    cache rows, S = Q~ K^T with the 128 heads as M, fp32
+//                    online softmax, O~ += P V.  CTA r of the pair owns latent
+//                    columns [256r, 256r+256) and rotary columns [32r, 32r+32);
+//                    the two partial score tiles are summed through
+//                    distributed shared memory.
+//   merge_uv_kernel  log-sum-exp merge of the partial outputs of each row,
+//                    then O = O~ W_UV^T per head (tcgen05, value dim as M,
+//                    batch as N)
+#include <cuda_fp16.h>
 #include <math.h>
 
 #include "common.cuh"
 #include "host_util.h"
+
+// Optional per-role cycle accounting of the attend kernel (build with
+// -DSHLA_TRACE; the default build compiles the hooks away).  Each hook adds
+// the cycles since the previous hook to one bucket.
+#ifdef SHLA_TRACE
+namespace shla {
+__device__ unsigned long long g_trace[512][3][16];
+}
+#define SHLA_TRACE_DECL unsigned long long tr_[16] = {}; unsigned long long tp_ = clock64();
+#define SHLA_T(i) do { const unsigned long long n_ = clock64(); tr_[i] += n_ - tp_; tp_ = n_; } while (0)
+#define SHLA_TRACE_FLUSH(role) do { if (blockIdx.x < 512) for (int i_ = 0; i_ < 16; ++i_) \
+    atomicAdd(&shla::g_trace[blockIdx.x][role][i_], tr_[i_]); } while (0)
+#else
+#define SHLA_TRACE_DECL
+#define SHLA_T(i) do { } while (0)
+#define SHLA_TRACE_FLUSH(role) do { } while (0)
+#endif
 
 namespace shla {
 
@@ -108,67 +128,96 @@ __global__ void __launch_bounds__(128) fold_kernel(const __nv_bfloat16* __restri
 }
 
 // ===========================================================================
-// K2: sparse attention core on a 2-CTA cluster
+// K2: sparse attention core, persistent 2-CTA clusters
 //
-// Warp roles per CTA (288 threads):
-//   warps 0-3  softmax: one thread per head row (TMEM lane); exchange of the
-//              partial score tile with the peer CTA through DSMEM, running
-//              max / sum, P (bf16) into shared memory, O rescaling
-//   warps 4-7  gather: cp.async of this CTA's 288 columns of each selected
-//              cache row into a NST-deep ring of key tiles
-//   warp 8     TMEM owner and MMA issuer (one thread)
-// Per key tile j (KT keys):  S_j = Q~_half K_j_half^T (M=128, N=KT, K=288)
-// into one of two TMEM score buffers; after the softmax, O_half += P_j V_j_half
-// (M=128, N=256, K=KT) where V is the same shared-memory tile read MN-major.
+// The flattened list of key tiles (batch row b, tile j of row b) is cut into
+// one contiguous range per cluster, so every cluster gets the same number of
+// tiles whatever B and k are.  A range covers one or more "segments" (the
+// part of one batch row it holds); each segment ends with a partial output
+// (O~ normalised by its own sum, plus its log-sum-exp) that the merge kernel
+// combines.
+//
+// CTA r of the pair owns latent columns [256r, 256r+256) and rotary columns
+// [32r, 32r+32) of Q~ and of every selected cache row; both CTAs hold all 128
+// heads.  Per key tile (KT keys):
+//   S (partial)  = Q~_half K_half^T       M=128 heads, N=KT, K=288   (tcgen05)
+//   S            = S(own) + S(peer)      partials scaled to log2 units, rounded
+//                                        to fp16 and exchanged through DSMEM
+//   P            = 2^(S - m)             fp32 running max m and sum l
+//   O_half      += P V_half              M=128, N=256, K=KT          (tcgen05)
+// V is the same shared-memory tile as K, read MN-major.
+//
+// Warp roles (256 threads):
+//   warps 0-3  softmax, one thread per head row (TMEM lane); they also load
+//              this CTA's half of Q~ into TMEM at each segment start and
+//              write the segment outputs
+//   warps 4-6  gather: TMA tile::gather4 of the selected rows (4 rows per
+//              instruction); group g of four keys goes to warp 4 + g % 3
+//   warp 7     TMEM owner and MMA issuer (one thread)
+// TMEM (512 columns): S [0,KT), Q~ half [64,208) as bf16 pairs, P [224,256)
+// as bf16 pairs, O half [256,512) fp32.
 // ===========================================================================
 namespace core {
-constexpr int KT = 32;                       // keys per tile
-constexpr int NST = 6;                       // gather ring depth
-constexpr int NTHREADS = 288;
-constexpr int OFF_QC = 0;                    // Q~ latent half: 4 atoms x 128 rows x 128 B
-constexpr int OFF_QR = 65536;                // q_pe half: 128 rows x 64 B (64 B swizzle)
-constexpr int OFF_ST = 73728;                // key tiles
+constexpr int KT = 64;                       // keys per tile
+constexpr int NST = 4;                       // gather ring depth
+constexpr int NTHREADS = 256;
+constexpr int NGATHER = 3;                   // gather warps
+constexpr int MMA_WARP = 4 + NGATHER;
 constexpr int ST_ATOM = KT * 128;            // one 64-column latent atom of a tile
 constexpr int ST_KR = 4 * ST_ATOM;           // rotary part of a tile (64 B swizzle)
-constexpr int ST_BYTES = ST_KR + KT * 64;
-constexpr int OFF_P = OFF_ST + NST * ST_BYTES;   // P: 128 rows x KT bf16 (64 B swizzle)
-constexpr int P_BYTES = 128 * KT * 2;
-constexpr int OFF_XS = OFF_P + P_BYTES;          // two buffers of exchanged partial scores
-constexpr int XS_STRIDE = KT * 4 + 16;           // padded fp32 row
+constexpr int ST_BYTES = ST_KR + KT * 64;    // 36864
+constexpr int OFF_ST = 0;
+constexpr int OFF_XS = OFF_ST + NST * ST_BYTES;  // two buffers of exchanged partial scores
+constexpr int XS_STRIDE = KT * 2 + 16;           // padded fp16 row
 constexpr int XS_BYTES = 128 * XS_STRIDE;
 constexpr int OFF_END = OFF_XS + 2 * XS_BYTES;
-constexpr uint32_t XS_TX_BYTES = 128 * KT * 4;   // partial scores received per tile
 constexpr int SMEM_BYTES = OFF_END + 1024;       // + alignment slack
-constexpr uint32_t TMEM_COLS = 512;              // S0 @0, S1 @KT, O half @256
+constexpr uint32_t XS_TX_BYTES = 128 * KT * 2;   // partial scores received per tile
+constexpr uint32_t GROUP_TX_BYTES = ST_BYTES / 16;  // bytes of one group of four keys
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t T_S = 0, T_Q = 64, T_P = 224, T_O = 256;
 constexpr float kRescaleThreshold = 8.0f;        // log2 units
-constexpr int PER_PRODUCER = KT * 36 / 128;      // 16-byte chunks per gather thread per tile
-static_assert(KT * 36 % 128 == 0, "gather split");
-static_assert(ST_BYTES % 1024 == 0 && OFF_ST % 1024 == 0 && OFF_P % 512 == 0, "alignment");
-static_assert(SMEM_BYTES + 256 <= 232448, "shared memory budget");
+constexpr float kExchangeClamp = 60000.f;        // fp16 exchange saturates here
+static_assert(ST_BYTES % 1024 == 0 && OFF_XS % 16 == 0, "alignment");
+static_assert(SMEM_BYTES + 512 <= 232448, "shared memory budget");
+static_assert(T_Q + 144 <= T_P && T_P + KT / 2 <= T_O, "TMEM plan");
+static_assert(KT / 4 == 16, "sixteen groups of four keys per tile");
+
+// Schedule: tiles [bnd(c), bnd(c+1)) of the flattened list belong to cluster c.
+struct Sched {
+  int nt;    // tiles per batch row
+  int tot;   // B * nt
+  int nc;    // clusters
+  __host__ __device__ long long bnd(int c) const { return (long long)c * tot / nc; }
+  // first / last cluster whose range meets batch row b
+  __host__ __device__ int c_first(int b) const {
+    return (int)(((long long)b * nt + 1) * nc + tot - 1) / tot - 1;
+  }
+  __host__ __device__ int c_last(int b) const {
+    return (int)(((long long)(b + 1) * nt) * nc + tot - 1) / tot - 1;
+  }
+};
 
 struct Params {
   const __nv_bfloat16* q_tilde;   // [B][128][512]
   const __nv_bfloat16* q_pe;      // [B][128][64]
-  const __nv_bfloat16* c_kv;
-  long long ckv_bs;
-  int ckv_rs;
-  const __nv_bfloat16* k_pe;
-  long long kpe_bs;
-  int kpe_rs;
+  long long rows_per_b;           // row-index distance between batch rows in the cache maps
   int T;
   const int32_t* topk;
   int k;
   const int32_t* end_pos;
-  int B, splits, tiles_per_split, ntiles;
+  int B;
+  Sched sch;
+  int slots;                      // partial-output slots per batch row
   float scale_log2;               // softmax scale * log2(e)
-  __nv_bfloat16* opart;           // [B][splits][128][512], normalised per split
-  float* lse;                     // [B][splits][128], log2 units of scaled scores
+  __nv_bfloat16* opart;           // [B][slots][128][512], normalised per segment
+  float* lse;                     // [B][slots][128], log2 units of scaled scores
   int32_t* status;
 };
 
 struct Bars {
-  uint64_t full[NST], empty[NST], s_full[2], s_empty[2], p_full, o_done, xs_full[2], xs_free[2],
-      drain;
+  uint64_t full[NST], empty[NST], s_full, s_empty, p_full, o_done, q_ready, xs_full[2],
+      xs_free[2], drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -178,7 +227,8 @@ DEV bool key_valid(int v, int lim) { return v >= 0 && v < lim; }
 }  // namespace core
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
-    core_kernel(const core::Params p) {
+    core_kernel(const core::Params p, const __grid_constant__ CUtensorMap map_c,
+                const __grid_constant__ CUtensorMap map_r) {
   using namespace core;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -188,171 +238,176 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
   const int cid = blockIdx.x >> 1;
-  const int b = cid / p.splits;
-  const int sp = cid - b * p.splits;
-  const int tile0 = sp * p.tiles_per_split;
-  const int nt = min(p.ntiles, tile0 + p.tiles_per_split) - tile0;
-  const int lim = min(p.end_pos[b], p.T);
+  const int t_begin = (int)p.sch.bnd(cid), t_end = (int)p.sch.bnd(cid + 1);
+  const int n = t_end - t_begin;  // tiles of this cluster (>= 1)
+  const int nt = p.sch.nt;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sbase = smem_u32(smem);
-  const int32_t* topk_b = p.topk + (size_t)b * p.k;
+  auto row_of = [&](int i) { return (t_begin + i) / nt; };          // batch row of local tile i
+  auto seg_start = [&](int i) { return i == 0 || (t_begin + i) % nt == 0; };
+  auto lim_of = [&](int bb) { return min(p.end_pos[bb], p.T); };
 
-  if (warp == 8) {
+  if (warp == MMA_WARP) {
     tmem_alloc(&bars.tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
   if (tid == 0) {
     for (int s = 0; s < NST; ++s) {
-      mbar_init(&bars.full[s], 128);
-      mbar_init(&bars.empty[s], 1);
+      mbar_init(&bars.full[s], NGATHER);  // one expect_tx arrival per gather warp + bytes
+      mbar_init(&bars.empty[s], 1);       // MMA commit after the tile's value product
     }
+    mbar_init(&bars.s_full, 1);
+    mbar_init(&bars.s_empty, 128);
+    mbar_init(&bars.p_full, 128);
+    mbar_init(&bars.o_done, 1);
+    mbar_init(&bars.q_ready, 128);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.s_full[i], 1);
-      mbar_init(&bars.s_empty[i], 128);
       mbar_init(&bars.xs_full[i], 1);    // own expect_tx arrival + the peer's st.async bytes
       mbar_init(&bars.xs_free[i], 4);    // one arrival per softmax warp of the peer
     }
-    mbar_init(&bars.p_full, 128);
-    mbar_init(&bars.o_done, 1);
     mbar_init(&bars.drain, 1);
     bars.abort = 0;
     fence_mbarrier_init_cluster();
-    // first use of each exchange buffer: expect one tile of partial scores
     mbar_arrive_expect_tx(&bars.xs_full[0], XS_TX_BYTES);
     mbar_arrive_expect_tx(&bars.xs_full[1], XS_TX_BYTES);
   }
-  // this CTA's half of Q~ (latent) and of q_pe (rotary)
-  for (int q = tid; q < 128 * 36; q += NTHREADS) {
-    const int h = q / 36, ch = q - h * 36;
-    if (ch < 32)
-      cp_async_16(sbase + OFF_QC + (ch >> 3) * 16384 + sw128_off(h, ch & 7),
-                  p.q_tilde + ((size_t)b * kH + h) * kC + rank * 256 + ch * 8, 16);
-    else
-      cp_async_16(sbase + OFF_QR + sw64_off(h, ch - 32),
-                  p.q_pe + ((size_t)b * kH + h) * kR + rank * 32 + (ch - 32) * 8, 16);
-  }
-  cp_async_wait_all();
-  fence_proxy_async_smem();
   tc_fence_before();
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
 
-  if (warp >= 4 && warp < 8) {
-    // ---------------- gather ----------------
-    const int pt = tid - 128;
+  if (warp >= 4 && warp < MMA_WARP) {
+    // ---------------- gather (TMA tile::gather4) ----------------
+    // lane l holds the index of key l and key 32 + l of the tile; lanes
+    // 0..ng-1 each issue the five loads of one group of four keys
+    const int gw = warp - 4;
+    const int ng = (16 - gw + NGATHER - 1) / NGATHER;  // groups of this warp
     int bad = 0;
-    const __nv_bfloat16* ckv_b = p.c_kv + (size_t)b * p.ckv_bs + rank * 256;
-    const __nv_bfloat16* kpe_b = p.k_pe + (size_t)b * p.kpe_bs + rank * 32;
-    int key[PER_PRODUCER], ch[PER_PRODUCER], v[PER_PRODUCER];
-#pragma unroll
-    for (int i = 0; i < PER_PRODUCER; ++i) {
-      const int q = pt + 128 * i;
-      key[i] = q / 36;
-      ch[i] = q - key[i] * 36;
-      const int j = tile0 * KT + key[i];
-      v[i] = j < p.k ? topk_b[j] : -1;
-    }
+    int va = -1, vb = -1;
+    auto load_idx = [&](int i) {
+      const int bb = row_of(i);
+      const int j = ((t_begin + i) - bb * nt) * KT + lane;
+      const int32_t* tk = p.topk + (size_t)bb * p.k;
+      va = j < p.k ? tk[j] : -1;
+      vb = j + 32 < p.k ? tk[j + 32] : -1;
+    };
+    load_idx(0);
+    SHLA_TRACE_DECL
 #pragma unroll 1
-    for (int jj = 0; jj < nt; ++jj) {
-      const int s = jj % NST;
-      if (!mbar_wait(&bars.empty[s], ((jj / NST) & 1) ^ 1, abort, p.status)) break;
-      const uint32_t stage = sbase + OFF_ST + s * ST_BYTES;
+    for (int i = 0; i < n; ++i) {
+      const int s = i % NST;
+      const int bb = row_of(i);
+      const int lim = lim_of(bb);
+      const bool oka = key_valid(va, lim), okb = key_valid(vb, lim);
+      if (rank == 0 && gw == 0) bad += (!oka && va != -1) + (!okb && vb != -1);
+      // TMA rows: valid keys map to their cache row, others to row -1 (zero fill)
+      const int ra = oka ? (int)((long long)bb * p.rows_per_b + va) : -1;
+      const int rb = okb ? (int)((long long)bb * p.rows_per_b + vb) : -1;
+      if (i + 1 < n) load_idx(i + 1);
+      SHLA_T(1);
+      if (!warp_wait(&bars.empty[s], ((i / NST) & 1) ^ 1, abort, p.status)) break;
+      SHLA_T(0);
+      if (lane == 0) mbar_arrive_expect_tx(&bars.full[s], ng * GROUP_TX_BYTES);
+      __syncwarp();
+      const int g = gw + NGATHER * (lane < ng ? lane : 0);  // this lane's group
+      const int k0 = 4 * g;                                 // its first key (0..60)
+      const int src = k0 & 31;
+      const int y0 = __shfl_sync(0xffffffffu, ra, src);
+      const int y0b = __shfl_sync(0xffffffffu, rb, src);
+      const int y1 = __shfl_sync(0xffffffffu, ra, src + 1);
+      const int y1b = __shfl_sync(0xffffffffu, rb, src + 1);
+      const int y2 = __shfl_sync(0xffffffffu, ra, src + 2);
+      const int y2b = __shfl_sync(0xffffffffu, rb, src + 2);
+      const int y3 = __shfl_sync(0xffffffffu, ra, src + 3);
+      const int y3b = __shfl_sync(0xffffffffu, rb, src + 3);
+      if (lane < ng) {
+        const bool hi = k0 >= 32;
+        const int r0 = hi ? y0b : y0, r1 = hi ? y1b : y1, r2 = hi ? y2b : y2, r3 = hi ? y3b : y3;
+        const uint32_t stage = sbase + OFF_ST + s * ST_BYTES;
 #pragma unroll
-      for (int i = 0; i < PER_PRODUCER; ++i) {
-        const bool ok = key_valid(v[i], lim);
-        if (rank == 0 && ch[i] == 0 && !ok && v[i] != -1) ++bad;
-        const long long vv = ok ? v[i] : 0;
-        const void* src;
-        uint32_t dst;
-        if (ch[i] < 32) {
-          src = ckv_b + vv * p.ckv_rs + ch[i] * 8;
-          dst = stage + (ch[i] >> 3) * ST_ATOM + sw128_off(key[i], ch[i] & 7);
-        } else {
-          src = kpe_b + vv * p.kpe_rs + (ch[i] - 32) * 8;
-          dst = stage + ST_KR + sw64_off(key[i], ch[i] - 32);
-        }
-        cp_async_16(dst, src, ok ? 16u : 0u);
+        for (int a = 0; a < 4; ++a)
+          tma_gather4(stage + a * ST_ATOM + k0 * 128, &map_c, rank * 256 + a * 64, r0, r1, r2, r3,
+                      &bars.full[s]);
+        tma_gather4(stage + ST_KR + k0 * 64, &map_r, rank * 32, r0, r1, r2, r3, &bars.full[s]);
       }
-      cp_async_arrive_noinc(&bars.full[s]);
-      // indices of the next tile, loaded while this one is in flight
-      if (jj + 1 < nt) {
-#pragma unroll
-        for (int i = 0; i < PER_PRODUCER; ++i) {
-          const int j = (tile0 + jj + 1) * KT + key[i];
-          v[i] = j < p.k ? topk_b[j] : -1;
-        }
-      }
+      SHLA_T(2);
     }
-    cp_async_wait_all();
-    if (bad && p.status) atomicAdd(p.status + 1, bad);
-  } else if (warp == 8) {
+    if (lane == 0 && gw == 0) SHLA_TRACE_FLUSH(1);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);
+    if (lane == 0 && bad && p.status) atomicAdd(p.status + 1, bad);
+  } else if (warp == MMA_WARP) {
     // ---------------- MMA issuer ----------------
-    // Event loop: a score tile is computed as soon as its keys have landed
-    // and a score buffer is free (up to two tiles ahead of the softmax); a
-    // value product as soon as its P is in shared memory.
+    // Event loop: a value product as soon as its P is in TMEM (first, so the
+    // softmax never waits behind a score tile queued after it); a score tile
+    // as soon as its keys have landed, the score buffer has been read and
+    // this segment's Q~ is in TMEM.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, KT, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, 0, 1);
-      const uint32_t qc = sbase + OFF_QC, qr = sbase + OFF_QR, pb = sbase + OFF_P;
-      int qk = 0, pv = 0, idle = 0;
+      int qk = 0, pv = 0, idle = 0, qseg = -1;
+      bool alive = true;
       uint64_t t_last = globaltimer_ns();
+      SHLA_TRACE_DECL
 #pragma unroll 1
-      while (pv < nt) {
+      while (alive && pv < n) {
         bool did = false;
-        if (qk < nt && mbar_test(&bars.full[qk % NST], (qk / NST) & 1) &&
-            mbar_test(&bars.s_empty[qk & 1], ((qk >> 1) & 1) ^ 1)) {
-          fence_proxy_async_smem();
-          tc_fence_after();
-          const uint32_t st = sbase + OFF_ST + (qk % NST) * ST_BYTES;
-          const uint32_t d = tmem + (qk & 1) * KT;
-#pragma unroll
-          for (int ks = 0; ks < 16; ++ks) {
-            const uint64_t ad =
-                smem_desc(qc + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSwizzle128B);
-            const uint64_t bd =
-                smem_desc(st + (ks >> 2) * ST_ATOM + (ks & 3) * 32, 16, 1024, kSwizzle128B);
-            tc_mma(d, ad, bd, idesc_qk, ks > 0);
-          }
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-            const uint64_t ad = smem_desc(qr + ks * 32, 16, 512, kSwizzle64B);
-            const uint64_t bd = smem_desc(st + ST_KR + ks * 32, 16, 512, kSwizzle64B);
-            tc_mma(d, ad, bd, idesc_qk, 1);
-          }
-          tc_commit(&bars.s_full[qk & 1]);
-          ++qk;
-          did = true;
-        }
         if (pv < qk && mbar_test(&bars.p_full, pv & 1)) {
           tc_fence_after();
           const int s = pv % NST;
           const uint32_t st = sbase + OFF_ST + s * ST_BYTES;
+          const bool first = seg_start(pv);
 #pragma unroll
           for (int ks = 0; ks < KT / 16; ++ks) {
-            const uint64_t ad = smem_desc(pb + ks * 32, 16, 512, kSwizzle64B);
             const uint64_t bd = smem_desc(st + ks * 2048, ST_ATOM, 1024, kSwizzle128B);
-            tc_mma(tmem + 256, ad, bd, idesc_pv, (pv > 0 || ks > 0) ? 1u : 0u);
+            tc_mma_tmem_a(tmem + T_O, tmem + T_P + ks * 8, bd, idesc_pv,
+                          (!first || ks > 0) ? 1u : 0u);
           }
           tc_commit(&bars.o_done);
           tc_commit(&bars.empty[s]);
           ++pv;
           did = true;
+          SHLA_T(1);
         }
+        if (qk < n && mbar_test(&bars.full[qk % NST], (qk / NST) & 1) &&
+            (qk == 0 || mbar_test(&bars.s_empty, (qk - 1) & 1))) {
+          const int seg = seg_start(qk) ? qseg + 1 : qseg;
+          if (seg == qseg || mbar_test(&bars.q_ready, seg & 1)) {
+            qseg = seg;
+            tc_fence_after();
+            const uint32_t st = sbase + OFF_ST + (qk % NST) * ST_BYTES;
+#pragma unroll
+            for (int ks = 0; ks < 16; ++ks) {
+              const uint64_t bd =
+                  smem_desc(st + (ks >> 2) * ST_ATOM + (ks & 3) * 32, 16, 1024, kSwizzle128B);
+              tc_mma_tmem_a(tmem + T_S, tmem + T_Q + ks * 8, bd, idesc_qk, ks > 0);
+            }
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks) {
+              const uint64_t bd = smem_desc(st + ST_KR + ks * 32, 16, 512, kSwizzle64B);
+              tc_mma_tmem_a(tmem + T_S, tmem + T_Q + 128 + ks * 8, bd, idesc_qk, 1);
+            }
+            tc_commit(&bars.s_full);
+            ++qk;
+            did = true;
+            SHLA_T(2);
+          }
+        }
+        SHLA_T(0);
         if (did) {
           idle = 0;
+          t_last = globaltimer_ns();
         } else if (++idle >= 64) {
           idle = 0;
-          const uint64_t now = globaltimer_ns();
           if (*abort) break;
-          if (now - t_last > kWaitLimitNs) {
+          if (globaltimer_ns() - t_last > kWaitLimitNs) {
             *abort = 1;
             report_timeout(p.status);
             break;
           }
         }
-        if (did) t_last = globaltimer_ns();
       }
+      SHLA_TRACE_FLUSH(2);
       // everything issued so far has finished before TMEM is released
       tc_commit(&bars.drain);
       mbar_wait(&bars.drain, 0, nullptr, p.status);
@@ -362,161 +417,238 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     // ---------------- softmax (one thread per head row) ----------------
     const int h = tid;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    // this CTA's half of Q~ (256 latent + 32 rotary values) of batch row bb
+    // into TMEM as bf16 pairs (9 stores of 16 columns), then q_ready
+    auto load_q = [&](int bb) {
+      const __nv_bfloat16* qrow = p.q_tilde + ((size_t)bb * kH + h) * kC + rank * 256;
+      const __nv_bfloat16* rrow = p.q_pe + ((size_t)bb * kH + h) * kR + rank * 32;
+#pragma unroll
+      for (int c = 0; c < 9; ++c) {
+        const __nv_bfloat16* src = c < 8 ? qrow + c * 32 : rrow;
+        uint32_t r[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 q = ld_global_nc_v4(src + i * 8);
+          r[4 * i] = q.x;
+          r[4 * i + 1] = q.y;
+          r[4 * i + 2] = q.z;
+          r[4 * i + 3] = q.w;
+        }
+        tmem_st16(tmem + lane_base + T_Q + c * 16, r);
+      }
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars.q_ready);
+    };
+    load_q(row_of(0));
+
     // exchange buffer / barrier i sits at +i*XS_BYTES / +i*8 from buffer 0 in
     // both CTAs, so the peer addresses follow from one mapa each
     const uint32_t xs_row0 = sbase + OFF_XS + h * XS_STRIDE;
     const uint32_t xs_peer_row0 = mapa_shared(xs_row0, peer);
     const uint32_t xs_full_peer0 = mapa_shared(smem_u32(&bars.xs_full[0]), peer);
-    // (each exchange buffer's xs_full phase expects XS_TX_BYTES from the peer)
     const uint32_t xs_free_peer0 = mapa_shared(smem_u32(&bars.xs_free[0]), peer);
-    const uint32_t prow = sbase + OFF_P;
     float m_used = -INFINITY, l = 0.f;
-    float sn[KT];  // own partial scores of the tile after the current one
+    uint32_t sa[KT / 2], sb[KT / 2];  // own scaled partial scores (fp16 pairs): current, next
     bool alive = true;
+    SHLA_TRACE_DECL
 
-    // own partial of tile t: TMEM -> registers -> peer's exchange buffer
-    auto fetch_send = [&](int t) -> bool {
+    // own partial of tile t: TMEM -> scaled, fp16 -> the peer's exchange buffer
+    auto fetch_send = [&](int t, uint32_t (&dst)[KT / 2]) -> bool {
       const int b2 = t & 1;
-      if (!warp_wait(&bars.s_full[b2], (t >> 1) & 1, abort, p.status)) return false;
+      SHLA_T(11);
+      if (!warp_wait(&bars.s_full, t & 1, abort, p.status)) return false;
+      SHLA_T(0);
       tc_fence_after();
       {
-        uint32_t r[16];
+        uint32_t r[4][16];
 #pragma unroll
-        for (int c = 0; c < KT; c += 16) {
-          tmem_ld16(tmem + lane_base + b2 * KT + c, r);
-          tc_wait_ld();
+        for (int c = 0; c < 4; ++c) tmem_ld16(tmem + lane_base + T_S + c * 16, r[c]);
+        tc_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) sn[c + i] = __uint_as_float(r[i]);
-        }
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float x0 = fminf(fmaxf(__uint_as_float(r[c][2 * i]) * p.scale_log2, -kExchangeClamp), kExchangeClamp);
+            const float x1 = fminf(fmaxf(__uint_as_float(r[c][2 * i + 1]) * p.scale_log2, -kExchangeClamp), kExchangeClamp);
+            const __half2 hv = __floats2half2_rn(x0, x1);
+            dst[c * 8 + i] = *reinterpret_cast<const uint32_t*>(&hv);
+          }
       }
       tc_fence_before();
-      mbar_arrive(&bars.s_empty[b2]);
+      mbar_arrive(&bars.s_empty);
+      // the next tile starts a new segment: its Q~ replaces this one (the score
+      // tile just read was the last product that used it)
+      if (t + 1 < n && seg_start(t + 1)) load_q(row_of(t + 1));
+      SHLA_T(1);
       if (!warp_wait<true>(&bars.xs_free[b2], ((t >> 1) & 1) ^ 1, abort, p.status)) return false;
+      SHLA_T(2);
 #pragma unroll
-      for (int i = 0; i < KT; i += 4)
-        st_async_v4(xs_peer_row0 + b2 * XS_BYTES + i * 4, sn[i], sn[i + 1], sn[i + 2], sn[i + 3],
-                    xs_full_peer0 + b2 * 8);
+      for (int i = 0; i < KT / 2; i += 4)
+        st_async_v4(xs_peer_row0 + b2 * XS_BYTES + i * 4, __uint_as_float(dst[i]),
+                    __uint_as_float(dst[i + 1]), __uint_as_float(dst[i + 2]),
+                    __uint_as_float(dst[i + 3]), xs_full_peer0 + b2 * 8);
+      SHLA_T(3);
       return true;
     };
 
-    int vpre = (tile0 * KT + lane < p.k) ? topk_b[tile0 * KT + lane] : -1;
-    alive = fetch_send(0);
+    // epilogue of a segment: this CTA's latent half of O~ / l into the
+    // segment's slot, and (rank 0) the row's log-sum-exp
+    auto flush = [&](int i_last) -> bool {
+      if (!warp_wait(&bars.o_done, i_last & 1, abort, p.status)) return false;
+      tc_fence_after();
+      const int bb = row_of(i_last);
+      const int slot = cid - p.sch.c_first(bb);
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* dst = p.opart + (((size_t)bb * p.slots + slot) * kH + h) * kC + rank * 256;
+      uint32_t r[16];
 #pragma unroll 1
-    for (int jj = 0; jj < nt && alive; ++jj) {
-      const uint32_t valid = __ballot_sync(0xffffffffu, key_valid(vpre, lim));
-      if (jj + 1 < nt) {
-        const int j = (tile0 + jj + 1) * KT + lane;
-        vpre = j < p.k ? topk_b[j] : -1;
+      for (int c = 0; c < 256; c += 16) {
+        tmem_ld16(tmem + lane_base + T_O + c, r);
+        tc_wait_ld();
+        uint4 lo, hi;
+        lo.x = pack_bf16x2(__uint_as_float(r[0]) * inv, __uint_as_float(r[1]) * inv);
+        lo.y = pack_bf16x2(__uint_as_float(r[2]) * inv, __uint_as_float(r[3]) * inv);
+        lo.z = pack_bf16x2(__uint_as_float(r[4]) * inv, __uint_as_float(r[5]) * inv);
+        lo.w = pack_bf16x2(__uint_as_float(r[6]) * inv, __uint_as_float(r[7]) * inv);
+        hi.x = pack_bf16x2(__uint_as_float(r[8]) * inv, __uint_as_float(r[9]) * inv);
+        hi.y = pack_bf16x2(__uint_as_float(r[10]) * inv, __uint_as_float(r[11]) * inv);
+        hi.z = pack_bf16x2(__uint_as_float(r[12]) * inv, __uint_as_float(r[13]) * inv);
+        hi.w = pack_bf16x2(__uint_as_float(r[14]) * inv, __uint_as_float(r[15]) * inv);
+        *reinterpret_cast<uint4*>(dst + c) = lo;
+        *reinterpret_cast<uint4*>(dst + c + 8) = hi;
       }
-      float s[KT];
-#pragma unroll
-      for (int i = 0; i < KT; ++i) s[i] = sn[i];
-      if (jj + 1 < nt && !fetch_send(jj + 1)) { alive = false; break; }
+      if (rank == 0)
+        p.lse[((size_t)bb * p.slots + slot) * kH + h] = l > 0.f ? m_used + log2f(l) : -INFINITY;
+      tc_fence_before();
+      return true;
+    };
 
+    auto tile_idx = [&](int i, int off) {
+      const int bb = row_of(i);
+      const int j = ((t_begin + i) - bb * nt) * KT + off + lane;
+      return j < p.k ? p.topk[(size_t)bb * p.k + j] : -1;
+    };
+    int vlo = tile_idx(0, 0), vhi = tile_idx(0, 32);
+
+    // one key tile: `cur` holds this CTA's partial scores of tile i on entry;
+    // the next tile's partial is fetched into `nxt` and sent before the wait
+    auto step = [&](int i, uint32_t (&cur)[KT / 2], uint32_t (&nxt)[KT / 2]) -> bool {
+      const int lim = lim_of(row_of(i));
+      const uint32_t vmask_lo = __ballot_sync(0xffffffffu, key_valid(vlo, lim));
+      const uint32_t vmask_hi = __ballot_sync(0xffffffffu, key_valid(vhi, lim));
+      if (i + 1 < n) {
+        vlo = tile_idx(i + 1, 0);
+        vhi = tile_idx(i + 1, 32);
+        if (!fetch_send(i + 1, nxt)) return false;
+      }
       // add the peer's partial scores (other latent half) of this tile
-      const int b2 = jj & 1;
-      if (!warp_wait<true>(&bars.xs_full[b2], (jj >> 1) & 1, abort, p.status)) { alive = false; break; }
+      const int b2 = i & 1;
+      SHLA_T(11);
+      if (!warp_wait<true>(&bars.xs_full[b2], (i >> 1) & 1, abort, p.status)) return false;
+      SHLA_T(4);
+      float sc[KT];
 #pragma unroll
-      for (int i = 0; i < KT; i += 4) {
-        float4 o;
-        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                     : "=f"(o.x), "=f"(o.y), "=f"(o.z), "=f"(o.w)
-                     : "r"(xs_row0 + b2 * XS_BYTES + i * 4));
-        s[i] += o.x;
-        s[i + 1] += o.y;
-        s[i + 2] += o.z;
-        s[i + 3] += o.w;
+      for (int c = 0; c < KT / 2; c += 4) {
+        uint4 o;
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(o.x), "=r"(o.y), "=r"(o.z), "=r"(o.w)
+                     : "r"(xs_row0 + b2 * XS_BYTES + c * 4));
+        const uint32_t peer_w[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&cur[c + u]));
+          const float2 q = __half22float2(*reinterpret_cast<const __half2*>(&peer_w[u]));
+          sc[2 * (c + u)] = a.x + q.x;
+          sc[2 * (c + u) + 1] = a.y + q.y;
+        }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(xs_free_peer0 + b2 * 8);
-      // next use of this buffer (tile jj + 2): expect the peer's bytes again
-      if (tid == 0 && jj + 2 < nt) mbar_arrive_expect_tx(&bars.xs_full[b2], XS_TX_BYTES);
+      // next use of this buffer (tile i + 2): expect the peer's bytes again
+      if (tid == 0 && i + 2 < n) mbar_arrive_expect_tx(&bars.xs_full[b2], XS_TX_BYTES);
+      SHLA_T(5);
 
-      // scale, mask, running max (log2 domain)
+      // a new segment: write out the previous one and restart the running sums
+      const bool first = seg_start(i);
+      if (first && i > 0) {
+        if (!flush(i - 1)) return false;
+        m_used = -INFINITY;
+        l = 0.f;
+      }
+      // mask and running max (scores are already in log2 units)
       float mt = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < KT; ++i) {
-        s[i] = ((valid >> i) & 1u) ? s[i] * p.scale_log2 : -INFINITY;
-        mt = fmaxf(mt, s[i]);
+      for (int u = 0; u < KT; ++u) {
+        const uint32_t bit = u < 32 ? (vmask_lo >> u) & 1u : (vmask_hi >> (u - 32)) & 1u;
+        sc[u] = bit ? sc[u] : -INFINITY;
+        mt = fmaxf(mt, sc[u]);
       }
       const float m_new = fmaxf(m_used, mt);
       const bool rescale = m_new > m_used + kRescaleThreshold;
-      if (jj > 0) {
-        if (!warp_wait(&bars.o_done, (jj - 1) & 1, abort, p.status)) { alive = false; break; }
+      SHLA_T(6);
+      if (i > 0 && !first) {
+        if (!warp_wait(&bars.o_done, (i - 1) & 1, abort, p.status)) return false;
         tc_fence_after();
       }
+      SHLA_T(7);
       const float alpha = rescale ? fast_exp2(m_used - m_new) : 1.f;
       l *= alpha;
-      if (jj > 0 && __any_sync(0xffffffffu, rescale)) {
+      if (!first && __any_sync(0xffffffffu, rescale)) {
         // warp-collective: rows that keep their maximum scale by 1
         uint32_t r[16];
 #pragma unroll 1
         for (int c = 0; c < 256; c += 16) {
-          const uint32_t ta = tmem + lane_base + 256 + c;
+          const uint32_t ta = tmem + lane_base + T_O + c;
           tmem_ld16(ta, r);
           tc_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          for (int u = 0; u < 16; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * alpha);
           tmem_st16(ta, r);
         }
-        tc_wait_st();
       }
       if (rescale) m_used = m_new;
-      // P = 2^(s - m) in bf16; the row sum adds the rounded values
+      SHLA_T(8);
+      // P = 2^(s - m) as bf16 pairs into TMEM; the row sum adds the rounded values
       const bool live = m_used != -INFINITY;
-      float psum = 0.f;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < KT / 8; ++c) {
-        uint32_t w[4];
+      for (int c = 0; c < KT / 32; ++c) {
+        uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float e0 = live ? fast_exp2(s[c * 8 + 2 * i] - m_used) : 0.f;
-          const float e1 = live ? fast_exp2(s[c * 8 + 2 * i + 1] - m_used) : 0.f;
+        for (int u = 0; u < 16; ++u) {
+          const float e0 = live ? fast_exp2(sc[c * 32 + 2 * u] - m_used) : 0.f;
+          const float e1 = live ? fast_exp2(sc[c * 32 + 2 * u + 1] - m_used) : 0.f;
           const __nv_bfloat162 pr = __floats2bfloat162_rn(e0, e1);
           const float2 back = __bfloat1622float2(pr);
-          psum += back.x + back.y;
-          w[i] = *reinterpret_cast<const uint32_t*>(&pr);
+          ps[u & 3] += back.x + back.y;
+          w[u] = *reinterpret_cast<const uint32_t*>(&pr);
         }
-        st_shared_v4(prow + sw64_off(h, c), w[0], w[1], w[2], w[3]);
+        tmem_st16(tmem + lane_base + T_P + c * 16, w);
       }
-      l += psum;
-      fence_proxy_async_smem();
+      l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+      tc_wait_st();
       tc_fence_before();
       mbar_arrive(&bars.p_full);
-    }
-    // epilogue: this CTA's latent half of O~ / l, and (rank 0) the row's log-sum-exp
-    if (__all_sync(0xffffffffu, alive && !*abort)) {
-      if (warp_wait(&bars.o_done, (nt - 1) & 1, abort, p.status)) {
-        tc_fence_after();
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        __nv_bfloat16* dst =
-            p.opart + (((size_t)b * p.splits + sp) * kH + h) * kC + rank * 256;
-        uint32_t r[16];
+      // this tile's exchange buffer can take the peer's tile i + 2
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster_relaxed(xs_free_peer0 + b2 * 8);
+      SHLA_T(9);
+      return true;
+    };
+
+    alive = fetch_send(0, sa);
 #pragma unroll 1
-        for (int c = 0; c < 256; c += 16) {
-          tmem_ld16(tmem + lane_base + 256 + c, r);
-          tc_wait_ld();
-          uint4 lo, hi;
-          lo.x = pack_bf16x2(__uint_as_float(r[0]) * inv, __uint_as_float(r[1]) * inv);
-          lo.y = pack_bf16x2(__uint_as_float(r[2]) * inv, __uint_as_float(r[3]) * inv);
-          lo.z = pack_bf16x2(__uint_as_float(r[4]) * inv, __uint_as_float(r[5]) * inv);
-          lo.w = pack_bf16x2(__uint_as_float(r[6]) * inv, __uint_as_float(r[7]) * inv);
-          hi.x = pack_bf16x2(__uint_as_float(r[8]) * inv, __uint_as_float(r[9]) * inv);
-          hi.y = pack_bf16x2(__uint_as_float(r[10]) * inv, __uint_as_float(r[11]) * inv);
-          hi.z = pack_bf16x2(__uint_as_float(r[12]) * inv, __uint_as_float(r[13]) * inv);
-          hi.w = pack_bf16x2(__uint_as_float(r[14]) * inv, __uint_as_float(r[15]) * inv);
-          *reinterpret_cast<uint4*>(dst + c) = lo;
-          *reinterpret_cast<uint4*>(dst + c + 8) = hi;
-        }
-        if (rank == 0)
-          p.lse[((size_t)b * p.splits + sp) * kH + h] = l > 0.f ? m_used + log2f(l) : -INFINITY;
-      }
+    for (int i = 0; i < n && alive; i += 2) {
+      if (!step(i, sa, sb)) { alive = false; break; }
+      if (i + 1 < n && !step(i + 1, sb, sa)) { alive = false; break; }
     }
+    SHLA_T(10);
+    if (lane == 0) SHLA_TRACE_FLUSH(0);
+    if (__all_sync(0xffffffffu, alive && !*abort)) flush(n - 1);
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
@@ -525,24 +657,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
 }
 
 // ===========================================================================
-// K3: merge the key splits and apply W_UV.
+// K3: merge the partial outputs of each batch row and apply W_UV.
+//   O~[b,h,:] = sum_s w_s O~_s,  w_s = 2^(lse_s - max) / sum   (log-sum-exp merge)
 //   D^T[d, b] = sum_c W_UV[h][d][c] O~[b][h][c]
 //   A = W_UV[h] (M = 128 value dims, K = c), K-major
 //   B = merged O~ rows (N = batch rows, K = c), K-major, built in shared memory
 // grid (128 heads, batch blocks of NB); 256 threads; K in 4 chunks of 128.
 // ===========================================================================
+constexpr int kMaxSlots = 32;
+
 template <int NB>
 __global__ void __launch_bounds__(256) merge_uv_kernel(const __nv_bfloat16* __restrict__ wkv_b,
                                                         const __nv_bfloat16* __restrict__ opart,
                                                         const float* __restrict__ lse, int B,
-                                                        int splits, __nv_bfloat16* __restrict__ O,
+                                                        core::Sched sch, int slots,
+                                                        __nv_bfloat16* __restrict__ O,
                                                         int32_t* status) {
   constexpr uint32_t NCOLS = NB <= 32 ? 32 : NB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const uint32_t sA = smem_u32(smem);               // [2 katoms][128 d][128 B] = 32 KB
   const uint32_t sB = sA + 32768;                   // [2 katoms][NB][128 B]
-  float* wts = reinterpret_cast<float*>(smem + 32768 + NB * 256);   // [NB][splits]
+  float* wts = reinterpret_cast<float*>(smem + 32768 + NB * 256);   // [NB][slots]
   __shared__ uint64_t bar;
   __shared__ uint32_t tmem_base;
   const int h = blockIdx.x, b0 = blockIdx.y * NB;
@@ -556,24 +692,24 @@ __global__ void __launch_bounds__(256) merge_uv_kernel(const __nv_bfloat16* __re
     mbar_init(&bar, 1);
     fence_mbarrier_init_cluster();
   }
-  // split weights: w_s = 2^(lse_s - max) / sum
-  for (int n = tid; n < NB; n += 256) {
-    const int b = b0 + n;
-    float* w = wts + n * splits;
-    if (b >= B) {
-      for (int s = 0; s < splits; ++s) w[s] = 0.f;
-      continue;
-    }
+  // merge weights of the slots used by each row (others 0)
+  for (int nn = tid; nn < NB; nn += 256) {
+    const int b = b0 + nn;
+    float* w = wts + nn * slots;
+    for (int s = 0; s < slots; ++s) w[s] = 0.f;
+    if (b >= B) continue;
+    const int used = sch.c_last(b) - sch.c_first(b) + 1;
     float mx = -INFINITY;
-    for (int s = 0; s < splits; ++s) mx = fmaxf(mx, lse[((size_t)b * splits + s) * kH + h]);
+    for (int s = 0; s < used; ++s) mx = fmaxf(mx, lse[((size_t)b * slots + s) * kH + h]);
+    if (mx == -INFINITY) continue;
     float sum = 0.f;
-    for (int s = 0; s < splits; ++s) {
-      const float e = mx == -INFINITY ? 0.f : exp2f(lse[((size_t)b * splits + s) * kH + h] - mx);
+    for (int s = 0; s < used; ++s) {
+      const float e = exp2f(lse[((size_t)b * slots + s) * kH + h] - mx);
       w[s] = e;
       sum += e;
     }
-    const float inv = sum > 0.f ? 1.f / sum : 0.f;
-    for (int s = 0; s < splits; ++s) w[s] *= inv;
+    const float inv = 1.f / sum;
+    for (int s = 0; s < used; ++s) w[s] *= inv;
   }
   tc_fence_before();
   __syncthreads();
@@ -600,17 +736,17 @@ __global__ void __launch_bounds__(256) merge_uv_kernel(const __nv_bfloat16* __re
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
 #pragma unroll 1
-      for (int s = 0; s < splits; ++s) {
+      for (int s = 0; s < slots; ++s) {
         uint4 v[4];
         float w[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int q = q0 + 256 * u;
-          const int n = q >> 4, ch = q & 15, b = b0 + n;
-          w[u] = (q < NB * 16 && b < B) ? wts[n * splits + s] : 0.f;
+          const int nn = q >> 4, ch = q & 15, b = b0 + nn;
+          w[u] = (q < NB * 16 && b < B) ? wts[nn * slots + s] : 0.f;
           v[u] = make_uint4(0, 0, 0, 0);
           if (w[u] != 0.f)
-            v[u] = ld_global_nc_v4(opart + (((size_t)b * splits + s) * kH + h) * kC + kc * 128 +
+            v[u] = ld_global_nc_v4(opart + (((size_t)b * slots + s) * kH + h) * kC + kc * 128 +
                                    ch * 8);
         }
 #pragma unroll
@@ -628,8 +764,8 @@ __global__ void __launch_bounds__(256) merge_uv_kernel(const __nv_bfloat16* __re
       for (int u = 0; u < 4; ++u) {
         const int q = q0 + 256 * u;
         if (q < NB * 16) {
-          const int n = q >> 4, ch = q & 15;
-          st_shared_v4(sB + (ch >> 3) * (NB * 128) + sw128_off(n, ch & 7),
+          const int nn = q >> 4, ch = q & 15;
+          st_shared_v4(sB + (ch >> 3) * (NB * 128) + sw128_off(nn, ch & 7),
                        pack_bf16x2(acc[u][0], acc[u][1]), pack_bf16x2(acc[u][2], acc[u][3]),
                        pack_bf16x2(acc[u][4], acc[u][5]), pack_bf16x2(acc[u][6], acc[u][7]));
         }
@@ -684,51 +820,73 @@ __global__ void __launch_bounds__(256) merge_uv_kernel(const __nv_bfloat16* __re
 // host side
 // ===========================================================================
 
-constexpr int kMaxSplits = 32;
-
 static int ntiles_of(int k) { return (k + core::KT - 1) / core::KT; }
 
-// Pick how many key splits each batch row gets: balance waves of 2-SM
-// clusters against the traffic of the per-split partial outputs.
-static int choose_splits(int B, int k, int sm_count) {
-  const int ntiles = ntiles_of(k);
-  const int pairs = sm_count / 2 > 0 ? sm_count / 2 : 1;
-  int best_s = 1;
-  double best = 1e300;
-  const int smax = ntiles < kMaxSplits ? ntiles : kMaxSplits;
-  for (int s = 1; s <= smax; ++s) {
-    const int tps = (ntiles + s - 1) / s;
-    const int se = (ntiles + tps - 1) / tps;
-    const long long clusters = (long long)B * se;
-    const long long waves = (clusters + pairs - 1) / pairs;
-    const double cost = (double)waves * (tps + 1.0) + 3.5 * se * (double)B / pairs;
-    if (cost < best - 1e-9) {
-      best = cost;
-      best_s = se;
-    }
+// Clusters of the attend kernel that fit on the device at once (cached per
+// device); every cluster is persistent over its range of tiles.
+static int max_clusters() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 74;
   }
-  return best_s;
+  if (dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * 512);
+  cfg.blockDim = dim3(core::NTHREADS);
+  cfg.dynamicSmemBytes = core::SMEM_BYTES;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaFuncSetAttribute(core_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           core::SMEM_BYTES) != cudaSuccess ||
+      cudaOccupancyMaxActiveClusters(&n, core_kernel, &cfg) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    int sms = 148;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      sms = 148;
+    }
+    n = sms / 2;
+  }
+  if (dev < 64) cached[dev] = n;
+  return n;
 }
 
-static int sm_count_or_default() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess &&
-      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
-    return n;
-  cudaGetLastError();
-  return 148;
+static core::Sched make_sched(int B, int k, int clusters) {
+  core::Sched s;
+  s.nt = ntiles_of(k);
+  s.tot = B * s.nt;
+  s.nc = clusters < s.tot ? clusters : s.tot;
+  return s;
+}
+
+// partial-output slots per batch row: the most clusters that meet one row
+static int slots_of(const core::Sched& s, int B) {
+  int m = 1;
+  for (int b = 0; b < B; ++b) {
+    const int u = s.c_last(b) - s.c_first(b) + 1;
+    if (u > m) m = u;
+  }
+  return m;
 }
 
 struct WsLayout {
   size_t q_tilde, opart, lse, total;
 };
 
-static WsLayout ws_layout(int B, int splits) {
+static WsLayout ws_layout(int B, int slots) {
   WsLayout w;
   w.q_tilde = 0;
   w.opart = round_up(w.q_tilde + (size_t)B * kH * kC * 2, 256);
-  w.lse = round_up(w.opart + (size_t)B * splits * kH * kC * 2, 256);
-  w.total = round_up(w.lse + (size_t)B * splits * kH * 4, 256);
+  w.lse = round_up(w.opart + (size_t)B * slots * kH * kC * 2, 256);
+  w.total = round_up(w.lse + (size_t)B * slots * kH * 4, 256);
   return w;
 }
 
@@ -754,23 +912,67 @@ static int launch_fold(const __nv_bfloat16* q_nope, const __nv_bfloat16* wkv_b,
 
 template <int NB>
 static int launch_merge_nb(const __nv_bfloat16* wkv_b, const __nv_bfloat16* opart,
-                           const float* lse, int B, int splits, __nv_bfloat16* O,
-                           int32_t* status, cudaStream_t st) {
-  const int smem = 32768 + NB * 256 + NB * kMaxSplits * 4 + 1024;
+                           const float* lse, int B, const core::Sched& sch, int slots,
+                           __nv_bfloat16* O, int32_t* status, cudaStream_t st) {
+  const int smem = 32768 + NB * 256 + NB * kMaxSlots * 4 + 1024;
   static unsigned long long attr_done = 0;
   if (int e = ensure_smem_attr(merge_uv_kernel<NB>, smem, &attr_done)) return e;
   dim3 grid(kH, (B + NB - 1) / NB);
-  merge_uv_kernel<NB><<<grid, 256, smem, st>>>(wkv_b, opart, lse, B, splits, O, status);
+  merge_uv_kernel<NB><<<grid, 256, smem, st>>>(wkv_b, opart, lse, B, sch, slots, O, status);
   return launch_status();
 }
 
 static int launch_merge(const __nv_bfloat16* wkv_b, const __nv_bfloat16* opart, const float* lse,
-                        int B, int splits, __nv_bfloat16* O, int32_t* status, cudaStream_t st) {
-  if (B <= 16) return launch_merge_nb<16>(wkv_b, opart, lse, B, splits, O, status, st);
-  if (B <= 32) return launch_merge_nb<32>(wkv_b, opart, lse, B, splits, O, status, st);
-  if (B <= 64) return launch_merge_nb<64>(wkv_b, opart, lse, B, splits, O, status, st);
-  if (B <= 128) return launch_merge_nb<128>(wkv_b, opart, lse, B, splits, O, status, st);
-  return launch_merge_nb<256>(wkv_b, opart, lse, B, splits, O, status, st);
+                        int B, const core::Sched& sch, int slots, __nv_bfloat16* O,
+                        int32_t* status, cudaStream_t st) {
+  if (B <= 16) return launch_merge_nb<16>(wkv_b, opart, lse, B, sch, slots, O, status, st);
+  if (B <= 32) return launch_merge_nb<32>(wkv_b, opart, lse, B, sch, slots, O, status, st);
+  if (B <= 64) return launch_merge_nb<64>(wkv_b, opart, lse, B, sch, slots, O, status, st);
+  if (B <= 128) return launch_merge_nb<128>(wkv_b, opart, lse, B, sch, slots, O, status, st);
+  return launch_merge_nb<256>(wkv_b, opart, lse, B, sch, slots, O, status, st);
+}
+
+// The number of clusters is capped so that no batch row meets more than
+// kMaxSlots of them (only matters for very small B x k).
+static core::Sched schedule_for(int B, int k) {
+  int nc = max_clusters();
+  core::Sched s = make_sched(B, k, nc);
+  while (slots_of(s, B) > kMaxSlots && s.nc > 1) s = make_sched(B, k, s.nc - 1);
+  return s;
+}
+
+// 2-D tensor map over cache rows: dims {cols, rows}, row pitch rstride
+// elements, box {box_cols, 1} (one row high, as tile::gather4 requires).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+static int make_row_map(CUtensorMap* map, const void* base, int cols, unsigned long long rows,
+                        int rstride, int box_cols, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return MLA_ERR_CUDA;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)rstride * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)box_cols, 1};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
 static int check_cache_args(const void* c_kv, int64_t ckv_bstride, int ckv_rstride,
@@ -781,6 +983,11 @@ static int check_cache_args(const void* c_kv, int64_t ckv_bstride, int ckv_rstri
   if (!aligned16(c_kv) || !aligned16(k_pe) || (ckv_rstride % 8) || (kpe_rstride % 8) ||
       (ckv_bstride % 8) || (kpe_bstride % 8))
     return MLA_ERR_ALIGN;
+  // the gather addresses rows as b * (bstride / rstride) + t in both caches
+  if (ckv_bstride % ckv_rstride || kpe_bstride % kpe_rstride ||
+      ckv_bstride / ckv_rstride != kpe_bstride / kpe_rstride ||
+      (ckv_bstride != 0 && ckv_bstride / ckv_rstride < T))
+    return MLA_ERR_SHAPE;
   return MLA_OK;
 }
 
@@ -790,12 +997,13 @@ using namespace shla;
 
 extern "C" int mla_decode_num_splits(int B, int k) {
   if (B < 1 || k < 1) return 0;
-  return choose_splits(B, k, sm_count_or_default());
+  return slots_of(schedule_for(B, k), B);
 }
 
 extern "C" size_t mla_decode_workspace_bytes(int B, int k) {
   if (B < 1 || k < 1) return 0;
-  return ws_layout(B, choose_splits(B, k, sm_count_or_default())).total;
+  const core::Sched s = schedule_for(B, k);
+  return ws_layout(B, slots_of(s, B)).total;
 }
 
 extern "C" int mla_fold_wuk(const mla_bf16_t* q_nope, const mla_bf16_t* wkv_b, int B,
@@ -823,10 +1031,10 @@ static int decode_impl(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_
   if (!aligned16(q_nope) || !aligned16(q_pe) || !aligned16(wkv_b) || !aligned16(O))
     return MLA_ERR_ALIGN;
   if (!ws || !aligned256(ws)) return MLA_ERR_WORKSPACE;
-  int sms = 0;
-  if (int e = check_device(&sms)) return e;
-  const int splits = choose_splits(B, k, sms);
-  const WsLayout L = ws_layout(B, splits);
+  if (int e = check_device()) return e;
+  const core::Sched sch = schedule_for(B, k);
+  const int slots = slots_of(sch, B);
+  const WsLayout L = ws_layout(B, slots);
   if (ws_bytes < L.total) return MLA_ERR_WORKSPACE;
   cudaStream_t st = as_stream(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
@@ -843,32 +1051,32 @@ static int decode_impl(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_
   core::Params p;
   p.q_tilde = q_tilde;
   p.q_pe = reinterpret_cast<const __nv_bfloat16*>(q_pe);
-  p.c_kv = reinterpret_cast<const __nv_bfloat16*>(c_kv);
-  p.ckv_bs = ckv_bstride;
-  p.ckv_rs = ckv_rstride;
-  p.k_pe = reinterpret_cast<const __nv_bfloat16*>(k_pe);
-  p.kpe_bs = kpe_bstride;
-  p.kpe_rs = kpe_rstride;
+  p.rows_per_b = ckv_bstride / ckv_rstride;
   p.T = T;
   p.topk = topk;
   p.k = k;
   p.end_pos = end_pos;
   p.B = B;
-  p.ntiles = ntiles_of(k);
-  p.tiles_per_split = (p.ntiles + splits - 1) / splits;
-  p.splits = splits;
+  p.sch = sch;
+  p.slots = slots;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.opart = opart;
   p.lse = lse;
   p.status = status;
   if (phase == 0 || phase == 2) {
+    alignas(64) CUtensorMap map_c, map_r;
+    const unsigned long long rows = (unsigned long long)(B - 1) * p.rows_per_b + T;
+    if (int e = make_row_map(&map_c, c_kv, kC, rows, ckv_rstride, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+      return e;
+    if (int e = make_row_map(&map_r, k_pe, kR, rows, kpe_rstride, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+      return e;
     static unsigned long long core_attr = 0;
     if (int e = ensure_smem_attr(core_kernel, core::SMEM_BYTES, &core_attr)) return e;
-    core_kernel<<<dim3(2 * B * splits), core::NTHREADS, core::SMEM_BYTES, st>>>(p);
+    core_kernel<<<dim3(2 * sch.nc), core::NTHREADS, core::SMEM_BYTES, st>>>(p, map_c, map_r);
     if (int e = launch_status()) return e;
   }
   if (phase == 0 || phase == 3)
-    return launch_merge(reinterpret_cast<const __nv_bfloat16*>(wkv_b), opart, lse, B, splits,
+    return launch_merge(reinterpret_cast<const __nv_bfloat16*>(wkv_b), opart, lse, B, sch, slots,
                         reinterpret_cast<__nv_bfloat16*>(O), status, st);
   return MLA_OK;
 }
@@ -893,3 +1101,14 @@ extern "C" int mla_decode_phase(int phase, const mla_bf16_t* q_nope, const mla_b
                      kpe_bstride, kpe_rstride, T, topk, k, end_pos, B, scale, O, ws, ws_bytes,
                      status, stream);
 }
+
+#ifdef SHLA_TRACE
+extern "C" int mla_trace_read(void* host, size_t bytes) {
+  if (bytes < sizeof(shla::g_trace)) return MLA_ERR_SHAPE;
+  return cudaMemcpyFromSymbol(host, shla::g_trace, sizeof(shla::g_trace)) == cudaSuccess ? 0 : MLA_ERR_CUDA;
+}
+extern "C" int mla_trace_clear() {
+  static unsigned long long z[512][3][16];
+  return cudaMemcpyToSymbol(shla::g_trace, z, sizeof(z)) == cudaSuccess ? 0 : MLA_ERR_CUDA;
+}
+#endif
