@@ -71,7 +71,7 @@ const char* mla_status_string(int code);
 
 /*
  * Rotary embedding of feature pairs ("Rotated shared key" page,
- * apply_rotary_emb, model.py 405-425).
+ * the apply_rotary_emb code excerpt).
  *   x    bf16  [B, S, Hx, 64]
  *   rope fp32  [S, 32, 2]: (cos, sin) of the angle for sequence slot s and
  *              pair j; slot s of x uses row s (the caller offsets the table to
@@ -86,8 +86,9 @@ int mla_rope(const mla_bf16_t* x, const float* rope, int B, int S, int Hx, int i
              mla_bf16_t* y, void* stream);
 
 /*
- * Cache write for new positions ("KV compression" page, model.py 565-568,
- * and the cache write of 576 values per position, model.py 572-573):
+ * Cache write for new positions ("KV compression" page: the key-value
+ * down-projection code excerpt, and its Explanation of the 576 values cached
+ * per position):
  *   kv = x W_KVa (fp32 accumulation); latent = RMSNorm(kv[0:512]) * norm_w
  *   (y = v / sqrt(mean(v^2) + eps) * w, fp32); k_pe = interleaved RoPE of
  *   kv[512:576] at the row's position; both stored as bf16.
@@ -112,7 +113,7 @@ int mla_cache_write(const mla_bf16_t* x, const mla_bf16_t* w_kva, const mla_bf16
 
 /*
  * Absorbed sparse decode, one query per batch row ("Mix and project" page,
- * decode branch, model.py 590-606):
+ * decode ("MQA decode") code excerpt):
  *   q~[b,h,:]  = q_nope[b,h,:] W_UK[h]            W_UK[h] = wkv_b[h, 0:128, :]
  *   s[b,h,t]   = (q~[b,h,:].c_KV[b,t,:] + q_pe[b,h,:].k_pe[b,t,:]) * scale
  *                for t in the selected set of row b

@@ -12,16 +12,17 @@ rotary width and head dims are taken from the arguments) so that tests can
 run them on hand-sized problems.
 
 Sources (page title, section):
-  * "Mix and project" (decode branch, model.py 590-606): absorbed decode --
+  * "Mix and project" (the decode code excerpt): absorbed decode --
     fold W_UK into q_nope, score against the cached latent plus the shared
     rotary key over the indexer's selected positions, scale, softmax, mix
     the latent, apply W_UV per head.
-  * "Key heads" (equations k^C = c^KV W_UK, K_i = [K^C_i ; k^R]; prefill
-    listing, model.py 574-589): the materialised path used as a cross-check.
-  * "KV compression" (model.py 565-568) and "Rotated shared key"
-    (apply_rotary_emb, model.py 405-425): cache write and rotary embedding.
+  * "Key heads" (equations k^C = c^KV W_UK, K_i = [K^C_i ; k^R]; the
+    prefill code excerpt): the materialised path used as a cross-check.
+  * "KV compression" (the key-value down-projection excerpt) and "Rotated
+    shared key" (the apply_rotary_emb excerpt): cache write and rotary
+    embedding.
 
-Readings taken where the pages are silent (also listed in the design doc):
+Readings taken where the pages are silent:
   * index semantics follow the decode mask built by scatter of 0 into a -inf
     row over [0, end_pos): a position counts once however often it is
     listed; -1 is padding; any other index outside [0, end_pos) is ignored
@@ -218,7 +219,7 @@ def rope(x, R, interleaved=True):
 
 
 # ---------------------------------------------------------------------------
-# cache write ("KV compression", model.py 565-568)
+# cache write ("KV compression", key-value down-projection excerpt)
 # ---------------------------------------------------------------------------
 
 

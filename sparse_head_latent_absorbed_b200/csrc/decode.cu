@@ -1,5 +1,5 @@
-// Absorbed sparse MLA decode for sm_100a ("Mix and project" page, decode
-// branch, model.py 590-606).  Three kernels on the caller's stream:
+// Absorbed sparse MLA decode for sm_100a ("Mix and project" page, the decode
+// ("MQA decode") code excerpt).  Three kernels on the caller's stream:
 //
 //   fold_kernel      q~ = q_nope W_UK per head (tcgen05, latent as M, batch as N)
 //   core_kernel      persistent 2-CTA clusters over equal ranges of the
