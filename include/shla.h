@@ -112,6 +112,36 @@ int mla_cache_write(const mla_bf16_t* x, const mla_bf16_t* w_kva, const mla_bf16
                     void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * The cache write above without a workspace argument, for callers that
+ * cannot allocate device memory when they call it: code running inside
+ * callbacks of graph-based or embedding runtimes, decode loops whose runtime
+ * forbids allocation after start-up, and hosts whose device memory belongs to
+ * another allocator.  The pages describe no such variant; it exists only for
+ * those callers.
+ *
+ * The split-K partial products go to one fixed device array inside this
+ * library (MLA_NOALLOC_MAX_ROWS rows of partials, 4,128,768 bytes), which every
+ * GPU that loads the library holds until the process exits.  Arguments,
+ * layouts and results are those of mla_cache_write; B*S above
+ * MLA_NOALLOC_MAX_ROWS returns MLA_ERR_SHAPE without touching the GPU.  The
+ * function allocates nothing.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the array and it keeps the last call's contents;
+ * every value a call reads from it is written earlier in the same call, so
+ * nothing needs clearing, but calls that can overlap on the GPU (different
+ * streams, or different host threads) race on it and must be serialised by
+ * the caller.
+ */
+#define MLA_NOALLOC_MAX_ROWS 64
+int mla_cache_write_noalloc(const mla_bf16_t* x, const mla_bf16_t* w_kva,
+                            const mla_bf16_t* norm_w, float eps, const float* rope, int B, int S,
+                            int start_pos, mla_bf16_t* c_kv, int64_t ckv_bstride,
+                            int ckv_rstride, mla_bf16_t* k_pe, int64_t kpe_bstride,
+                            int kpe_rstride, int T, void* stream);
+
+/*
  * Absorbed sparse decode, one query per batch row ("Mix and project" page,
  * decode ("MQA decode") code excerpt):
  *   q~[b,h,:]  = q_nope[b,h,:] W_UK[h]            W_UK[h] = wkv_b[h, 0:128, :]

@@ -10,6 +10,7 @@ from ._lib import (  # noqa: F401
     LIB_PATH,
     MLAError,
     mla_cache_write,
+    mla_cache_write_noalloc,
     mla_cache_write_workspace_bytes,
     mla_decode,
     mla_decode_num_splits,

@@ -26,6 +26,8 @@ _SIGS = {
     "mla_cache_write": (_c_int, [_vp, _vp, _vp, _c_float, _vp, _c_int, _c_int, _c_int,
                                  _vp, _c_i64, _c_int, _vp, _c_i64, _c_int, _c_int,
                                  _vp, _c_size, _vp]),
+    "mla_cache_write_noalloc": (_c_int, [_vp, _vp, _vp, _c_float, _vp, _c_int, _c_int, _c_int,
+                                         _vp, _c_i64, _c_int, _vp, _c_i64, _c_int, _c_int, _vp]),
     "mla_decode_workspace_bytes": (_c_size, [_c_int, _c_int]),
     "mla_decode_num_splits": (_c_int, [_c_int, _c_int]),
     "mla_decode": (_c_int, [_vp, _vp, _vp, _vp, _c_i64, _c_int, _vp, _c_i64, _c_int, _c_int,
@@ -134,6 +136,27 @@ def mla_cache_write(x: torch.Tensor, w_kva: torch.Tensor, norm_w: torch.Tensor, 
                                B, S, int(start_pos), _p(c_kv), cbs, crs, _p(k_pe), kbs, krs,
                                cache.shape[1], _p(ws), ws.numel(), _stream(x.device)),
            "mla_cache_write")
+
+
+NOALLOC_MAX_ROWS = 64
+
+
+def mla_cache_write_noalloc(x: torch.Tensor, w_kva: torch.Tensor, norm_w: torch.Tensor,
+                            eps: float, rope: torch.Tensor, start_pos: int,
+                            cache: torch.Tensor) -> None:
+    """mla_cache_write without a workspace: for callers that cannot allocate
+    device memory at call time.  Uses the library's fixed scratch array
+    (at most NOALLOC_MAX_ROWS = B*S rows); calls that overlap on the GPU race
+    on that array."""
+    _need(x, torch.bfloat16, "x")
+    if x.dim() == 2:
+        x = x.unsqueeze(1)
+    B, S, _ = x.shape
+    c_kv, cbs, crs, k_pe, kbs, krs = _split_cache(cache)
+    _check(LIB.mla_cache_write_noalloc(_p(x.contiguous()), _p(w_kva), _p(norm_w), float(eps),
+                                       _p(rope), B, S, int(start_pos), _p(c_kv), cbs, crs,
+                                       _p(k_pe), kbs, krs, cache.shape[1], _stream(x.device)),
+           "mla_cache_write_noalloc")
 
 
 def mla_decode_workspace_bytes(B: int, k: int) -> int:

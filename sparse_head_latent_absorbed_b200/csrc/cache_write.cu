@@ -1,5 +1,6 @@
-// Cache write for new positions ("KV compression" page, model.py 565-568;
-// 576 cached values per position, model.py 572-573).
+// Cache write for new positions ("KV compression" page: the key-value
+// down-projection code excerpt, and its Explanation: 576 cached values per
+// position).
 //
 //   cw_gemm_kernel     split-K partial products of kv = x W_KVa on tcgen05:
 //                      D^T[o, r] = sum_i W_KVa[i][o] x[r][i] with the 576
@@ -9,6 +10,8 @@
 //                      (fp32), interleaved RoPE of the 64-wide rotary key at
 //                      the row's position, bf16 store into the cache.
 #include <math.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "host_util.h"
@@ -197,6 +200,84 @@ extern "C" int mla_cache_write(const mla_bf16_t* x, const mla_bf16_t* w_kva,
   else if (rows <= 64) e = launch_cw_gemm<64>(xb, wb, rows, part, st);
   else if (rows <= 128) e = launch_cw_gemm<128>(xb, wb, rows, part, st);
   else e = launch_cw_gemm<256>(xb, wb, rows, part, st);
+  if (e) return e;
+  cw_finalize_kernel<<<rows, 256, 0, st>>>(
+      part, rows, reinterpret_cast<const __nv_bfloat16*>(norm_w), eps, rope, S, start_pos,
+      reinterpret_cast<__nv_bfloat16*>(c_kv), ckv_bstride, ckv_rstride,
+      reinterpret_cast<__nv_bfloat16*>(k_pe), kpe_bstride, kpe_rstride);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the cache write.
+//
+// For callers that cannot allocate device memory at the point of the call:
+// code running inside CUDA graph node callbacks or other library callbacks,
+// runtimes that forbid allocation in their decode loop, and embedders whose
+// memory is owned by another allocator they cannot call into.  The split-K
+// partial products then go to a fixed, file-scope device array instead of a
+// caller workspace.
+//
+// The array holds partials for at most MLA_NOALLOC_MAX_ROWS rows
+// (28 x 64 x 576 floats = 4,128,768 bytes) on every GPU that loads this
+// library, until the process exits.  Its host-side name is only a stand-in:
+// the device address is looked up with cudaGetSymbolAddress once per device,
+// by the first call made with that device current.
+// ---------------------------------------------------------------------------
+namespace shla {
+namespace noalloc {
+constexpr int kMaxRows = MLA_NOALLOC_MAX_ROWS;
+static __device__ __align__(256) float g_scratch[cw::NKCH * kMaxRows * cw::kOut];
+
+static std::mutex g_mu;
+static float* g_addr[64] = {nullptr};
+
+// device address of g_scratch for the current device (set-up on first use)
+static int scratch_for_current_device(float** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MLA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return MLA_ERR_CUDA;
+    }
+    g_addr[dev] = static_cast<float*>(p);
+  }
+  *out = g_addr[dev];
+  return MLA_OK;
+}
+}  // namespace noalloc
+}  // namespace shla
+
+extern "C" int mla_cache_write_noalloc(const mla_bf16_t* x, const mla_bf16_t* w_kva,
+                                       const mla_bf16_t* norm_w, float eps, const float* rope,
+                                       int B, int S, int start_pos, mla_bf16_t* c_kv,
+                                       int64_t ckv_bstride, int ckv_rstride, mla_bf16_t* k_pe,
+                                       int64_t kpe_bstride, int kpe_rstride, int T,
+                                       void* stream) {
+  if (!x || !w_kva || !norm_w || !rope || !c_kv || !k_pe) return MLA_ERR_NULL;
+  if (B < 1 || S < 1 || (long long)B * S > noalloc::kMaxRows || T < 1 || start_pos < 0 ||
+      (long long)start_pos + S > T || ckv_rstride < 512 || kpe_rstride < 64 || ckv_bstride < 0 ||
+      kpe_bstride < 0 || !(eps >= 0.f))
+    return MLA_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(w_kva) || !aligned16(rope) || !aligned16(c_kv) ||
+      !aligned16(k_pe))
+    return MLA_ERR_ALIGN;
+  if (int e = check_device()) return e;
+  float* part = nullptr;
+  if (int e = noalloc::scratch_for_current_device(&part)) return e;
+  const int rows = B * S;
+  cudaStream_t st = as_stream(stream);
+  const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+  const __nv_bfloat16* wb = reinterpret_cast<const __nv_bfloat16*>(w_kva);
+  // every element of the partial buffer that the finalize step reads is
+  // written by the GEMM step of the same call, so nothing needs clearing
+  int e;
+  if (rows <= 16) e = launch_cw_gemm<16>(xb, wb, rows, part, st);
+  else if (rows <= 32) e = launch_cw_gemm<32>(xb, wb, rows, part, st);
+  else e = launch_cw_gemm<64>(xb, wb, rows, part, st);
   if (e) return e;
   cw_finalize_kernel<<<rows, 256, 0, st>>>(
       part, rows, reinterpret_cast<const __nv_bfloat16*>(norm_w), eps, rope, S, start_pos,
