@@ -361,6 +361,14 @@ DEV void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_
                : "memory");
 }
 
+// 32-bit read-only load issued where it stands (asm volatile keeps the
+// compiler from sinking it to its first use, so prefetches stay prefetches)
+DEV int ld_global_nc_s32_early(const int32_t* p) {
+  int v;
+  asm volatile("ld.global.nc.s32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
 DEV uint4 ld_global_nc_v4(const void* p) {
   uint4 v;
   asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"

@@ -141,28 +141,80 @@ __global__ void __launch_bounds__(128) fold_kernel(const __nv_bfloat16* __restri
 // [32r, 32r+32) of Q~ and of every selected cache row; both CTAs hold all 128
 // heads.  Per key tile (KT keys):
 //   S (partial)  = Q~_half K_half^T       M=128 heads, N=KT, K=288   (tcgen05)
-//   S            = S(own) + S(peer)      partials scaled to log2 units, rounded
-//                                        to fp16 and exchanged through DSMEM
-//   P            = 2^(S - m)             fp32 running max m and sum l
+//   S            = S(own) + S(peer)      partials scaled to log2 units (invalid
+//                                        keys -inf), rounded to fp16 and
+//                                        exchanged through DSMEM; added, maxed
+//                                        and exponentiated as fp16 pairs
+//   P            = 2^(S - m)             running max m; row sum l on the
+//                                        tensor core (P x ones)
 //   O_half      += P V_half              M=128, N=256, K=KT          (tcgen05)
 // V is the same shared-memory tile as K, read MN-major.
 //
-// Warp roles (256 threads):
-//   warps 0-3  softmax, one thread per head row (TMEM lane); they also load
-//              this CTA's half of Q~ into TMEM at each segment start and
-//              write the segment outputs
-//   warps 4-6  gather: TMA tile::gather4 of the selected rows (4 rows per
-//              instruction); group g of four keys goes to warp 4 + g % 3
-//   warp 7     TMEM owner and MMA issuer (one thread)
-// TMEM (512 columns): S [0,KT), Q~ half [64,208) as bf16 pairs, P [224,256)
-// as bf16 pairs, O half [256,512) fp32.
+// Warp roles (384 threads):
+//   warps 0-7  softmax: warps w and w+4 share the TMEM lanes 32(w%4).. (head
+//              rows) and take keys [0,32) / [32,64) of each tile; the two
+//              halves of a row combine their maxima through shared memory.
+//              They also load this CTA's half of Q~ into TMEM at each segment
+//              start and write the segment outputs
+//   warps 8-10 gather: TMA tile::gather4 of the selected rows (4 rows per
+//              instruction); group g of four keys goes to warp 8 + g % 3
+//   warp 11    TMEM owner and MMA issuer (one thread)
+// TMEM (512 columns): S [0,KT), Q~ half [64,208) as bf16 pairs, row sums
+// [208,224) (P times a ones tile, so l sums exactly the bf16 P the value
+// product uses), P [224,256) as bf16 pairs, O half [256,512) fp32.
 // ===========================================================================
+// packed fp16 pair helpers (low half = first element)
+DEV uint32_t f16x2_from_f32_sat(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+DEV uint32_t hadd2_u(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("add.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+DEV uint32_t hsub2_u(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+DEV uint32_t hmax2_u(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+DEV uint32_t hex2_u(uint32_t a) {  // 2^x of both halves (special-function unit)
+  uint32_t r;
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(a));
+  return r;
+}
+DEV float2 f16x2_to_f32x2(uint32_t h) {
+  float lo, hi;
+  asm("{.reg .f16 l, h; mov.b32 {l, h}, %2; cvt.f32.f16 %0, l; cvt.f32.f16 %1, h;}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(h));
+  return make_float2(lo, hi);
+}
+DEV uint32_t bf16x2_from_f32(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+DEV uint32_t f16x2_splat(float v) {  // v exactly representable in fp16
+  const __half hv = __float2half_rn(v);
+  const uint16_t b = *reinterpret_cast<const uint16_t*>(&hv);
+  return (uint32_t)b | ((uint32_t)b << 16);
+}
+
 namespace core {
 constexpr int KT = 64;                       // keys per tile
-constexpr int NST = 4;                       // gather ring depth
-constexpr int NTHREADS = 256;
+constexpr int NST = 5;                       // gather ring depth
+constexpr int NSOFT = 8;                     // softmax warps (two per TMEM lane quarter)
 constexpr int NGATHER = 3;                   // gather warps
-constexpr int MMA_WARP = 4 + NGATHER;
+constexpr int GATHER_WARP0 = NSOFT;
+constexpr int MMA_WARP = NSOFT + NGATHER;
+constexpr int NTHREADS = 32 * (MMA_WARP + 1);  // 384
 constexpr int ST_ATOM = KT * 128;            // one 64-column latent atom of a tile
 constexpr int ST_KR = 4 * ST_ATOM;           // rotary part of a tile (64 B swizzle)
 constexpr int ST_BYTES = ST_KR + KT * 64;    // 36864
@@ -170,17 +222,19 @@ constexpr int OFF_ST = 0;
 constexpr int OFF_XS = OFF_ST + NST * ST_BYTES;  // two buffers of exchanged partial scores
 constexpr int XS_STRIDE = KT * 2 + 16;           // padded fp16 row
 constexpr int XS_BYTES = 128 * XS_STRIDE;
-constexpr int OFF_END = OFF_XS + 2 * XS_BYTES;
+constexpr int OFF_ONES = OFF_XS + 2 * XS_BYTES;  // 16 x 64 bf16 ones (row sums on the tensor core)
+constexpr int OFF_BIAS = OFF_ONES + 2048;         // per softmax warp: 0 / -inf per key of its half tile
+constexpr int OFF_PMAX = OFF_BIAS + NSOFT * 32 * 4;   // [2 tile parities][2 halves][128 rows] partial maxima
+constexpr int OFF_END = OFF_PMAX + 2 * 2 * 128 * 4;
 constexpr int SMEM_BYTES = OFF_END + 1024;       // + alignment slack
 constexpr uint32_t XS_TX_BYTES = 128 * KT * 2;   // partial scores received per tile
 constexpr uint32_t GROUP_TX_BYTES = ST_BYTES / 16;  // bytes of one group of four keys
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t T_S = 0, T_Q = 64, T_P = 224, T_O = 256;
+constexpr uint32_t T_S = 0, T_Q = 64, T_L = 208, T_P = 224, T_O = 256;
 constexpr float kRescaleThreshold = 8.0f;        // log2 units
-constexpr float kExchangeClamp = 60000.f;        // fp16 exchange saturates here
-static_assert(ST_BYTES % 1024 == 0 && OFF_XS % 16 == 0, "alignment");
+static_assert(ST_BYTES % 1024 == 0 && OFF_XS % 16 == 0 && OFF_ONES % 1024 == 0, "alignment");
 static_assert(SMEM_BYTES + 512 <= 232448, "shared memory budget");
-static_assert(T_Q + 144 <= T_P && T_P + KT / 2 <= T_O, "TMEM plan");
+static_assert(T_Q + 144 <= T_L && T_L + 16 <= T_P && T_P + KT / 2 <= T_O, "TMEM plan");
 static_assert(KT / 4 == 16, "sixteen groups of four keys per tile");
 
 // Schedule: tiles [bnd(c), bnd(c+1)) of the flattened list belong to cluster c.
@@ -224,6 +278,13 @@ struct Bars {
 
 DEV bool key_valid(int v, int lim) { return v >= 0 && v < lim; }
 
+// Position of a tile in the flattened list, advanced one tile at a time
+// (no division in the loops): batch row, tile within the row, the row's
+// valid-position limit and the tile's indices (lane l: keys l and 32 + l).
+struct TileCur {
+  int bb, jt, lim, ilo, ihi;
+};
+
 }  // namespace core
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
@@ -243,9 +304,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
   const int nt = p.sch.nt;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sbase = smem_u32(smem);
-  auto row_of = [&](int i) { return (t_begin + i) / nt; };          // batch row of local tile i
-  auto seg_start = [&](int i) { return i == 0 || (t_begin + i) % nt == 0; };
-  auto lim_of = [&](int bb) { return min(p.end_pos[bb], p.T); };
+  const int bb0 = t_begin / nt, jt0 = t_begin - bb0 * nt;  // row / tile-in-row of tile 0
+  auto lim_of = [&](int bb) { return min(ld_global_nc_s32_early(p.end_pos + bb), p.T); };
+  // the tile after `c` (indices and limit loaded, not yet consumed)
+  auto advance = [&](const TileCur& c) {
+    TileCur d;
+    d.bb = c.bb;
+    d.jt = c.jt + 1;
+    d.lim = c.lim;
+    if (d.jt == nt) {
+      d.jt = 0;
+      ++d.bb;
+      d.lim = d.bb < p.B ? lim_of(d.bb) : 0;
+    }
+    d.ilo = d.ihi = -1;
+    if (d.bb < p.B) {
+      const int j = d.jt * KT + lane;
+      const int32_t* tk = p.topk + (size_t)d.bb * p.k;
+      d.ilo = j < p.k ? ld_global_nc_s32_early(tk + j) : -1;
+      d.ihi = j + 32 < p.k ? ld_global_nc_s32_early(tk + j + 32) : -1;
+    }
+    return d;
+  };
+  auto first_cur = [&]() {
+    TileCur c;
+    c.bb = bb0;
+    c.jt = jt0 - 1;  // advance() from the tile before
+    c.lim = lim_of(bb0);
+    c.ilo = c.ihi = -1;
+    return advance(c);
+  };
 
   if (warp == MMA_WARP) {
     tmem_alloc(&bars.tmem_base, TMEM_COLS);
@@ -257,13 +345,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       mbar_init(&bars.empty[s], 1);       // MMA commit after the tile's value product
     }
     mbar_init(&bars.s_full, 1);
-    mbar_init(&bars.s_empty, 128);
-    mbar_init(&bars.p_full, 128);
+    mbar_init(&bars.s_empty, 32 * NSOFT);
+    mbar_init(&bars.p_full, 32 * NSOFT);
     mbar_init(&bars.o_done, 1);
-    mbar_init(&bars.q_ready, 128);
+    mbar_init(&bars.q_ready, 32 * NSOFT);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.xs_full[i], 1);    // own expect_tx arrival + the peer's st.async bytes
-      mbar_init(&bars.xs_free[i], 4);    // one arrival per softmax warp of the peer
+      mbar_init(&bars.xs_full[i], 1);      // own expect_tx arrival + the peer's st.async bytes
+      mbar_init(&bars.xs_free[i], NSOFT);  // one arrival per softmax warp of the peer
     }
     mbar_init(&bars.drain, 1);
     bars.abort = 0;
@@ -271,39 +359,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     mbar_arrive_expect_tx(&bars.xs_full[0], XS_TX_BYTES);
     mbar_arrive_expect_tx(&bars.xs_full[1], XS_TX_BYTES);
   }
+  // the ones tile (bf16 1.0): any swizzle of it is the same tile
+  for (int i = tid; i < 2048 / 16; i += NTHREADS)
+    st_shared_v4(sbase + OFF_ONES + i * 16, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+  fence_proxy_async_smem();
   tc_fence_before();
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
 
-  if (warp >= 4 && warp < MMA_WARP) {
+  if (warp >= GATHER_WARP0 && warp < MMA_WARP) {
     // ---------------- gather (TMA tile::gather4) ----------------
     // lane l holds the index of key l and key 32 + l of the tile; lanes
     // 0..ng-1 each issue the five loads of one group of four keys
-    const int gw = warp - 4;
+    const int gw = warp - GATHER_WARP0;
     const int ng = (16 - gw + NGATHER - 1) / NGATHER;  // groups of this warp
     int bad = 0;
-    int va = -1, vb = -1;
-    auto load_idx = [&](int i) {
-      const int bb = row_of(i);
-      const int j = ((t_begin + i) - bb * nt) * KT + lane;
-      const int32_t* tk = p.topk + (size_t)bb * p.k;
-      va = j < p.k ? tk[j] : -1;
-      vb = j + 32 < p.k ? tk[j + 32] : -1;
-    };
-    load_idx(0);
+    TileCur cur = first_cur();
     SHLA_TRACE_DECL
 #pragma unroll 1
     for (int i = 0; i < n; ++i) {
       const int s = i % NST;
-      const int bb = row_of(i);
-      const int lim = lim_of(bb);
-      const bool oka = key_valid(va, lim), okb = key_valid(vb, lim);
-      if (rank == 0 && gw == 0) bad += (!oka && va != -1) + (!okb && vb != -1);
+      const bool oka = key_valid(cur.ilo, cur.lim), okb = key_valid(cur.ihi, cur.lim);
+      if (rank == 0 && gw == 0) bad += (!oka && cur.ilo != -1) + (!okb && cur.ihi != -1);
       // TMA rows: valid keys map to their cache row, others to row -1 (zero fill)
-      const int ra = oka ? (int)((long long)bb * p.rows_per_b + va) : -1;
-      const int rb = okb ? (int)((long long)bb * p.rows_per_b + vb) : -1;
-      if (i + 1 < n) load_idx(i + 1);
+      const int ra = oka ? (int)((long long)cur.bb * p.rows_per_b + cur.ilo) : -1;
+      const int rb = okb ? (int)((long long)cur.bb * p.rows_per_b + cur.ihi) : -1;
+      if (i + 1 < n) cur = advance(cur);
       SHLA_T(1);
       if (!warp_wait(&bars.empty[s], ((i / NST) & 1) ^ 1, abort, p.status)) break;
       SHLA_T(0);
@@ -345,7 +427,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, KT, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, 0, 1);
+      constexpr uint32_t idesc_l = idesc_bf16_f32(128, 16, 0, 0);
       int qk = 0, pv = 0, idle = 0, qseg = -1;
+      int jq = jt0, jp = jt0;  // tile-in-row of the next score / value product
       bool alive = true;
       uint64_t t_last = globaltimer_ns();
       SHLA_TRACE_DECL
@@ -356,22 +440,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
           tc_fence_after();
           const int s = pv % NST;
           const uint32_t st = sbase + OFF_ST + s * ST_BYTES;
-          const bool first = seg_start(pv);
+          const bool first = pv == 0 || jp == 0;
 #pragma unroll
           for (int ks = 0; ks < KT / 16; ++ks) {
             const uint64_t bd = smem_desc(st + ks * 2048, ST_ATOM, 1024, kSwizzle128B);
             tc_mma_tmem_a(tmem + T_O, tmem + T_P + ks * 8, bd, idesc_pv,
                           (!first || ks > 0) ? 1u : 0u);
           }
+          // row sums: l += P x ones (16 identical columns)
+#pragma unroll
+          for (int ks = 0; ks < KT / 16; ++ks) {
+            const uint64_t bd = smem_desc(sbase + OFF_ONES + ks * 32, 16, 1024, kSwizzle128B);
+            tc_mma_tmem_a(tmem + T_L, tmem + T_P + ks * 8, bd, idesc_l,
+                          (!first || ks > 0) ? 1u : 0u);
+          }
           tc_commit(&bars.o_done);
           tc_commit(&bars.empty[s]);
           ++pv;
+          if (++jp == nt) jp = 0;
           did = true;
           SHLA_T(1);
         }
         if (qk < n && mbar_test(&bars.full[qk % NST], (qk / NST) & 1) &&
             (qk == 0 || mbar_test(&bars.s_empty, (qk - 1) & 1))) {
-          const int seg = seg_start(qk) ? qseg + 1 : qseg;
+          const int seg = (qk == 0 || jq == 0) ? qseg + 1 : qseg;
           if (seg == qseg || mbar_test(&bars.q_ready, seg & 1)) {
             qseg = seg;
             tc_fence_after();
@@ -389,6 +481,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
             }
             tc_commit(&bars.s_full);
             ++qk;
+            if (++jq == nt) jq = 0;
             did = true;
             SHLA_T(2);
           }
@@ -414,77 +507,110 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     }
     __syncwarp();
   } else {
-    // ---------------- softmax (one thread per head row) ----------------
-    const int h = tid;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    // ---------------- softmax (two threads per head row) ----------------
+    const int quarter = warp & 3;             // TMEM lane quarter
+    const int half = warp >> 2;               // keys [32*half, 32*half + 32) of a tile
+    const int h = quarter * 32 + lane;        // head row = TMEM lane
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    constexpr int KH = KT / 2;                // keys per thread per tile
     // this CTA's half of Q~ (256 latent + 32 rotary values) of batch row bb
-    // into TMEM as bf16 pairs (9 stores of 16 columns), then q_ready
+    // into TMEM as bf16 pairs: chunks of 16 columns, 0-4 by the first half,
+    // 5-8 by the second; then q_ready
     auto load_q = [&](int bb) {
       const __nv_bfloat16* qrow = p.q_tilde + ((size_t)bb * kH + h) * kC + rank * 256;
       const __nv_bfloat16* rrow = p.q_pe + ((size_t)bb * kH + h) * kR + rank * 32;
+      const int c_lo = half ? 5 : 0, c_n = half ? 4 : 5;
+      uint4 q[5][4];
 #pragma unroll
-      for (int c = 0; c < 9; ++c) {
-        const __nv_bfloat16* src = c < 8 ? qrow + c * 32 : rrow;
-        uint32_t r[16];
+      for (int c = 0; c < 5; ++c) {
+        if (c < c_n) {
+          const int cc = c_lo + c;
+          const __nv_bfloat16* src = cc < 8 ? qrow + cc * 32 : rrow;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint4 q = ld_global_nc_v4(src + i * 8);
-          r[4 * i] = q.x;
-          r[4 * i + 1] = q.y;
-          r[4 * i + 2] = q.z;
-          r[4 * i + 3] = q.w;
+          for (int i = 0; i < 4; ++i) q[c][i] = ld_global_nc_v4(src + i * 8);
         }
-        tmem_st16(tmem + lane_base + T_Q + c * 16, r);
+      }
+#pragma unroll
+      for (int c = 0; c < 5; ++c) {
+        if (c < c_n) {
+          uint32_t r[16];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            r[4 * i] = q[c][i].x;
+            r[4 * i + 1] = q[c][i].y;
+            r[4 * i + 2] = q[c][i].z;
+            r[4 * i + 3] = q[c][i].w;
+          }
+          tmem_st16(tmem + lane_base + T_Q + (c_lo + c) * 16, r);
+        }
       }
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&bars.q_ready);
     };
-    load_q(row_of(0));
 
     // exchange buffer / barrier i sits at +i*XS_BYTES / +i*8 from buffer 0 in
-    // both CTAs, so the peer addresses follow from one mapa each
-    const uint32_t xs_row0 = sbase + OFF_XS + h * XS_STRIDE;
+    // both CTAs, so the peer addresses follow from one mapa each; this thread
+    // owns bytes [64*half, 64*half + 64) of its row
+    const uint32_t xs_row0 = sbase + OFF_XS + h * XS_STRIDE + half * 64;
     const uint32_t xs_peer_row0 = mapa_shared(xs_row0, peer);
     const uint32_t xs_full_peer0 = mapa_shared(smem_u32(&bars.xs_full[0]), peer);
     const uint32_t xs_free_peer0 = mapa_shared(smem_u32(&bars.xs_free[0]), peer);
-    float m_used = -INFINITY, l = 0.f;
-    uint32_t sa[KT / 2], sb[KT / 2];  // own scaled partial scores (fp16 pairs): current, next
+    const uint32_t bias_w = sbase + OFF_BIAS + warp * (32 * 4);
+    const uint32_t pmax_own = sbase + OFF_PMAX + (half * 128 + h) * 4;
+    const uint32_t pmax_other = sbase + OFF_PMAX + ((half ^ 1) * 128 + h) * 4;
+    const uint32_t pair_bar = 1 + quarter;    // named barrier of warps w and w+4
+    float m_used = -INFINITY;
+    uint32_t sa[KH / 2], sb[KH / 2];  // scaled partial scores as fp16 pairs: current, next
     bool alive = true;
     SHLA_TRACE_DECL
 
-    // own partial of tile t: TMEM -> scaled, fp16 -> the peer's exchange buffer
-    auto fetch_send = [&](int t, uint32_t (&dst)[KT / 2]) -> bool {
+    // own partial of tile t (position ct): TMEM -> x scale + (0 | -inf) per
+    // key -> fp16 pairs -> the peer's exchange buffer.  When the next tile
+    // (position cn) starts a new batch row, its Q~ replaces this one.
+    auto fetch_send = [&](int t, uint32_t (&dst)[KH / 2], const TileCur& ct,
+                          const TileCur& cn) -> bool {
       const int b2 = t & 1;
+      __syncwarp();
+      asm volatile("st.shared.f32 [%0], %1;" ::"r"(bias_w + lane * 4),
+                   "f"(key_valid(half ? ct.ihi : ct.ilo, ct.lim) ? 0.f : -INFINITY)
+                   : "memory");
+      __syncwarp();
       SHLA_T(11);
       if (!warp_wait(&bars.s_full, t & 1, abort, p.status)) return false;
       SHLA_T(0);
       tc_fence_after();
       {
-        uint32_t r[4][16];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld16(tmem + lane_base + T_S + c * 16, r[c]);
+        uint32_t r[2][16];
+        tmem_ld16(tmem + lane_base + T_S + half * KH, r[0]);
+        tmem_ld16(tmem + lane_base + T_S + half * KH + 16, r[1]);
         tc_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 2; ++c) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float x0 = fminf(fmaxf(__uint_as_float(r[c][2 * i]) * p.scale_log2, -kExchangeClamp), kExchangeClamp);
-            const float x1 = fminf(fmaxf(__uint_as_float(r[c][2 * i + 1]) * p.scale_log2, -kExchangeClamp), kExchangeClamp);
-            const __half2 hv = __floats2half2_rn(x0, x1);
-            dst[c * 8 + i] = *reinterpret_cast<const uint32_t*>(&hv);
+          for (int q = 0; q < 4; ++q) {
+            float4 bv;
+            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                         : "=f"(bv.x), "=f"(bv.y), "=f"(bv.z), "=f"(bv.w)
+                         : "r"(bias_w + (c * 16 + q * 4) * 4));
+            const float x0 = fmaf(__uint_as_float(r[c][4 * q]), p.scale_log2, bv.x);
+            const float x1 = fmaf(__uint_as_float(r[c][4 * q + 1]), p.scale_log2, bv.y);
+            const float x2 = fmaf(__uint_as_float(r[c][4 * q + 2]), p.scale_log2, bv.z);
+            const float x3 = fmaf(__uint_as_float(r[c][4 * q + 3]), p.scale_log2, bv.w);
+            dst[c * 8 + 2 * q] = f16x2_from_f32_sat(x0, x1);
+            dst[c * 8 + 2 * q + 1] = f16x2_from_f32_sat(x2, x3);
           }
+        }
       }
       tc_fence_before();
       mbar_arrive(&bars.s_empty);
-      // the next tile starts a new segment: its Q~ replaces this one (the score
-      // tile just read was the last product that used it)
-      if (t + 1 < n && seg_start(t + 1)) load_q(row_of(t + 1));
+      // (the score tile just read was the last product that used the old Q~)
+      if (t + 1 < n && cn.jt == 0) load_q(cn.bb);
       SHLA_T(1);
       if (!warp_wait<true>(&bars.xs_free[b2], ((t >> 1) & 1) ^ 1, abort, p.status)) return false;
       SHLA_T(2);
 #pragma unroll
-      for (int i = 0; i < KT / 2; i += 4)
+      for (int i = 0; i < KH / 2; i += 4)
         st_async_v4(xs_peer_row0 + b2 * XS_BYTES + i * 4, __uint_as_float(dst[i]),
                     __uint_as_float(dst[i + 1]), __uint_as_float(dst[i + 2]),
                     __uint_as_float(dst[i + 3]), xs_full_peer0 + b2 * 8);
@@ -492,19 +618,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       return true;
     };
 
-    // epilogue of a segment: this CTA's latent half of O~ / l into the
-    // segment's slot, and (rank 0) the row's log-sum-exp
-    auto flush = [&](int i_last) -> bool {
+    // epilogue of a segment: this thread's 128 columns of the CTA's latent
+    // half of O~ / l into the segment's slot, and (rank 0, first half) the
+    // row's log-sum-exp
+    auto flush = [&](int i_last, int bb) -> bool {
       if (!warp_wait(&bars.o_done, i_last & 1, abort, p.status)) return false;
       tc_fence_after();
-      const int bb = row_of(i_last);
       const int slot = cid - p.sch.c_first(bb);
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* dst = p.opart + (((size_t)bb * p.slots + slot) * kH + h) * kC + rank * 256;
       uint32_t r[16];
+      tmem_ld16(tmem + lane_base + T_L, r);
+      tc_wait_ld();
+      const float l = __uint_as_float(r[0]);
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* dst = p.opart + (((size_t)bb * p.slots + slot) * kH + h) * kC + rank * 256 +
+                           half * 128;
 #pragma unroll 1
-      for (int c = 0; c < 256; c += 16) {
-        tmem_ld16(tmem + lane_base + T_O + c, r);
+      for (int c = 0; c < 128; c += 16) {
+        tmem_ld16(tmem + lane_base + T_O + half * 128 + c, r);
         tc_wait_ld();
         uint4 lo, hi;
         lo.x = pack_bf16x2(__uint_as_float(r[0]) * inv, __uint_as_float(r[1]) * inv);
@@ -518,69 +648,62 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
         *reinterpret_cast<uint4*>(dst + c) = lo;
         *reinterpret_cast<uint4*>(dst + c + 8) = hi;
       }
-      if (rank == 0)
+      if (rank == 0 && half == 0)
         p.lse[((size_t)bb * p.slots + slot) * kH + h] = l > 0.f ? m_used + log2f(l) : -INFINITY;
       tc_fence_before();
       return true;
     };
 
-    auto tile_idx = [&](int i, int off) {
-      const int bb = row_of(i);
-      const int j = ((t_begin + i) - bb * nt) * KT + off + lane;
-      return j < p.k ? p.topk[(size_t)bb * p.k + j] : -1;
-    };
-    int vlo = tile_idx(0, 0), vhi = tile_idx(0, 32);
+    // tile positions: c0 = tile i, c1 = tile i + 1, c2 = tile i + 2
+    TileCur c0 = first_cur();
+    TileCur c1 = n > 1 ? advance(c0) : c0;
+    TileCur c2 = c1;
+    int prev_bb = c0.bb;
+    load_q(c0.bb);
 
-    // one key tile: `cur` holds this CTA's partial scores of tile i on entry;
-    // the next tile's partial is fetched into `nxt` and sent before the wait
-    auto step = [&](int i, uint32_t (&cur)[KT / 2], uint32_t (&nxt)[KT / 2]) -> bool {
-      const int lim = lim_of(row_of(i));
-      const uint32_t vmask_lo = __ballot_sync(0xffffffffu, key_valid(vlo, lim));
-      const uint32_t vmask_hi = __ballot_sync(0xffffffffu, key_valid(vhi, lim));
+    // one key tile: `cur` holds this thread's scaled partial scores of tile i
+    // on entry; the next tile's partial is fetched into `nxt` and sent first
+    auto step = [&](int i, uint32_t (&cur)[KH / 2], uint32_t (&nxt)[KH / 2]) -> bool {
       if (i + 1 < n) {
-        vlo = tile_idx(i + 1, 0);
-        vhi = tile_idx(i + 1, 32);
-        if (!fetch_send(i + 1, nxt)) return false;
+        c2 = i + 2 < n ? advance(c1) : c1;
+        SHLA_T(12);
+        if (!fetch_send(i + 1, nxt, c1, c2)) return false;
       }
       // add the peer's partial scores (other latent half) of this tile
       const int b2 = i & 1;
       SHLA_T(11);
       if (!warp_wait<true>(&bars.xs_full[b2], (i >> 1) & 1, abort, p.status)) return false;
       SHLA_T(4);
-      float sc[KT];
+      uint32_t mx2 = 0xFC00FC00u;  // (-inf, -inf)
 #pragma unroll
-      for (int c = 0; c < KT / 2; c += 4) {
+      for (int c = 0; c < KH / 2; c += 4) {
         uint4 o;
         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                      : "=r"(o.x), "=r"(o.y), "=r"(o.z), "=r"(o.w)
                      : "r"(xs_row0 + b2 * XS_BYTES + c * 4));
-        const uint32_t peer_w[4] = {o.x, o.y, o.z, o.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&cur[c + u]));
-          const float2 q = __half22float2(*reinterpret_cast<const __half2*>(&peer_w[u]));
-          sc[2 * (c + u)] = a.x + q.x;
-          sc[2 * (c + u) + 1] = a.y + q.y;
-        }
+        cur[c] = hadd2_u(cur[c], o.x);
+        cur[c + 1] = hadd2_u(cur[c + 1], o.y);
+        cur[c + 2] = hadd2_u(cur[c + 2], o.z);
+        cur[c + 3] = hadd2_u(cur[c + 3], o.w);
+        mx2 = hmax2_u(mx2, hmax2_u(hmax2_u(cur[c], cur[c + 1]), hmax2_u(cur[c + 2], cur[c + 3])));
       }
       // next use of this buffer (tile i + 2): expect the peer's bytes again
       if (tid == 0 && i + 2 < n) mbar_arrive_expect_tx(&bars.xs_full[b2], XS_TX_BYTES);
+      // row maximum of the tile: combine with the other half of the row
+      const float2 mxf = f16x2_to_f32x2(mx2);
+      const float mt_own = fmaxf(mxf.x, mxf.y);
+      asm volatile("st.shared.f32 [%0], %1;" ::"r"(pmax_own + b2 * 1024), "f"(mt_own) : "memory");
+      asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+      float mt_other;
+      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(mt_other) : "r"(pmax_other + b2 * 1024) : "memory");
+      const float mt = fmaxf(mt_own, mt_other);
       SHLA_T(5);
 
-      // a new segment: write out the previous one and restart the running sums
-      const bool first = seg_start(i);
+      // a new segment: write out the previous one and restart the running max
+      const bool first = i == 0 || c0.jt == 0;
       if (first && i > 0) {
-        if (!flush(i - 1)) return false;
+        if (!flush(i - 1, prev_bb)) return false;
         m_used = -INFINITY;
-        l = 0.f;
-      }
-      // mask and running max (scores are already in log2 units)
-      float mt = -INFINITY;
-#pragma unroll
-      for (int u = 0; u < KT; ++u) {
-        const uint32_t bit = u < 32 ? (vmask_lo >> u) & 1u : (vmask_hi >> (u - 32)) & 1u;
-        sc[u] = bit ? sc[u] : -INFINITY;
-        mt = fmaxf(mt, sc[u]);
       }
       const float m_new = fmaxf(m_used, mt);
       const bool rescale = m_new > m_used + kRescaleThreshold;
@@ -590,14 +713,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
         tc_fence_after();
       }
       SHLA_T(7);
-      const float alpha = rescale ? fast_exp2(m_used - m_new) : 1.f;
-      l *= alpha;
       if (!first && __any_sync(0xffffffffu, rescale)) {
-        // warp-collective: rows that keep their maximum scale by 1
+        // warp-collective over this thread's 128 accumulator columns (and the
+        // row sums, first half): rows that keep their maximum scale by 1
+        const float alpha = rescale ? fast_exp2(m_used - m_new) : 1.f;
         uint32_t r[16];
 #pragma unroll 1
-        for (int c = 0; c < 256; c += 16) {
-          const uint32_t ta = tmem + lane_base + T_O + c;
+        for (int c = half ? 0 : -16; c < 128; c += 16) {
+          const uint32_t ta = tmem + lane_base + (c < 0 ? T_L : T_O + half * 128 + c);
           tmem_ld16(ta, r);
           tc_wait_ld();
 #pragma unroll
@@ -607,43 +730,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       }
       if (rescale) m_used = m_new;
       SHLA_T(8);
-      // P = 2^(s - m) as bf16 pairs into TMEM; the row sum adds the rounded values
+      // P = 2^(s - m) on fp16 pairs, stored to TMEM as bf16 pairs
       const bool live = m_used != -INFINITY;
-      float ps[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < KT / 32; ++c) {
+      const uint32_t m2 = live ? f16x2_splat(m_used) : 0u;
+      {
         uint32_t w[16];
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
-          const float e0 = live ? fast_exp2(sc[c * 32 + 2 * u] - m_used) : 0.f;
-          const float e1 = live ? fast_exp2(sc[c * 32 + 2 * u + 1] - m_used) : 0.f;
-          const __nv_bfloat162 pr = __floats2bfloat162_rn(e0, e1);
-          const float2 back = __bfloat1622float2(pr);
-          ps[u & 3] += back.x + back.y;
-          w[u] = *reinterpret_cast<const uint32_t*>(&pr);
+          if (live) {
+            const float2 e = f16x2_to_f32x2(hex2_u(hsub2_u(cur[u], m2)));
+            w[u] = bf16x2_from_f32(e.x, e.y);
+          } else {
+            w[u] = 0u;
+          }
         }
-        tmem_st16(tmem + lane_base + T_P + c * 16, w);
+        tmem_st16(tmem + lane_base + T_P + half * 16, w);
       }
-      l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&bars.p_full);
-      // this tile's exchange buffer can take the peer's tile i + 2
+      // this tile's exchange buffer can take the peer's tile i + 2 (its reads
+      // completed above)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster_relaxed(xs_free_peer0 + b2 * 8);
+      prev_bb = c0.bb;
+      c0 = c1;
+      c1 = c2;
       SHLA_T(9);
       return true;
     };
 
-    alive = fetch_send(0, sa);
+    alive = fetch_send(0, sa, c0, c1);
 #pragma unroll 1
-    for (int i = 0; i < n && alive; i += 2) {
+    for (int i = 0; i < n && alive; ++i) {
       if (!step(i, sa, sb)) { alive = false; break; }
-      if (i + 1 < n && !step(i + 1, sb, sa)) { alive = false; break; }
+#pragma unroll
+      for (int u = 0; u < KH / 2; ++u) sa[u] = sb[u];
     }
     SHLA_T(10);
     if (lane == 0) SHLA_TRACE_FLUSH(0);
-    if (__all_sync(0xffffffffu, alive && !*abort)) flush(n - 1);
+    if (__all_sync(0xffffffffu, alive && !*abort)) flush(n - 1, prev_bb);
   }
 
   tc_fence_before();
