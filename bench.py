@@ -22,9 +22,8 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -123,58 +122,96 @@ def barrier(world: int):
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clocks and clock-event (throttle) reasons, polled through NVML from a
+    background thread every few milliseconds while the timed steps run.
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    Only reads the device state; nothing here changes a clock or a limit.
+    `wait_live()` returns once the first sample is in, so that a short timed
+    region is still covered."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
-    def __enter__(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
+    def __init__(self, device, period_s: float = 0.005):
+        self.device = device
+        self.period = period_s
+        self.rows = []          # (sm_mhz, max_mhz, reasons bitmask, power_w)
+        self.error = None
+        self._stop = threading.Event()
+        self._live = threading.Event()
+        self._thread = None
+
+    def _handle(self, nv):
+        import torch
+        props = torch.cuda.get_device_properties(self.device)
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-i", str(self.gpu), "-lms", "100"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            return nv.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
         except Exception:
-            self.proc = None
-        return self
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
 
-    def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-
-    def summary(self):
-        rows = []
+    def _run(self):
         try:
-            with open(self.path) as f:
-                for line in f:
-                    parts = [p.strip() for p in line.split(",")]
-                    if len(parts) >= 9:
-                        rows.append(parts)
+            import pynvml as nv
+            nv.nvmlInit()
+        except Exception as e:  # no NVML: the line says so
+            self.error = f"nvml unavailable: {e}"
+            self._live.set()
+            return
+        try:
+            h = self._handle(nv)
+            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            while not self._stop.is_set():
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                try:
+                    pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                except Exception:
+                    pw = None
+                self.rows.append((sm, mx, rs, pw))
+                self._live.set()
+                self._stop.wait(self.period)
+        except Exception as e:
+            self.error = f"nvml query failed: {e}"
+            self._live.set()
         finally:
             try:
-                os.unlink(self.path)
+                nv.nvmlShutdown()
             except Exception:
                 pass
+
+    def __enter__(self):
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+        return self
+
+    def wait_live(self, timeout_s: float = 10.0):
+        self._live.wait(timeout_s)
+
+    def mark(self):
+        """Index of the next sample: samples from here on fall in the region."""
+        return len(self.rows)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
+
+    def summary(self, start: int = 0):
+        rows = self.rows[start:]
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
-                "samples": len(rows)}
+            return {"sm_mhz": None, "sm_max_mhz": None,
+                    "reasons": [self.error or "no samples"], "samples": 0}
+        import pynvml as nv
+        reasons = sorted({name for _, _, rs, _ in rows for name, const in self.REASONS
+                          if rs & getattr(nv, const, 0)})
+        pw = [r[3] for r in rows if r[3] is not None]
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows), "source": "nvml",
+                "power_w_median": statistics.median(pw) if pw else None}
 
 
 # ---------------------------------------------------------------------------
@@ -300,17 +337,19 @@ def run_ours(args):
         shla.mla_decode(wl.q_nope, wl.q_pe, wl.wkv_b, wl.cache, wl.topk, wl.end_pos, wl.scale,
                         out=out, ws=ws, status=status)
 
-    launches_per_step = 3 + (2 if write else 0)
-    smi_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0]) \
-        if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local
+    # fold, attend, W_UV; the combine kernel runs when rows are split
+    launches_per_step = 3 + (1 if shla.mla_decode_num_splits(B, k) > 1 else 0) \
+        + (2 if write else 0)
 
     # ---- device-timed steps ----
-    with ClockSampler(smi_index) as clk:
+    with ClockSampler(dev) as clk:
         for _ in range(args.warmup):
             flush.zero_()
             step()
         torch.cuda.synchronize()
+        clk.wait_live()
         barrier(world)
+        clk_start = clk.mark()
         starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         for i in range(args.steps):
@@ -320,7 +359,7 @@ def run_ours(args):
             ends[i].record(stream)
         torch.cuda.synchronize()
         barrier(world)
-    clocks = clk.summary()
+    clocks = clk.summary(clk_start)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = reduce_max(sum(step_ms), world, dev)
     ms_per_step = total_ms / args.steps

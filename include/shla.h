@@ -176,11 +176,13 @@ int mla_decode(const mla_bf16_t* q_nope, const mla_bf16_t* q_pe, const mla_bf16_
                mla_bf16_t* O, void* ws, size_t ws_bytes, int32_t* status, void* stream);
 
 /*
- * The same call split into its three launches, for timing one of them alone:
+ * The same call split into its three phases, for timing one of them alone:
  *   phase 1: fold of W_UK into the queries (writes q~ into ws)
- *   phase 2: gather + scores + softmax + latent mix per key split (reads q~,
- *            writes the per-split partial outputs into ws)
- *   phase 3: merge of the splits and W_UV (reads ws, writes O)
+ *   phase 2: gather + scores + softmax + latent mix (reads q~; writes the
+ *            mixed latent O~ of each row held by one cluster, and the
+ *            partial O~ and log-sum-exp of each segment of a split row, into ws)
+ *   phase 3: log-sum-exp merge of the split rows (one launch, skipped when no
+ *            row is split), then O = O~ W_UV^T (reads ws, writes O)
  *   phase 0: all three (identical to mla_decode)
  * Phases must run in order on one stream with the same arguments and
  * workspace; each phase alone leaves O undefined until phase 3 has run.

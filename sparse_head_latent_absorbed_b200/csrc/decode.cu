@@ -9,9 +9,9 @@
 //                    columns [256r, 256r+256) and rotary columns [32r, 32r+32);
 //                    the two partial score tiles are summed through
 //                    distributed shared memory.
-//   merge_uv_kernel  log-sum-exp merge of the partial outputs of each row,
-//                    then O = O~ W_UV^T per head (tcgen05, value dim as M,
-//                    batch as N)
+//   combine_kernel   log-sum-exp merge of the rows split across clusters
+//   uv_kernel        O = O~ W_UV^T per head on the merged O~ (tcgen05, value
+//                    dim as M, batch as N)
 #include <cuda_fp16.h>
 #include <math.h>
 
@@ -104,8 +104,11 @@ __global__ void __launch_bounds__(128) fold_kernel(const __nv_bfloat16* __restri
   __syncwarp();
   const bool ok = warp_wait(&bar, 0, nullptr, status);
   tc_fence_after();
+  // epilogue: D^T[c][b] through shared memory (reusing the operand area) as
+  // [b][128 c] bf16 rows, then 16-byte stores of q~[b][h][ct*128 ..]
+  const uint32_t stage = sA;
   if (ok) {
-    const int c = ct * 128 + warp * 32 + lane;
+    const int cl = warp * 32 + lane;  // this thread's c within the tile
 #pragma unroll 1
     for (int n0 = 0; n0 < NB; n0 += 16) {
       uint32_t r[16];
@@ -113,13 +116,26 @@ __global__ void __launch_bounds__(128) fold_kernel(const __nv_bfloat16* __restri
       tc_wait_ld();
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const int b = b0 + n0 + j;
-        if (b < B)
-          q_tilde[((size_t)b * kH + h) * kC + c] = __float2bfloat16_rn(__uint_as_float(r[j]));
+        const __nv_bfloat16 v = __float2bfloat16_rn(__uint_as_float(r[j]));
+        asm volatile("st.shared.b16 [%0], %1;" ::"r"(stage + (n0 + j) * 256 + cl * 2),
+                     "h"(*reinterpret_cast<const unsigned short*>(&v))
+                     : "memory");
       }
     }
   }
   tc_fence_before();
+  __syncthreads();
+  if (ok) {
+    for (int q = tid; q < NB * 16; q += 128) {
+      const int nn = q >> 4, ch = q & 15, b = b0 + nn;
+      if (b >= B) continue;
+      uint4 v;
+      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                   : "r"(stage + nn * 256 + ch * 16));
+      *reinterpret_cast<uint4*>(q_tilde + ((size_t)b * kH + h) * kC + ct * 128 + ch * 8) = v;
+    }
+  }
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
@@ -266,6 +282,7 @@ struct Params {
   float scale_log2;               // softmax scale * log2(e)
   __nv_bfloat16* opart;           // [B][slots][128][512], normalised per segment
   float* lse;                     // [B][slots][128], log2 units of scaled scores
+  __nv_bfloat16* omerged;         // [B][128][512]: O~ of rows held by a single cluster
   int32_t* status;
 };
 
@@ -624,14 +641,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     auto flush = [&](int i_last, int bb) -> bool {
       if (!warp_wait(&bars.o_done, i_last & 1, abort, p.status)) return false;
       tc_fence_after();
-      const int slot = cid - p.sch.c_first(bb);
+      const int cf = p.sch.c_first(bb);
+      const int used = p.sch.c_last(bb) - cf + 1;  // clusters holding a segment of row bb
+      const int slot = cid - cf;
       uint32_t r[16];
       tmem_ld16(tmem + lane_base + T_L, r);
       tc_wait_ld();
       const float l = __uint_as_float(r[0]);
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* dst = p.opart + (((size_t)bb * p.slots + slot) * kH + h) * kC + rank * 256 +
-                           half * 128;
+      // a row held by one cluster is final here; otherwise this is one segment
+      // of the row, merged by combine_kernel
+      __nv_bfloat16* dst =
+          (used == 1 ? p.omerged + ((size_t)bb * kH + h) * kC
+                     : p.opart + (((size_t)bb * p.slots + slot) * kH + h) * kC) +
+          rank * 256 + half * 128;
 #pragma unroll 1
       for (int c = 0; c < 128; c += 16) {
         tmem_ld16(tmem + lane_base + T_O + half * 128 + c, r);
@@ -648,9 +671,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
         *reinterpret_cast<uint4*>(dst + c) = lo;
         *reinterpret_cast<uint4*>(dst + c + 8) = hi;
       }
-      if (rank == 0 && half == 0)
-        p.lse[((size_t)bb * p.slots + slot) * kH + h] = l > 0.f ? m_used + log2f(l) : -INFINITY;
       tc_fence_before();
+      if (used > 1 && rank == 0 && half == 0)
+        p.lse[((size_t)bb * p.slots + slot) * kH + h] = l > 0.f ? m_used + log2f(l) : -INFINITY;
       return true;
     };
 
@@ -783,29 +806,82 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
 }
 
 // ===========================================================================
-// K3: merge the partial outputs of each batch row and apply W_UV.
-//   O~[b,h,:] = sum_s w_s O~_s,  w_s = 2^(lse_s - max) / sum   (log-sum-exp merge)
+// K3a: merge the segments of the rows that more than one cluster held
+//   O~[b,h,:] = sum_s 2^(lse_s - max) O~_s / sum_s 2^(lse_s - max)
+// grid (B rows, 8 groups of 16 heads); 256 threads, 4 x 16 bytes each per
+// segment; rows held by one cluster were written final by the attend kernel.
+// ===========================================================================
+__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ opart,
+                                                       const float* __restrict__ lse,
+                                                       core::Sched sch, int slots,
+                                                       __nv_bfloat16* __restrict__ omerged) {
+  const int b = blockIdx.x;
+  const int used = sch.c_last(b) - sch.c_first(b) + 1;
+  if (used <= 1) return;
+  const int h = blockIdx.y * 16 + (threadIdx.x >> 4);
+  const int c0 = (threadIdx.x & 15) * 8;  // chunks c0, c0 + 128, c0 + 256, c0 + 384
+  const float* lse_b = lse + (size_t)b * slots * kH + h;
+  float mx = -INFINITY;
+  for (int s = 0; s < used; ++s) mx = fmaxf(mx, lse_b[(size_t)s * kH]);
+  float acc[4][8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
+  float wsum = 0.f;
+  const __nv_bfloat16* src = opart + ((size_t)b * slots * kH + h) * kC + c0;
+#pragma unroll 1
+  for (int s = 0; s < used; ++s) {
+    const float w = mx == -INFINITY ? 0.f : exp2f(lse_b[(size_t)s * kH] - mx);
+    wsum += w;
+    uint4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = ld_global_nc_v4(src + (size_t)s * kH * kC + j * 128);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&v[j]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(pv[e]);
+        acc[j][2 * e] += w * f.x;
+        acc[j][2 * e + 1] += w * f.y;
+      }
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  __nv_bfloat16* out = omerged + ((size_t)b * kH + h) * kC + c0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint4 o;
+    o.x = pack_bf16x2(acc[j][0] * inv, acc[j][1] * inv);
+    o.y = pack_bf16x2(acc[j][2] * inv, acc[j][3] * inv);
+    o.z = pack_bf16x2(acc[j][4] * inv, acc[j][5] * inv);
+    o.w = pack_bf16x2(acc[j][6] * inv, acc[j][7] * inv);
+    *reinterpret_cast<uint4*>(out + j * 128) = o;
+  }
+}
+
+// ===========================================================================
+// K3: O = O~ W_UV^T per head, on the merged O~ of each row.
 //   D^T[d, b] = sum_c W_UV[h][d][c] O~[b][h][c]
 //   A = W_UV[h] (M = 128 value dims, K = c), K-major
-//   B = merged O~ rows (N = batch rows, K = c), K-major, built in shared memory
-// grid (128 heads, batch blocks of NB); 256 threads; K in 4 chunks of 128.
+//   B = O~ rows (N = batch rows, K = c), K-major
+// grid (128 heads, batch blocks of NB); 128 threads; K in 4 chunks of 128,
+// double-buffered (cp.async for chunk k+2 while the MMAs of chunk k run).
 // ===========================================================================
 constexpr int kMaxSlots = 32;
 
 template <int NB>
-__global__ void __launch_bounds__(256) merge_uv_kernel(const __nv_bfloat16* __restrict__ wkv_b,
-                                                        const __nv_bfloat16* __restrict__ opart,
-                                                        const float* __restrict__ lse, int B,
-                                                        core::Sched sch, int slots,
-                                                        __nv_bfloat16* __restrict__ O,
-                                                        int32_t* status) {
+__global__ void __launch_bounds__(128) uv_kernel(const __nv_bfloat16* __restrict__ wkv_b,
+                                                  const __nv_bfloat16* __restrict__ omerged,
+                                                  int B, __nv_bfloat16* __restrict__ O,
+                                                  int32_t* status) {
   constexpr uint32_t NCOLS = NB <= 32 ? 32 : NB;
+  constexpr uint32_t BUF = 32768 + NB * 256;        // one chunk: A [2 katoms][128][128 B] + B
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  const uint32_t sA = smem_u32(smem);               // [2 katoms][128 d][128 B] = 32 KB
-  const uint32_t sB = sA + 32768;                   // [2 katoms][NB][128 B]
-  float* wts = reinterpret_cast<float*>(smem + 32768 + NB * 256);   // [NB][slots]
-  __shared__ uint64_t bar;
+  const uint32_t s0 = smem_u32(smem);
+  __shared__ uint64_t bar[2];
   __shared__ uint32_t tmem_base;
   const int h = blockIdx.x, b0 = blockIdx.y * NB;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -815,28 +891,28 @@ __global__ void __launch_bounds__(256) merge_uv_kernel(const __nv_bfloat16* __re
     tmem_relinquish();
   }
   if (tid == 0) {
-    mbar_init(&bar, 1);
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
     fence_mbarrier_init_cluster();
   }
-  // merge weights of the slots used by each row (others 0)
-  for (int nn = tid; nn < NB; nn += 256) {
-    const int b = b0 + nn;
-    float* w = wts + nn * slots;
-    for (int s = 0; s < slots; ++s) w[s] = 0.f;
-    if (b >= B) continue;
-    const int used = sch.c_last(b) - sch.c_first(b) + 1;
-    float mx = -INFINITY;
-    for (int s = 0; s < used; ++s) mx = fmaxf(mx, lse[((size_t)b * slots + s) * kH + h]);
-    if (mx == -INFINITY) continue;
-    float sum = 0.f;
-    for (int s = 0; s < used; ++s) {
-      const float e = exp2f(lse[((size_t)b * slots + s) * kH + h] - mx);
-      w[s] = e;
-      sum += e;
+  auto load_chunk = [&](int kc) {
+    const uint32_t sA = s0 + (kc & 1) * BUF, sB = sA + 32768;
+    for (int q = tid; q < 128 * 16; q += 128) {
+      const int d = q >> 4, ch = q & 15;
+      cp_async_16(sA + (ch >> 3) * 16384 + sw128_off(d, ch & 7),
+                  wkv_b + ((size_t)h * 256 + kDn + d) * kC + kc * 128 + ch * 8, 16);
     }
-    const float inv = 1.f / sum;
-    for (int s = 0; s < used; ++s) w[s] *= inv;
-  }
+    for (int q = tid; q < NB * 16; q += 128) {
+      const int nn = q >> 4, ch = q & 15, b = b0 + nn;
+      const bool in = b < B;
+      cp_async_16(sB + (ch >> 3) * (NB * 128) + sw128_off(nn, ch & 7),
+                  omerged + ((size_t)(in ? b : 0) * kH + h) * kC + kc * 128 + ch * 8,
+                  in ? 16u : 0u);
+    }
+    cp_async_commit();
+  };
+  load_chunk(0);
+  load_chunk(1);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -844,66 +920,14 @@ __global__ void __launch_bounds__(256) merge_uv_kernel(const __nv_bfloat16* __re
   bool ok = true;
 #pragma unroll 1
   for (int kc = 0; kc < 4; ++kc) {
-    if (kc > 0) {
-      ok = warp_wait(&bar, (kc - 1) & 1, nullptr, status) && ok;
-      tc_fence_after();
-    }
-    for (int q = tid; q < 128 * 16; q += 256) {
-      const int d = q >> 4, ch = q & 15;
-      cp_async_16(sA + (ch >> 3) * 16384 + sw128_off(d, ch & 7),
-                  wkv_b + ((size_t)h * 256 + kDn + d) * kC + kc * 128 + ch * 8, 16);
-    }
-    // merged O~ chunk: 4 independent 16-byte items per thread in flight
-#pragma unroll 1
-    for (int q0 = tid; q0 < NB * 16; q0 += 256 * 4) {
-      float acc[4][8];
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
-#pragma unroll 1
-      for (int s = 0; s < slots; ++s) {
-        uint4 v[4];
-        float w[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int q = q0 + 256 * u;
-          const int nn = q >> 4, ch = q & 15, b = b0 + nn;
-          w[u] = (q < NB * 16 && b < B) ? wts[nn * slots + s] : 0.f;
-          v[u] = make_uint4(0, 0, 0, 0);
-          if (w[u] != 0.f)
-            v[u] = ld_global_nc_v4(opart + (((size_t)b * slots + s) * kH + h) * kC + kc * 128 +
-                                   ch * 8);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 f = __bfloat1622float2(pv[i]);
-            acc[u][2 * i] += w[u] * f.x;
-            acc[u][2 * i + 1] += w[u] * f.y;
-          }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int q = q0 + 256 * u;
-        if (q < NB * 16) {
-          const int nn = q >> 4, ch = q & 15;
-          st_shared_v4(sB + (ch >> 3) * (NB * 128) + sw128_off(nn, ch & 7),
-                       pack_bf16x2(acc[u][0], acc[u][1]), pack_bf16x2(acc[u][2], acc[u][3]),
-                       pack_bf16x2(acc[u][4], acc[u][5]), pack_bf16x2(acc[u][6], acc[u][7]));
-        }
-      }
-    }
-    cp_async_wait_all();
+    if (kc < 3) cp_async_wait<1>(); else cp_async_wait<0>();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (tid == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, NB, 0, 0);
+      const uint32_t sA = s0 + (kc & 1) * BUF, sB = sA + 32768;
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         const uint64_t ad = smem_desc(sA + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSwizzle128B);
@@ -911,30 +935,51 @@ __global__ void __launch_bounds__(256) merge_uv_kernel(const __nv_bfloat16* __re
             smem_desc(sB + (ks >> 2) * (NB * 128) + (ks & 3) * 32, 16, 1024, kSwizzle128B);
         tc_mma(tmem, ad, bd, idesc, (kc > 0 || ks > 0) ? 1u : 0u);
       }
-      tc_commit(&bar);
+      tc_commit(&bar[kc & 1]);
     }
     __syncwarp();
+    if (kc + 2 < 4) {
+      // buffer kc&1 is refilled once the MMAs that read it are done
+      ok = warp_wait(&bar[kc & 1], (kc >> 1) & 1, nullptr, status) && ok;
+      load_chunk(kc + 2);
+    }
   }
-  ok = warp_wait(&bar, 1, nullptr, status) && ok;
+  // last two commits: chunk 2 (bar[0], phase 1) and chunk 3 (bar[1], phase 1)
+  ok = warp_wait(&bar[0], 1, nullptr, status) && ok;
+  ok = warp_wait(&bar[1], 1, nullptr, status) && ok;
   tc_fence_after();
+  // epilogue: D^T[d][b] through shared memory as [b][128 d] bf16 rows, then
+  // 16-byte stores of O[b][h][:]
+  const uint32_t stage = s0;
   if (ok) {
-    // warps w and w+4 share TMEM lanes 32(w%4).. and split the columns
-    const int d = (warp & 3) * 32 + lane;
-    const int half = warp >> 2;
-    constexpr int PER = NB / 2 < 16 ? 16 : NB / 2;
+    const int d = warp * 32 + lane;
 #pragma unroll 1
-    for (int n0 = half * PER; n0 < NB && n0 < (half + 1) * PER; n0 += 16) {
+    for (int n0 = 0; n0 < NB; n0 += 16) {
       uint32_t r[16];
-      tmem_ld16(tmem + ((uint32_t)((warp & 3) * 32) << 16) + n0, r);
+      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + n0, r);
       tc_wait_ld();
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const int b = b0 + n0 + j;
-        if (b < B) O[((size_t)b * kH + h) * kDv + d] = __float2bfloat16_rn(__uint_as_float(r[j]));
+        const __nv_bfloat16 v = __float2bfloat16_rn(__uint_as_float(r[j]));
+        asm volatile("st.shared.b16 [%0], %1;" ::"r"(stage + (n0 + j) * 256 + d * 2),
+                     "h"(*reinterpret_cast<const unsigned short*>(&v))
+                     : "memory");
       }
     }
   }
   tc_fence_before();
+  __syncthreads();
+  if (ok) {
+    for (int q = tid; q < NB * 16; q += 128) {
+      const int nn = q >> 4, ch = q & 15, b = b0 + nn;
+      if (b >= B) continue;
+      uint4 v;
+      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                   : "r"(stage + nn * 256 + ch * 16));
+      *reinterpret_cast<uint4*>(O + ((size_t)b * kH + h) * kDv + ch * 8) = v;
+    }
+  }
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
@@ -1004,7 +1049,7 @@ static int slots_of(const core::Sched& s, int B) {
 }
 
 struct WsLayout {
-  size_t q_tilde, opart, lse, total;
+  size_t q_tilde, opart, lse, omerged, total;
 };
 
 static WsLayout ws_layout(int B, int slots) {
@@ -1012,7 +1057,8 @@ static WsLayout ws_layout(int B, int slots) {
   w.q_tilde = 0;
   w.opart = round_up(w.q_tilde + (size_t)B * kH * kC * 2, 256);
   w.lse = round_up(w.opart + (size_t)B * slots * kH * kC * 2, 256);
-  w.total = round_up(w.lse + (size_t)B * slots * kH * 4, 256);
+  w.omerged = round_up(w.lse + (size_t)B * slots * kH * 4, 256);
+  w.total = round_up(w.omerged + (size_t)B * kH * kC * 2, 256);
   return w;
 }
 
@@ -1037,25 +1083,23 @@ static int launch_fold(const __nv_bfloat16* q_nope, const __nv_bfloat16* wkv_b,
 }
 
 template <int NB>
-static int launch_merge_nb(const __nv_bfloat16* wkv_b, const __nv_bfloat16* opart,
-                           const float* lse, int B, const core::Sched& sch, int slots,
-                           __nv_bfloat16* O, int32_t* status, cudaStream_t st) {
-  const int smem = 32768 + NB * 256 + NB * kMaxSlots * 4 + 1024;
+static int launch_uv_nb(const __nv_bfloat16* wkv_b, const __nv_bfloat16* omerged, int B,
+                        __nv_bfloat16* O, int32_t* status, cudaStream_t st) {
+  const int smem = 2 * (32768 + NB * 256) + 1024;
   static unsigned long long attr_done = 0;
-  if (int e = ensure_smem_attr(merge_uv_kernel<NB>, smem, &attr_done)) return e;
+  if (int e = ensure_smem_attr(uv_kernel<NB>, smem, &attr_done)) return e;
   dim3 grid(kH, (B + NB - 1) / NB);
-  merge_uv_kernel<NB><<<grid, 256, smem, st>>>(wkv_b, opart, lse, B, sch, slots, O, status);
+  uv_kernel<NB><<<grid, 128, smem, st>>>(wkv_b, omerged, B, O, status);
   return launch_status();
 }
 
-static int launch_merge(const __nv_bfloat16* wkv_b, const __nv_bfloat16* opart, const float* lse,
-                        int B, const core::Sched& sch, int slots, __nv_bfloat16* O,
-                        int32_t* status, cudaStream_t st) {
-  if (B <= 16) return launch_merge_nb<16>(wkv_b, opart, lse, B, sch, slots, O, status, st);
-  if (B <= 32) return launch_merge_nb<32>(wkv_b, opart, lse, B, sch, slots, O, status, st);
-  if (B <= 64) return launch_merge_nb<64>(wkv_b, opart, lse, B, sch, slots, O, status, st);
-  if (B <= 128) return launch_merge_nb<128>(wkv_b, opart, lse, B, sch, slots, O, status, st);
-  return launch_merge_nb<256>(wkv_b, opart, lse, B, sch, slots, O, status, st);
+static int launch_uv(const __nv_bfloat16* wkv_b, const __nv_bfloat16* omerged, int B,
+                     __nv_bfloat16* O, int32_t* status, cudaStream_t st) {
+  if (B <= 16) return launch_uv_nb<16>(wkv_b, omerged, B, O, status, st);
+  if (B <= 32) return launch_uv_nb<32>(wkv_b, omerged, B, O, status, st);
+  if (B <= 64) return launch_uv_nb<64>(wkv_b, omerged, B, O, status, st);
+  if (B <= 128) return launch_uv_nb<128>(wkv_b, omerged, B, O, status, st);
+  return launch_uv_nb<256>(wkv_b, omerged, B, O, status, st);
 }
 
 // The number of clusters is capped so that no batch row meets more than
@@ -1167,10 +1211,12 @@ static int decode_impl(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_
   __nv_bfloat16* q_tilde = reinterpret_cast<__nv_bfloat16*>(wsb + L.q_tilde);
   __nv_bfloat16* opart = reinterpret_cast<__nv_bfloat16*>(wsb + L.opart);
   float* lse = reinterpret_cast<float*>(wsb + L.lse);
+  __nv_bfloat16* omerged = reinterpret_cast<__nv_bfloat16*>(wsb + L.omerged);
 
   if (phase == 0 || phase == 1) {
     if (int e = launch_fold(reinterpret_cast<const __nv_bfloat16*>(q_nope),
-                            reinterpret_cast<const __nv_bfloat16*>(wkv_b), q_tilde, B, status, st))
+                            reinterpret_cast<const __nv_bfloat16*>(wkv_b), q_tilde, B, status,
+                            st))
       return e;
   }
 
@@ -1188,6 +1234,7 @@ static int decode_impl(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_
   p.scale_log2 = scale * 1.4426950408889634f;
   p.opart = opart;
   p.lse = lse;
+  p.omerged = omerged;
   p.status = status;
   if (phase == 0 || phase == 2) {
     alignas(64) CUtensorMap map_c, map_r;
@@ -1201,9 +1248,14 @@ static int decode_impl(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_
     core_kernel<<<dim3(2 * sch.nc), core::NTHREADS, core::SMEM_BYTES, st>>>(p, map_c, map_r);
     if (int e = launch_status()) return e;
   }
-  if (phase == 0 || phase == 3)
-    return launch_merge(reinterpret_cast<const __nv_bfloat16*>(wkv_b), opart, lse, B, sch, slots,
-                        reinterpret_cast<__nv_bfloat16*>(O), status, st);
+  if (phase == 0 || phase == 3) {
+    if (slots > 1) {
+      combine_kernel<<<dim3(B, kH / 16), 256, 0, st>>>(opart, lse, sch, slots, omerged);
+      if (int e = launch_status()) return e;
+    }
+    return launch_uv(reinterpret_cast<const __nv_bfloat16*>(wkv_b), omerged, B,
+                     reinterpret_cast<__nv_bfloat16*>(O), status, st);
+  }
   return MLA_OK;
 }
 
