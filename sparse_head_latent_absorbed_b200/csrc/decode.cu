@@ -235,22 +235,23 @@ constexpr int ST_ATOM = KT * 128;            // one 64-column latent atom of a t
 constexpr int ST_KR = 4 * ST_ATOM;           // rotary part of a tile (64 B swizzle)
 constexpr int ST_BYTES = ST_KR + KT * 64;    // 36864
 constexpr int OFF_ST = 0;
-constexpr int OFF_XS = OFF_ST + NST * ST_BYTES;  // two buffers of exchanged partial scores
-constexpr int XS_STRIDE = KT * 2 + 16;           // padded fp16 row
-constexpr int XS_BYTES = 128 * XS_STRIDE;
-constexpr int OFF_ONES = OFF_XS + 2 * XS_BYTES;  // 16 x 64 bf16 ones (row sums on the tensor core)
-constexpr int OFF_BIAS = OFF_ONES + 2048;         // per softmax warp: 0 / -inf per key of its half tile
-constexpr int OFF_PMAX = OFF_BIAS + NSOFT * 32 * 4;   // [2 tile parities][2 halves][128 rows] partial maxima
-constexpr int OFF_END = OFF_PMAX + 2 * 2 * 128 * 4;
+constexpr int OFF_QR = OFF_ST + NST * ST_BYTES;  // rotary half of Q: 128 rows x 64 B, 64 B swizzle
+constexpr int OFF_XS = OFF_QR + 128 * 64;        // two buffers of exchanged partial scores
+constexpr int XS_BYTES = 128 * KT * 2;           // per softmax warp 4 chunks x 32 lanes x 16 B
+constexpr int OFF_BIAS = OFF_XS + 2 * XS_BYTES;  // per softmax warp: 0 / -inf per key of the tile
+constexpr int OFF_END = OFF_BIAS + NSOFT * KT * 4;
 constexpr int SMEM_BYTES = OFF_END + 1024;       // + alignment slack
-constexpr uint32_t XS_TX_BYTES = 128 * KT * 2;   // partial scores received per tile
+constexpr uint32_t XS_TX_BYTES = XS_BYTES;       // partial scores received per tile
 constexpr uint32_t GROUP_TX_BYTES = ST_BYTES / 16;  // bytes of one group of four keys
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t T_S = 0, T_Q = 64, T_L = 208, T_P = 224, T_O = 256;
+// TMEM: Q~ latent half (bf16 pairs), the score tile, two P tiles (bf16
+// pairs), O~ (latent half, fp32)
+constexpr uint32_t T_Q = 0, T_S = 128, T_P = 192, T_O = 256;
 constexpr float kRescaleThreshold = 8.0f;        // log2 units
-static_assert(ST_BYTES % 1024 == 0 && OFF_XS % 16 == 0 && OFF_ONES % 1024 == 0, "alignment");
+static_assert(ST_BYTES % 1024 == 0 && OFF_QR % 1024 == 0 && OFF_XS % 16 == 0, "alignment");
 static_assert(SMEM_BYTES + 512 <= 232448, "shared memory budget");
-static_assert(T_Q + 144 <= T_L && T_L + 16 <= T_P && T_P + KT / 2 <= T_O, "TMEM plan");
+static_assert(T_Q + 128 <= T_S && T_S + KT <= T_P && T_P + KT <= T_O && T_O + 256 <= TMEM_COLS,
+              "TMEM plan");
 static_assert(KT / 4 == 16, "sixteen groups of four keys per tile");
 
 // Schedule: tiles [bnd(c), bnd(c+1)) of the flattened list belong to cluster c.
@@ -287,8 +288,13 @@ struct Params {
 };
 
 struct Bars {
-  uint64_t full[NST], empty[NST], s_full, s_empty, p_full, o_done, q_ready, xs_full[2],
-      xs_free[2], drain;
+  uint64_t full[NST], empty[NST];  // gather ring
+  uint64_t s_full, s_empty;        // score tile in TMEM / read by all softmax threads
+  uint64_t p_full[2];              // P of tile t is in TMEM buffer t & 1 (all softmax threads)
+  uint64_t o_done[2];              // the value product of tile t has completed
+  uint64_t q_ready;                // the segment's Q~ is in TMEM / shared memory
+  uint64_t xs_full[2], xs_free[2]; // exchange buffers (peer's partial scores)
+  uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -361,25 +367,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       mbar_init(&bars.full[s], NGATHER);  // one expect_tx arrival per gather warp + bytes
       mbar_init(&bars.empty[s], 1);       // MMA commit after the tile's value product
     }
-    mbar_init(&bars.s_full, 1);
-    mbar_init(&bars.s_empty, 32 * NSOFT);
-    mbar_init(&bars.p_full, 32 * NSOFT);
-    mbar_init(&bars.o_done, 1);
-    mbar_init(&bars.q_ready, 32 * NSOFT);
     for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.p_full[i], 32 * NSOFT);
+      mbar_init(&bars.o_done[i], 1);
       mbar_init(&bars.xs_full[i], 1);      // own expect_tx arrival + the peer's st.async bytes
       mbar_init(&bars.xs_free[i], NSOFT);  // one arrival per softmax warp of the peer
     }
+    mbar_init(&bars.s_full, 1);
+    mbar_init(&bars.s_empty, 32 * NSOFT);
+    mbar_init(&bars.q_ready, 32 * NSOFT);
     mbar_init(&bars.drain, 1);
     bars.abort = 0;
     fence_mbarrier_init_cluster();
     mbar_arrive_expect_tx(&bars.xs_full[0], XS_TX_BYTES);
     mbar_arrive_expect_tx(&bars.xs_full[1], XS_TX_BYTES);
   }
-  // the ones tile (bf16 1.0): any swizzle of it is the same tile
-  for (int i = tid; i < 2048 / 16; i += NTHREADS)
-    st_shared_v4(sbase + OFF_ONES + i * 16, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
-  fence_proxy_async_smem();
   tc_fence_before();
   cluster_sync_all();
   tc_fence_after();
@@ -391,7 +393,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     // 0..ng-1 each issue the five loads of one group of four keys
     const int gw = warp - GATHER_WARP0;
     const int ng = (16 - gw + NGATHER - 1) / NGATHER;  // groups of this warp
-    int bad = 0;
+    int bad = 0, issued = 0;
     TileCur cur = first_cur();
     SHLA_TRACE_DECL
 #pragma unroll 1
@@ -429,22 +431,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
                       &bars.full[s]);
         tma_gather4(stage + ST_KR + k0 * 64, &map_r, rank * 32, r0, r1, r2, r3, &bars.full[s]);
       }
+      issued = i + 1;
       SHLA_T(2);
     }
+    // on an abort, the loads still in flight land before the CTA can leave
+    // (the waits are bounded and already complete on the normal path)
+    for (int t = max(0, issued - NST); t < issued; ++t)
+      warp_wait(&bars.full[t % NST], (t / NST) & 1, nullptr, nullptr);
     if (lane == 0 && gw == 0) SHLA_TRACE_FLUSH(1);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);
     if (lane == 0 && bad && p.status) atomicAdd(p.status + 1, bad);
   } else if (warp == MMA_WARP) {
     // ---------------- MMA issuer ----------------
-    // Event loop: a value product as soon as its P is in TMEM (first, so the
-    // softmax never waits behind a score tile queued after it); a score tile
-    // as soon as its keys have landed, the score buffer has been read and
-    // this segment's Q~ is in TMEM.
+    // Event loop.  A value product (A = P of tile t from TMEM buffer t & 1)
+    // goes first whenever its P is ready; a score product as soon as its keys
+    // have landed, the previous score tile has been read and this segment's
+    // Q~ is in place.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, KT, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, 0, 1);
-      constexpr uint32_t idesc_l = idesc_bf16_f32(128, 16, 0, 0);
       int qk = 0, pv = 0, idle = 0, qseg = -1;
       int jq = jt0, jp = jt0;  // tile-in-row of the next score / value product
       bool alive = true;
@@ -453,25 +459,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
 #pragma unroll 1
       while (alive && pv < n) {
         bool did = false;
-        if (pv < qk && mbar_test(&bars.p_full, pv & 1)) {
+        if (pv < qk && mbar_test(&bars.p_full[pv & 1], (pv >> 1) & 1)) {
           tc_fence_after();
           const int s = pv % NST;
           const uint32_t st = sbase + OFF_ST + s * ST_BYTES;
+          const uint32_t tp = tmem + T_P + (pv & 1) * (KT / 2);
           const bool first = pv == 0 || jp == 0;
 #pragma unroll
           for (int ks = 0; ks < KT / 16; ++ks) {
             const uint64_t bd = smem_desc(st + ks * 2048, ST_ATOM, 1024, kSwizzle128B);
-            tc_mma_tmem_a(tmem + T_O, tmem + T_P + ks * 8, bd, idesc_pv,
-                          (!first || ks > 0) ? 1u : 0u);
+            tc_mma_tmem_a(tmem + T_O, tp + ks * 8, bd, idesc_pv, (!first || ks > 0) ? 1u : 0u);
           }
-          // row sums: l += P x ones (16 identical columns)
-#pragma unroll
-          for (int ks = 0; ks < KT / 16; ++ks) {
-            const uint64_t bd = smem_desc(sbase + OFF_ONES + ks * 32, 16, 1024, kSwizzle128B);
-            tc_mma_tmem_a(tmem + T_L, tmem + T_P + ks * 8, bd, idesc_l,
-                          (!first || ks > 0) ? 1u : 0u);
-          }
-          tc_commit(&bars.o_done);
+          tc_commit(&bars.o_done[pv & 1]);
           tc_commit(&bars.empty[s]);
           ++pv;
           if (++jp == nt) jp = 0;
@@ -485,16 +484,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
             qseg = seg;
             tc_fence_after();
             const uint32_t st = sbase + OFF_ST + (qk % NST) * ST_BYTES;
+            const uint32_t ts = tmem + T_S;
 #pragma unroll
             for (int ks = 0; ks < 16; ++ks) {
               const uint64_t bd =
                   smem_desc(st + (ks >> 2) * ST_ATOM + (ks & 3) * 32, 16, 1024, kSwizzle128B);
-              tc_mma_tmem_a(tmem + T_S, tmem + T_Q + ks * 8, bd, idesc_qk, ks > 0);
+              tc_mma_tmem_a(ts, tmem + T_Q + ks * 8, bd, idesc_qk, ks > 0);
             }
 #pragma unroll
             for (int ks = 0; ks < 2; ++ks) {
+              const uint64_t ad = smem_desc(sbase + OFF_QR + ks * 32, 16, 512, kSwizzle64B);
               const uint64_t bd = smem_desc(st + ST_KR + ks * 32, 16, 512, kSwizzle64B);
-              tc_mma_tmem_a(tmem + T_S, tmem + T_Q + 128 + ks * 8, bd, idesc_qk, 1);
+              tc_mma(ts, ad, bd, idesc_qk, 1);
             }
             tc_commit(&bars.s_full);
             ++qk;
@@ -524,73 +525,81 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     }
     __syncwarp();
   } else {
-    // ---------------- softmax (two threads per head row) ----------------
-    const int quarter = warp & 3;             // TMEM lane quarter
-    const int half = warp >> 2;               // keys [32*half, 32*half + 32) of a tile
-    const int h = quarter * 32 + lane;        // head row = TMEM lane
-    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    constexpr int KH = KT / 2;                // keys per thread per tile
-    // this CTA's half of Q~ (256 latent + 32 rotary values) of batch row bb
-    // into TMEM as bf16 pairs: chunks of 16 columns, 0-4 by the first half,
-    // 5-8 by the second; then q_ready
+    // ---------------- softmax (four threads per head row) ----------------
+    // Warp w covers the 16 head rows [32q + 16s, +16) (q = w & 3 its TMEM
+    // lane quarter, s = w >> 2).  Through the 16x256b TMEM shape thread t
+    // holds rows r0 = t/4 and r0 + 8 of them and, of each 8-key block j, the
+    // keys 8j + 2c and 8j + 2c + 1 (c = t % 4): a row's 64 keys sit in four
+    // adjacent lanes, so its maxima and sums take two shuffles.  Score pair u
+    // of a thread is block u/2 of row r0 (u even) or of row r0 + 8 (u odd).
+    const int quarter = warp & 3, sub = warp >> 2;
+    const int c4 = lane & 3;
+    const int row0 = quarter * 32 + sub * 16 + (lane >> 2);  // second row: row0 + 8
+    const uint32_t frag_base = (uint32_t)(quarter * 32 + sub * 16) << 16;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;  // 32x32b (Q~ load)
+    const int h = quarter * 32 + lane;  // this thread's row in 32x32b accesses
+    constexpr int NP = KT / 4;          // fp16 score pairs per thread per tile
+    // this CTA's half of Q~ for batch row bb: latent values [128 s, +128) of
+    // the CTA's 256 into TMEM as bf16 pairs (row h), rotary values [16 s, +16)
+    // of its 32 into the swizzled shared tile; then q_ready
     auto load_q = [&](int bb) {
-      const __nv_bfloat16* qrow = p.q_tilde + ((size_t)bb * kH + h) * kC + rank * 256;
-      const __nv_bfloat16* rrow = p.q_pe + ((size_t)bb * kH + h) * kR + rank * 32;
-      const int c_lo = half ? 5 : 0, c_n = half ? 4 : 5;
-      uint4 q[5][4];
+      const __nv_bfloat16* qrow = p.q_tilde + ((size_t)bb * kH + h) * kC + rank * 256 + sub * 128;
+      const __nv_bfloat16* rrow = p.q_pe + ((size_t)bb * kH + h) * kR + rank * 32 + sub * 16;
+      uint4 q[4][4], rq[2];
 #pragma unroll
-      for (int c = 0; c < 5; ++c) {
-        if (c < c_n) {
-          const int cc = c_lo + c;
-          const __nv_bfloat16* src = cc < 8 ? qrow + cc * 32 : rrow;
+      for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) q[c][i] = ld_global_nc_v4(src + i * 8);
+        for (int i = 0; i < 4; ++i) q[c][i] = ld_global_nc_v4(qrow + c * 32 + i * 8);
+      rq[0] = ld_global_nc_v4(rrow);
+      rq[1] = ld_global_nc_v4(rrow + 8);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          r[4 * i] = q[c][i].x;
+          r[4 * i + 1] = q[c][i].y;
+          r[4 * i + 2] = q[c][i].z;
+          r[4 * i + 3] = q[c][i].w;
         }
+        tmem_st16(tmem + lane_base + T_Q + sub * 64 + c * 16, r);
       }
 #pragma unroll
-      for (int c = 0; c < 5; ++c) {
-        if (c < c_n) {
-          uint32_t r[16];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            r[4 * i] = q[c][i].x;
-            r[4 * i + 1] = q[c][i].y;
-            r[4 * i + 2] = q[c][i].z;
-            r[4 * i + 3] = q[c][i].w;
-          }
-          tmem_st16(tmem + lane_base + T_Q + (c_lo + c) * 16, r);
-        }
-      }
+      for (int c = 0; c < 2; ++c)
+        st_shared_v4(sbase + OFF_QR + sw64_off(h, 2 * sub + c), rq[c].x, rq[c].y, rq[c].z,
+                     rq[c].w);
+      fence_proxy_async_smem();
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&bars.q_ready);
     };
 
-    // exchange buffer / barrier i sits at +i*XS_BYTES / +i*8 from buffer 0 in
-    // both CTAs, so the peer addresses follow from one mapa each; this thread
-    // owns bytes [64*half, 64*half + 64) of its row
-    const uint32_t xs_row0 = sbase + OFF_XS + h * XS_STRIDE + half * 64;
-    const uint32_t xs_peer_row0 = mapa_shared(xs_row0, peer);
+    // exchange buffer i of this warp: 4 chunks x 32 lanes x 16 bytes at
+    // +i*XS_BYTES (same offsets in both CTAs); a thread's 16 pairs are its
+    // chunks 0..3
+    const uint32_t xs_own0 = sbase + OFF_XS + warp * (XS_BYTES / NSOFT) + lane * 16;
+    const uint32_t xs_peer0 = mapa_shared(xs_own0, peer);
     const uint32_t xs_full_peer0 = mapa_shared(smem_u32(&bars.xs_full[0]), peer);
     const uint32_t xs_free_peer0 = mapa_shared(smem_u32(&bars.xs_free[0]), peer);
-    const uint32_t bias_w = sbase + OFF_BIAS + warp * (32 * 4);
-    const uint32_t pmax_own = sbase + OFF_PMAX + (half * 128 + h) * 4;
-    const uint32_t pmax_other = sbase + OFF_PMAX + ((half ^ 1) * 128 + h) * 4;
-    const uint32_t pair_bar = 1 + quarter;    // named barrier of warps w and w+4
-    float m_used = -INFINITY;
-    uint32_t sa[KH / 2], sb[KH / 2];  // scaled partial scores as fp16 pairs: current, next
+    int nx = 0;  // next tile whose exchange buffer this CTA consumes
+    const uint32_t bias_w = sbase + OFF_BIAS + warp * (KT * 4);  // this warp's copy of the tile's key biases
+    float m_used[2] = {-INFINITY, -INFINITY};  // running maxima of rows r0, r0 + 8 (log2 units)
+    float l_run[2] = {0.f, 0.f};               // this thread's parts of their row sums
+    uint32_t sa[NP], sb[NP];  // scaled partial scores as fp16 pairs: current, next
     bool alive = true;
     SHLA_TRACE_DECL
 
     // own partial of tile t (position ct): TMEM -> x scale + (0 | -inf) per
     // key -> fp16 pairs -> the peer's exchange buffer.  When the next tile
     // (position cn) starts a new batch row, its Q~ replaces this one.
-    auto fetch_send = [&](int t, uint32_t (&dst)[KH / 2], const TileCur& ct,
-                          const TileCur& cn) -> bool {
+    auto fetch_send = [&](int t, uint32_t (&dst)[NP], const TileCur& ct, const TileCur& cn) -> bool {
       const int b2 = t & 1;
       __syncwarp();
       asm volatile("st.shared.f32 [%0], %1;" ::"r"(bias_w + lane * 4),
-                   "f"(key_valid(half ? ct.ihi : ct.ilo, ct.lim) ? 0.f : -INFINITY)
+                   "f"(key_valid(ct.ilo, ct.lim) ? 0.f : -INFINITY)
+                   : "memory");
+      asm volatile("st.shared.f32 [%0], %1;" ::"r"(bias_w + (32 + lane) * 4),
+                   "f"(key_valid(ct.ihi, ct.lim) ? 0.f : -INFINITY)
                    : "memory");
       __syncwarp();
       SHLA_T(11);
@@ -598,25 +607,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       SHLA_T(0);
       tc_fence_after();
       {
-        uint32_t r[2][16];
-        tmem_ld16(tmem + lane_base + T_S + half * KH, r[0]);
-        tmem_ld16(tmem + lane_base + T_S + half * KH + 16, r[1]);
+        uint32_t r[32];
+        tmem_ld_16x256b_x8(tmem + frag_base + T_S, r);
         tc_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float4 bv;
-            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                         : "=f"(bv.x), "=f"(bv.y), "=f"(bv.z), "=f"(bv.w)
-                         : "r"(bias_w + (c * 16 + q * 4) * 4));
-            const float x0 = fmaf(__uint_as_float(r[c][4 * q]), p.scale_log2, bv.x);
-            const float x1 = fmaf(__uint_as_float(r[c][4 * q + 1]), p.scale_log2, bv.y);
-            const float x2 = fmaf(__uint_as_float(r[c][4 * q + 2]), p.scale_log2, bv.z);
-            const float x3 = fmaf(__uint_as_float(r[c][4 * q + 3]), p.scale_log2, bv.w);
-            dst[c * 8 + 2 * q] = f16x2_from_f32_sat(x0, x1);
-            dst[c * 8 + 2 * q + 1] = f16x2_from_f32_sat(x2, x3);
-          }
+        for (int j = 0; j < 8; ++j) {
+          float2 bv;
+          asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];"
+                       : "=f"(bv.x), "=f"(bv.y)
+                       : "r"(bias_w + (8 * j + 2 * c4) * 4));
+          const float x00 = fmaf(__uint_as_float(r[4 * j]), p.scale_log2, bv.x);
+          const float x01 = fmaf(__uint_as_float(r[4 * j + 1]), p.scale_log2, bv.y);
+          const float x10 = fmaf(__uint_as_float(r[4 * j + 2]), p.scale_log2, bv.x);
+          const float x11 = fmaf(__uint_as_float(r[4 * j + 3]), p.scale_log2, bv.y);
+          dst[2 * j] = f16x2_from_f32_sat(x00, x01);
+          dst[2 * j + 1] = f16x2_from_f32_sat(x10, x11);
         }
       }
       tc_fence_before();
@@ -627,53 +632,64 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       if (!warp_wait<true>(&bars.xs_free[b2], ((t >> 1) & 1) ^ 1, abort, p.status)) return false;
       SHLA_T(2);
 #pragma unroll
-      for (int i = 0; i < KH / 2; i += 4)
-        st_async_v4(xs_peer_row0 + b2 * XS_BYTES + i * 4, __uint_as_float(dst[i]),
-                    __uint_as_float(dst[i + 1]), __uint_as_float(dst[i + 2]),
-                    __uint_as_float(dst[i + 3]), xs_full_peer0 + b2 * 8);
+      for (int k = 0; k < 4; ++k)
+        st_async_v4(xs_peer0 + b2 * XS_BYTES + k * 512, __uint_as_float(dst[4 * k]),
+                    __uint_as_float(dst[4 * k + 1]), __uint_as_float(dst[4 * k + 2]),
+                    __uint_as_float(dst[4 * k + 3]), xs_full_peer0 + b2 * 8);
       SHLA_T(3);
       return true;
     };
 
-    // epilogue of a segment: this thread's 128 columns of the CTA's latent
-    // half of O~ / l into the segment's slot, and (rank 0, first half) the
-    // row's log-sum-exp
-    auto flush = [&](int i_last, int bb) -> bool {
-      if (!warp_wait(&bars.o_done, i_last & 1, abort, p.status)) return false;
+    // the value product of tile t has completed.  Sound because the softmax
+    // waits for the product of tile t - 2 (same barrier, previous phase)
+    // before it writes tile t's P, so at most one phase of each barrier is
+    // ever outstanding when it is tested.
+    auto wait_pv = [&](int t) -> bool {
+      if (!warp_wait(&bars.o_done[t & 1], (t >> 1) & 1, abort, p.status)) return false;
       tc_fence_after();
+      return true;
+    };
+
+    // epilogue of a segment: rows r0 and r0 + 8 of the CTA's latent half of
+    // O~ / l into the row's output (a row held by one cluster) or the
+    // segment's slot, and (rank 0) the segment's log-sum-exps
+    auto flush = [&](int i_last, int bb) -> bool {
+      float l[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        l[e] = l_run[e] + __shfl_xor_sync(0xffffffffu, l_run[e], 1);
+        l[e] += __shfl_xor_sync(0xffffffffu, l[e], 2);
+      }
+      if (!wait_pv(i_last)) return false;
       const int cf = p.sch.c_first(bb);
       const int used = p.sch.c_last(bb) - cf + 1;  // clusters holding a segment of row bb
       const int slot = cid - cf;
+      const float inv0 = l[0] > 0.f ? 1.f / l[0] : 0.f;
+      const float inv1 = l[1] > 0.f ? 1.f / l[1] : 0.f;
+      __nv_bfloat16* dst0 =
+          (used == 1 ? p.omerged + ((size_t)bb * kH + row0) * kC
+                     : p.opart + (((size_t)bb * p.slots + slot) * kH + row0) * kC) +
+          rank * 256 + 2 * c4;
+      __nv_bfloat16* dst1 = dst0 + 8 * kC;
       uint32_t r[16];
-      tmem_ld16(tmem + lane_base + T_L, r);
-      tc_wait_ld();
-      const float l = __uint_as_float(r[0]);
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      // a row held by one cluster is final here; otherwise this is one segment
-      // of the row, merged by combine_kernel
-      __nv_bfloat16* dst =
-          (used == 1 ? p.omerged + ((size_t)bb * kH + h) * kC
-                     : p.opart + (((size_t)bb * p.slots + slot) * kH + h) * kC) +
-          rank * 256 + half * 128;
 #pragma unroll 1
-      for (int c = 0; c < 128; c += 16) {
-        tmem_ld16(tmem + lane_base + T_O + half * 128 + c, r);
+      for (int cc = 0; cc < 256; cc += 32) {
+        tmem_ld_16x256b_x4(tmem + frag_base + T_O + cc, r);
         tc_wait_ld();
-        uint4 lo, hi;
-        lo.x = pack_bf16x2(__uint_as_float(r[0]) * inv, __uint_as_float(r[1]) * inv);
-        lo.y = pack_bf16x2(__uint_as_float(r[2]) * inv, __uint_as_float(r[3]) * inv);
-        lo.z = pack_bf16x2(__uint_as_float(r[4]) * inv, __uint_as_float(r[5]) * inv);
-        lo.w = pack_bf16x2(__uint_as_float(r[6]) * inv, __uint_as_float(r[7]) * inv);
-        hi.x = pack_bf16x2(__uint_as_float(r[8]) * inv, __uint_as_float(r[9]) * inv);
-        hi.y = pack_bf16x2(__uint_as_float(r[10]) * inv, __uint_as_float(r[11]) * inv);
-        hi.z = pack_bf16x2(__uint_as_float(r[12]) * inv, __uint_as_float(r[13]) * inv);
-        hi.w = pack_bf16x2(__uint_as_float(r[14]) * inv, __uint_as_float(r[15]) * inv);
-        *reinterpret_cast<uint4*>(dst + c) = lo;
-        *reinterpret_cast<uint4*>(dst + c + 8) = hi;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          *reinterpret_cast<uint32_t*>(dst0 + cc + 8 * j) =
+              pack_bf16x2(__uint_as_float(r[4 * j]) * inv0, __uint_as_float(r[4 * j + 1]) * inv0);
+          *reinterpret_cast<uint32_t*>(dst1 + cc + 8 * j) =
+              pack_bf16x2(__uint_as_float(r[4 * j + 2]) * inv1, __uint_as_float(r[4 * j + 3]) * inv1);
+        }
       }
       tc_fence_before();
-      if (used > 1 && rank == 0 && half == 0)
-        p.lse[((size_t)bb * p.slots + slot) * kH + h] = l > 0.f ? m_used + log2f(l) : -INFINITY;
+      if (used > 1 && rank == 0 && c4 == 0) {
+        float* lse = p.lse + ((size_t)bb * p.slots + slot) * kH + row0;
+        lse[0] = l[0] > 0.f ? m_used[0] + log2f(l[0]) : -INFINITY;
+        lse[8] = l[1] > 0.f ? m_used[1] + log2f(l[1]) : -INFINITY;
+      }
       return true;
     };
 
@@ -686,7 +702,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
 
     // one key tile: `cur` holds this thread's scaled partial scores of tile i
     // on entry; the next tile's partial is fetched into `nxt` and sent first
-    auto step = [&](int i, uint32_t (&cur)[KH / 2], uint32_t (&nxt)[KH / 2]) -> bool {
+    auto step = [&](int i, uint32_t (&cur)[NP], uint32_t (&nxt)[NP]) -> bool {
       if (i + 1 < n) {
         c2 = i + 2 < n ? advance(c1) : c1;
         SHLA_T(12);
@@ -696,82 +712,112 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       const int b2 = i & 1;
       SHLA_T(11);
       if (!warp_wait<true>(&bars.xs_full[b2], (i >> 1) & 1, abort, p.status)) return false;
+      nx = i + 1;
       SHLA_T(4);
-      uint32_t mx2 = 0xFC00FC00u;  // (-inf, -inf)
 #pragma unroll
-      for (int c = 0; c < KH / 2; c += 4) {
+      for (int k = 0; k < 4; ++k) {
         uint4 o;
         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                      : "=r"(o.x), "=r"(o.y), "=r"(o.z), "=r"(o.w)
-                     : "r"(xs_row0 + b2 * XS_BYTES + c * 4));
-        cur[c] = hadd2_u(cur[c], o.x);
-        cur[c + 1] = hadd2_u(cur[c + 1], o.y);
-        cur[c + 2] = hadd2_u(cur[c + 2], o.z);
-        cur[c + 3] = hadd2_u(cur[c + 3], o.w);
-        mx2 = hmax2_u(mx2, hmax2_u(hmax2_u(cur[c], cur[c + 1]), hmax2_u(cur[c + 2], cur[c + 3])));
+                     : "r"(xs_own0 + b2 * XS_BYTES + k * 512));
+        cur[4 * k] = hadd2_u(cur[4 * k], o.x);
+        cur[4 * k + 1] = hadd2_u(cur[4 * k + 1], o.y);
+        cur[4 * k + 2] = hadd2_u(cur[4 * k + 2], o.z);
+        cur[4 * k + 3] = hadd2_u(cur[4 * k + 3], o.w);
       }
       // next use of this buffer (tile i + 2): expect the peer's bytes again
       if (tid == 0 && i + 2 < n) mbar_arrive_expect_tx(&bars.xs_full[b2], XS_TX_BYTES);
-      // row maximum of the tile: combine with the other half of the row
-      const float2 mxf = f16x2_to_f32x2(mx2);
-      const float mt_own = fmaxf(mxf.x, mxf.y);
-      asm volatile("st.shared.f32 [%0], %1;" ::"r"(pmax_own + b2 * 1024), "f"(mt_own) : "memory");
-      asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
-      float mt_other;
-      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(mt_other) : "r"(pmax_other + b2 * 1024) : "memory");
-      const float mt = fmaxf(mt_own, mt_other);
+      // row maxima of the tile: the thread's pairs, then its row's four lanes
+      float mt[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        uint32_t mx2 = hmax2_u(hmax2_u(cur[e], cur[e + 2]), hmax2_u(cur[e + 4], cur[e + 6]));
+        mx2 = hmax2_u(mx2, hmax2_u(hmax2_u(cur[e + 8], cur[e + 10]), hmax2_u(cur[e + 12], cur[e + 14])));
+        const float2 f = f16x2_to_f32x2(mx2);
+        mt[e] = fmaxf(f.x, f.y);
+        mt[e] = fmaxf(mt[e], __shfl_xor_sync(0xffffffffu, mt[e], 1));
+        mt[e] = fmaxf(mt[e], __shfl_xor_sync(0xffffffffu, mt[e], 2));
+      }
       SHLA_T(5);
 
       // a new segment: write out the previous one and restart the running max
       const bool first = i == 0 || c0.jt == 0;
       if (first && i > 0) {
         if (!flush(i - 1, prev_bb)) return false;
-        m_used = -INFINITY;
+        m_used[0] = m_used[1] = -INFINITY;
+        l_run[0] = l_run[1] = 0.f;
       }
-      const float m_new = fmaxf(m_used, mt);
-      const bool rescale = m_new > m_used + kRescaleThreshold;
+      float m_new[2];
+      bool rescale[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        m_new[e] = fmaxf(m_used[e], mt[e]);
+        rescale[e] = m_new[e] > m_used[e] + kRescaleThreshold;
+      }
       SHLA_T(6);
-      if (i > 0 && !first) {
-        if (!warp_wait(&bars.o_done, (i - 1) & 1, abort, p.status)) return false;
-        tc_fence_after();
-      }
-      SHLA_T(7);
-      if (!first && __any_sync(0xffffffffu, rescale)) {
-        // warp-collective over this thread's 128 accumulator columns (and the
-        // row sums, first half): rows that keep their maximum scale by 1
-        const float alpha = rescale ? fast_exp2(m_used - m_new) : 1.f;
+      if (!first && __any_sync(0xffffffffu, rescale[0] || rescale[1])) {
+        // O~ must hold the value product of tile i - 1 before it is scaled;
+        // warp-collective over the warp's 16 rows x 256 accumulator columns:
+        // rows that keep their maximum scale by 1
+        if (!wait_pv(i - 1)) return false;
+        const float a0 = rescale[0] ? fast_exp2(m_used[0] - m_new[0]) : 1.f;
+        const float a1 = rescale[1] ? fast_exp2(m_used[1] - m_new[1]) : 1.f;
+        l_run[0] *= a0;
+        l_run[1] *= a1;
         uint32_t r[16];
 #pragma unroll 1
-        for (int c = half ? 0 : -16; c < 128; c += 16) {
-          const uint32_t ta = tmem + lane_base + (c < 0 ? T_L : T_O + half * 128 + c);
-          tmem_ld16(ta, r);
+        for (int cc = 0; cc < 256; cc += 32) {
+          const uint32_t ta = tmem + frag_base + T_O + cc;
+          tmem_ld_16x256b_x4(ta, r);
           tc_wait_ld();
 #pragma unroll
-          for (int u = 0; u < 16; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * alpha);
-          tmem_st16(ta, r);
+          for (int j = 0; j < 4; ++j) {
+            r[4 * j] = __float_as_uint(__uint_as_float(r[4 * j]) * a0);
+            r[4 * j + 1] = __float_as_uint(__uint_as_float(r[4 * j + 1]) * a0);
+            r[4 * j + 2] = __float_as_uint(__uint_as_float(r[4 * j + 2]) * a1);
+            r[4 * j + 3] = __float_as_uint(__uint_as_float(r[4 * j + 3]) * a1);
+          }
+          tmem_st_16x256b_x4(ta, r);
         }
       }
-      if (rescale) m_used = m_new;
-      SHLA_T(8);
-      // P = 2^(s - m) on fp16 pairs, stored to TMEM as bf16 pairs
-      const bool live = m_used != -INFINITY;
-      const uint32_t m2 = live ? f16x2_splat(m_used) : 0u;
-      {
-        uint32_t w[16];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          if (live) {
-            const float2 e = f16x2_to_f32x2(hex2_u(hsub2_u(cur[u], m2)));
-            w[u] = bf16x2_from_f32(e.x, e.y);
-          } else {
-            w[u] = 0u;
-          }
+      for (int e = 0; e < 2; ++e)
+        if (rescale[e]) m_used[e] = m_new[e];
+      SHLA_T(7);
+      // P buffer b2 was last read by the value product of tile i - 2
+      if (i >= 2 && !wait_pv(i - 2)) return false;
+      SHLA_T(8);
+      // P = 2^(s - m) on fp16 pairs, to TMEM buffer b2 as bf16 pairs (pair u
+      // lands in P column 4(u/2) + c of its row); the tile's row sums are
+      // added on fp16 pairs in a tree (each P <= 2^8 under the lazy rescale,
+      // so a thread's part of a row stays <= 2^12)
+      {
+        const bool live0 = m_used[0] != -INFINITY, live1 = m_used[1] != -INFINITY;
+        const uint32_t m20 = live0 ? f16x2_splat(m_used[0]) : 0u;
+        const uint32_t m21 = live1 ? f16x2_splat(m_used[1]) : 0u;
+        uint32_t w[NP], e[NP];
+#pragma unroll
+        for (int u = 0; u < NP; ++u) {
+          const bool live = (u & 1) ? live1 : live0;
+          e[u] = live ? hex2_u(hsub2_u(cur[u], (u & 1) ? m21 : m20)) : 0u;
+          const float2 f = f16x2_to_f32x2(e[u]);
+          w[u] = bf16x2_from_f32(f.x, f.y);
         }
-        tmem_st16(tmem + lane_base + T_P + half * 16, w);
+#pragma unroll
+        for (int d = 2; d < NP; d *= 2)
+#pragma unroll
+          for (int u = 0; u < NP; u += 2 * d) {
+            e[u] = hadd2_u(e[u], e[u + d]);
+            e[u + 1] = hadd2_u(e[u + 1], e[u + 1 + d]);
+          }
+        const float2 l0 = f16x2_to_f32x2(e[0]), l1 = f16x2_to_f32x2(e[1]);
+        l_run[0] += l0.x + l0.y;
+        l_run[1] += l1.x + l1.y;
+        tmem_st_16x128b_x8(tmem + frag_base + T_P + b2 * (KT / 2), w);
       }
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars.p_full);
+      mbar_arrive(&bars.p_full[b2]);
       // this tile's exchange buffer can take the peer's tile i + 2 (its reads
       // completed above)
       __syncwarp();
@@ -788,11 +834,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     for (int i = 0; i < n && alive; ++i) {
       if (!step(i, sa, sb)) { alive = false; break; }
 #pragma unroll
-      for (int u = 0; u < KH / 2; ++u) sa[u] = sb[u];
+      for (int u = 0; u < NP; ++u) sa[u] = sb[u];
     }
     SHLA_T(10);
     if (lane == 0) SHLA_TRACE_FLUSH(0);
     if (__all_sync(0xffffffffu, alive && !*abort)) flush(n - 1, prev_bb);
+    // on an abort, partial scores the peer may still be sending land before
+    // the CTA can leave: the armed, unconsumed phases (bounded waits; none
+    // remain on the normal path)
+    for (int t = nx; t < n && t < nx + 2; ++t)
+      warp_wait<true>(&bars.xs_full[t & 1], (t >> 1) & 1, nullptr, nullptr);
   }
 
   tc_fence_before();
