@@ -225,12 +225,18 @@ DEV uint32_t f16x2_splat(float v) {  // v exactly representable in fp16
 
 namespace core {
 constexpr int KT = 64;                       // keys per tile
-constexpr int NST = 5;                       // gather ring depth
+constexpr int NST = 4;                       // gather ring depth
 constexpr int NSOFT = 8;                     // softmax warps (two per TMEM lane quarter)
-constexpr int NGATHER = 3;                   // gather warps
+constexpr int NGATHER = 7;                   // gather warps
 constexpr int GATHER_WARP0 = NSOFT;
 constexpr int MMA_WARP = NSOFT + NGATHER;
-constexpr int NTHREADS = 32 * (MMA_WARP + 1);  // 384
+constexpr int NTHREADS = 32 * (MMA_WARP + 1);  // 512
+// Register split (setmaxnreg; the launch gives 128 per thread): the eight
+// softmax warps take 176, the gather and MMA warps keep 80:
+// 8 x 32 x 176 + 8 x 32 x 80 = 65536.
+constexpr int REGS_SOFTMAX = 176, REGS_OTHER = 80;
+static_assert(NSOFT * 32 * REGS_SOFTMAX + (NTHREADS - 32 * NSOFT) * REGS_OTHER <= 65536,
+              "register split");
 constexpr int ST_ATOM = KT * 128;            // one 64-column latent atom of a tile
 constexpr int ST_KR = 4 * ST_ATOM;           // rotary part of a tile (64 B swizzle)
 constexpr int ST_BYTES = ST_KR + KT * 64;    // 36864
@@ -388,6 +394,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
   const uint32_t tmem = bars.tmem_base;
 
   if (warp >= GATHER_WARP0 && warp < MMA_WARP) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_OTHER));
     // ---------------- gather (TMA tile::gather4) ----------------
     // lane l holds the index of key l and key 32 + l of the tile; lanes
     // 0..ng-1 each issue the five loads of one group of four keys
@@ -443,6 +450,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);
     if (lane == 0 && bad && p.status) atomicAdd(p.status + 1, bad);
   } else if (warp == MMA_WARP) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_OTHER));
     // ---------------- MMA issuer ----------------
     // Event loop.  A value product (A = P of tile t from TMEM buffer t & 1)
     // goes first whenever its P is ready; a score product as soon as its keys
@@ -526,6 +534,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     __syncwarp();
   } else {
     // ---------------- softmax (four threads per head row) ----------------
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
     // Warp w covers the 16 head rows [32q + 16s, +16) (q = w & 3 its TMEM
     // lane quarter, s = w >> 2).  Through the 16x256b TMEM shape thread t
     // holds rows r0 = t/4 and r0 + 8 of them and, of each 8-key block j, the
