@@ -462,7 +462,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       int qk = 0, pv = 0, idle = 0, qseg = -1;
       int jq = jt0, jp = jt0;  // tile-in-row of the next score / value product
       bool alive = true;
-      uint64_t t_last = globaltimer_ns();
+      uint64_t t_idle = 0;  // when the current idle stretch was first checked (0: not yet)
       SHLA_TRACE_DECL
 #pragma unroll 1
       while (alive && pv < n) {
@@ -513,13 +513,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
           }
         }
         SHLA_T(0);
+        // the time limit runs from the first check of an idle stretch (the
+        // timer is read only while nothing is ready)
         if (did) {
           idle = 0;
-          t_last = globaltimer_ns();
+          t_idle = 0;
         } else if (++idle >= 64) {
           idle = 0;
           if (*abort) break;
-          if (globaltimer_ns() - t_last > kWaitLimitNs) {
+          const uint64_t now = globaltimer_ns();
+          if (t_idle == 0) {
+            t_idle = now;
+          } else if (now - t_idle > kWaitLimitNs) {
             *abort = 1;
             report_timeout(p.status);
             break;
