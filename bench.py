@@ -218,9 +218,10 @@ class ClockSampler:
 # reference arm: the float64 oracle on the host cores
 # ---------------------------------------------------------------------------
 
-def oracle_sample_rate(wl, rows, repeats=1):
+def oracle_sample_rate(wl, rows, repeats=1, min_seconds=0.0):
     """Time the oracle (as it stands) on the compacted selected rows of the
-    given batch rows; returns (head*keys/s, seconds, threads)."""
+    given batch rows, `repeats` passes and then more until `min_seconds` of
+    CPU work have run; returns (head*keys/s, seconds, threads, passes)."""
     import numpy as np
 
     import mla_inputs as mi
@@ -239,13 +240,15 @@ def oracle_sample_rate(wl, rows, repeats=1):
                          r[None, :, 512:], np.arange(n)[None], np.array([n])))
     wkv = mi.f64(wl.wkv_b)
     keys = 0
+    passes = 0
     t0 = time.perf_counter()
-    for _ in range(repeats):
+    while passes < repeats or time.perf_counter() - t0 < min_seconds:
         for qn, qp, c, pe, idx, ep in prepared:
             orc.decode_absorbed(qn, qp, wkv, c, pe, idx, ep, wl.scale)
             keys += idx.shape[1]
+        passes += 1
     dt = time.perf_counter() - t0
-    return keys * HEADS / dt, dt, threads
+    return keys * HEADS / dt, dt, threads, passes
 
 
 def run_reference(args):
@@ -263,7 +266,7 @@ def run_reference(args):
         oracle_sample_rate(wl, rows[:1])
     rates, secs, threads = [], 0.0, 1
     for _ in range(args.steps):
-        r, dt, threads = oracle_sample_rate(wl, rows)
+        r, dt, threads, _ = oracle_sample_rate(wl, rows)
         rates.append(r)
         secs += dt
     value = len(rates) * len(rows) * wl.k * HEADS / secs
@@ -458,10 +461,10 @@ def run_ours(args):
     # ---- CPU baseline: the oracle on a bounded sample, rank 0 at N=1 ----
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         rows = list(range(min(args.cpu_rows, B)))
-        rate, dt, threads = oracle_sample_rate(wl, rows)
+        rate, dt, threads, passes = oracle_sample_rate(wl, rows, min_seconds=args.cpu_seconds)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
                                 "sample": f"{len(rows)} of {B} batch rows (their selected rows "
-                                          f"only), one pass, {dt:.1f} s"}
+                                          f"only), {passes} passes, {dt:.1f} s"}
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -479,6 +482,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", type=int, default=3, choices=[0, 1, 2, 3, 4])
     ap.add_argument("--cpu-rows", type=int, default=128)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="minimum seconds of oracle work in the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:

@@ -149,9 +149,10 @@ __global__ void __launch_bounds__(128) fold_kernel(const __nv_bfloat16* __restri
 // The flattened list of key tiles (batch row b, tile j of row b) is cut into
 // one contiguous range per cluster, so every cluster gets the same number of
 // tiles whatever B and k are.  A range covers one or more "segments" (the
-// part of one batch row it holds); each segment ends with a partial output
-// (O~ normalised by its own sum, plus its log-sum-exp) that the merge kernel
-// combines.
+// part of one batch row it holds); a segment that is the whole row ends with
+// the row's normalised O~, any other segment with a partial output (O~
+// normalised by its own sum, plus its log-sum-exp) that the combine kernel
+// merges.
 //
 // CTA r of the pair owns latent columns [256r, 256r+256) and rotary columns
 // [32r, 32r+32) of Q~ and of every selected cache row; both CTAs hold all 128
@@ -161,23 +162,23 @@ __global__ void __launch_bounds__(128) fold_kernel(const __nv_bfloat16* __restri
 //                                        keys -inf), rounded to fp16 and
 //                                        exchanged through DSMEM; added, maxed
 //                                        and exponentiated as fp16 pairs
-//   P            = 2^(S - m)             running max m; row sum l on the
-//                                        tensor core (P x ones)
+//   P            = 2^(S - m)             running max m, lazily raised; row
+//                                        sum l on the CUDA cores
 //   O_half      += P V_half              M=128, N=256, K=KT          (tcgen05)
 // V is the same shared-memory tile as K, read MN-major.
 //
-// Warp roles (384 threads):
-//   warps 0-7  softmax: warps w and w+4 share the TMEM lanes 32(w%4).. (head
-//              rows) and take keys [0,32) / [32,64) of each tile; the two
-//              halves of a row combine their maxima through shared memory.
-//              They also load this CTA's half of Q~ into TMEM at each segment
-//              start and write the segment outputs
-//   warps 8-10 gather: TMA tile::gather4 of the selected rows (4 rows per
-//              instruction); group g of four keys goes to warp 8 + g % 3
-//   warp 11    TMEM owner and MMA issuer (one thread)
-// TMEM (512 columns): S [0,KT), Q~ half [64,208) as bf16 pairs, row sums
-// [208,224) (P times a ones tile, so l sums exactly the bf16 P the value
-// product uses), P [224,256) as bf16 pairs, O half [256,512) fp32.
+// Warp roles (512 threads; setmaxnreg gives the softmax warps 176 registers
+// and the others 80):
+//   warps 0-7   softmax: warp w covers head rows [32(w%4) + 16(w/4), +16)
+//               through 16x256b TMEM fragments, four threads per row.  They
+//               also load this CTA's half of Q~ at each segment start and
+//               write the segment outputs
+//   warps 8-14  gather: TMA tile::gather4 of the selected rows (4 rows per
+//               instruction); group g of four keys goes to warp 8 + g % 7
+//   warp 15     TMEM owner and MMA issuer (one thread)
+// TMEM (512 columns): latent half of Q~ [0,128) as bf16 pairs, S [128,192),
+// two P buffers [192,256) as bf16 pairs, O half [256,512) fp32.  The rotary
+// half of Q sits in shared memory (64 B swizzle).
 // ===========================================================================
 // packed fp16 pair helpers (low half = first element)
 DEV uint32_t f16x2_from_f32_sat(float lo, float hi) {
