@@ -254,6 +254,26 @@ DEV void tc_mma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_
       : "memory");
 }
 
+// The two MMA forms above with the accumulate flag fixed at compile time
+template <bool kAccumulate>
+DEV void tc_mma_c(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "n"(kAccumulate ? 1 : 0)
+      : "memory");
+}
+template <bool kAccumulate>
+DEV void tc_mma_tmem_a_c(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "n"(kAccumulate ? 1 : 0)
+      : "memory");
+}
+
 // TMA gather of four rows (y0..y3) of a 2-D tensor, one box wide starting at
 // column x, into consecutive box rows at dst; completion counted in bytes on
 // the CTA-local mbarrier.  Rows outside the tensor are filled with zeros.
@@ -364,6 +384,20 @@ DEV uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes, u
   d |= static_cast<uint64_t>(1u) << 46;
   d |= static_cast<uint64_t>(layout & 7u) << 61;
   return d;
+}
+
+// The same descriptor in two 32-bit words: the low word (start address and
+// leading byte offset) changes with the tile position, the high word (stride
+// byte offset, version, layout) does not.  For a start address a + off inside
+// shared memory, desc_lo(a + off, lbo) == desc_lo(a, lbo) + off / 16.
+DEV uint32_t desc_lo(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+__host__ __device__ constexpr uint32_t desc_hi(uint32_t sbo_bytes, uint32_t layout) {
+  return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | ((layout & 7u) << 29);
+}
+DEV uint64_t desc_join(uint32_t lo, uint32_t hi) {
+  return (static_cast<uint64_t>(hi) << 32) | lo;
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation.

@@ -460,7 +460,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, KT, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, 0, 1);
+      // descriptors: a stage's low word plus a constant per K-step
+      constexpr uint32_t hi_k128 = desc_hi(1024, kSwizzle128B);  // K-major, 128 B swizzle
+      constexpr uint32_t hi_k64 = desc_hi(512, kSwizzle64B);     // K-major, 64 B swizzle
+      const uint32_t lo_qr = desc_lo(sbase + OFF_QR, 16);        // rotary half of Q
       int qk = 0, pv = 0, idle = 0, qseg = -1;
+      int qs = 0, qph = 0, ps = 0;  // stage of the next score product (and its phase), value product
       int jq = jt0, jp = jt0;  // tile-in-row of the next score / value product
       bool alive = true;
       uint64_t t_idle = 0;  // when the current idle stretch was first checked (0: not yet)
@@ -470,44 +475,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
         bool did = false;
         if (pv < qk && mbar_test(&bars.p_full[pv & 1], (pv >> 1) & 1)) {
           tc_fence_after();
-          const int s = pv % NST;
-          const uint32_t st = sbase + OFF_ST + s * ST_BYTES;
+          const int s = ps;
+          const uint32_t lo = desc_lo(sbase + OFF_ST + s * ST_BYTES, ST_ATOM);  // V, MN-major
           const uint32_t tp = tmem + T_P + (pv & 1) * (KT / 2);
           const bool first = pv == 0 || jp == 0;
+          if (first)
+            tc_mma_tmem_a_c<false>(tmem + T_O, tp, desc_join(lo, hi_k128), idesc_pv);
+          else
+            tc_mma_tmem_a_c<true>(tmem + T_O, tp, desc_join(lo, hi_k128), idesc_pv);
 #pragma unroll
-          for (int ks = 0; ks < KT / 16; ++ks) {
-            const uint64_t bd = smem_desc(st + ks * 2048, ST_ATOM, 1024, kSwizzle128B);
-            tc_mma_tmem_a(tmem + T_O, tp + ks * 8, bd, idesc_pv, (!first || ks > 0) ? 1u : 0u);
-          }
+          for (int ks = 1; ks < KT / 16; ++ks)
+            tc_mma_tmem_a_c<true>(tmem + T_O, tp + ks * 8, desc_join(lo + ks * (2048 >> 4), hi_k128),
+                                  idesc_pv);
           tc_commit(&bars.o_done[pv & 1]);
           tc_commit(&bars.empty[s]);
           ++pv;
+          if (++ps == NST) ps = 0;
           if (++jp == nt) jp = 0;
           did = true;
           SHLA_T(1);
         }
-        if (qk < n && mbar_test(&bars.full[qk % NST], (qk / NST) & 1) &&
+        if (qk < n && mbar_test(&bars.full[qs], qph) &&
             (qk == 0 || mbar_test(&bars.s_empty, (qk - 1) & 1))) {
           const int seg = (qk == 0 || jq == 0) ? qseg + 1 : qseg;
           if (seg == qseg || mbar_test(&bars.q_ready, seg & 1)) {
             qseg = seg;
             tc_fence_after();
-            const uint32_t st = sbase + OFF_ST + (qk % NST) * ST_BYTES;
+            const uint32_t st = sbase + OFF_ST + qs * ST_BYTES;
+            const uint32_t lo = desc_lo(st, 16), lo_r = desc_lo(st + ST_KR, 16);
             const uint32_t ts = tmem + T_S;
+            tc_mma_tmem_a_c<false>(ts, tmem + T_Q, desc_join(lo, hi_k128), idesc_qk);
 #pragma unroll
-            for (int ks = 0; ks < 16; ++ks) {
-              const uint64_t bd =
-                  smem_desc(st + (ks >> 2) * ST_ATOM + (ks & 3) * 32, 16, 1024, kSwizzle128B);
-              tc_mma_tmem_a(ts, tmem + T_Q + ks * 8, bd, idesc_qk, ks > 0);
-            }
+            for (int ks = 1; ks < 16; ++ks)
+              tc_mma_tmem_a_c<true>(
+                  ts, tmem + T_Q + ks * 8,
+                  desc_join(lo + (((ks >> 2) * ST_ATOM + (ks & 3) * 32) >> 4), hi_k128), idesc_qk);
 #pragma unroll
-            for (int ks = 0; ks < 2; ++ks) {
-              const uint64_t ad = smem_desc(sbase + OFF_QR + ks * 32, 16, 512, kSwizzle64B);
-              const uint64_t bd = smem_desc(st + ST_KR + ks * 32, 16, 512, kSwizzle64B);
-              tc_mma(ts, ad, bd, idesc_qk, 1);
-            }
+            for (int ks = 0; ks < 2; ++ks)
+              tc_mma_c<true>(ts, desc_join(lo_qr + ks * 2, hi_k64), desc_join(lo_r + ks * 2, hi_k64),
+                             idesc_qk);
             tc_commit(&bars.s_full);
             ++qk;
+            if (++qs == NST) {
+              qs = 0;
+              qph ^= 1;
+            }
             if (++jq == nt) jq = 0;
             did = true;
             SHLA_T(2);
