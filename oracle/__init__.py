@@ -11,6 +11,7 @@ from .mla_oracle import (  # noqa: F401
     fold_wuk,
     index_mask,
     mix_latent,
+    out_proj,
     parameter_counts,
     rmsnorm,
     rope,

@@ -21,6 +21,8 @@ Sources (page title, section):
   * "KV compression" (the key-value down-projection excerpt) and "Rotated
     shared key" (the apply_rotary_emb excerpt): cache write and rotary
     embedding.
+  * "Mix and project" (the output projection wo and its parameter count):
+    Delta_attn = flatten(O) W_O^T.
 
 Readings taken where the pages are silent:
   * index semantics follow the decode mask built by scatter of 0 into a -inf
@@ -238,6 +240,23 @@ def cache_write(x, w_kva, norm_w, eps, R_pos, C, interleaved=True):
     lat = rmsnorm(lat, norm_w, eps)
     pe = rope(pe[:, None, :], R_pos, interleaved)[:, 0, :]
     return lat, pe
+
+
+# ---------------------------------------------------------------------------
+# output projection ("Mix and project": the output projection wo, the only
+# step that mixes heads; Delta_attn [B, dim])
+# ---------------------------------------------------------------------------
+
+
+def out_proj(o, w_o):
+    """Delta[b, n] = sum over heads h and value dims d of O[b,h,d] * W_O[n, h*Dv + d].
+
+    O [B, H, Dv] is flattened over (head, value dim) in that order, as the
+    decode excerpt's wo(x.flatten(2)) does; W_O is stored [out, in] =
+    [dim, H*Dv] and applied as x W_O^T."""
+    o = np.asarray(o, dtype=np.float64)
+    x = o.reshape(o.shape[0], -1)
+    return x @ np.asarray(w_o, dtype=np.float64).T
 
 
 # ---------------------------------------------------------------------------

@@ -34,6 +34,12 @@ ROPE_PINS = [
     pins.test_cache_write_with_selection_weights,
 ]
 NORM_PINS = [pins.test_rmsnorm_unit_rms, pins.test_cache_write_with_selection_weights]
+OUT_PROJ_PINS = [
+    pins.test_out_proj_one_hot_selects_a_weight_column,
+    pins.test_out_proj_is_linear,
+    pins.test_out_proj_mixes_heads_under_a_joint_permutation_only,
+    pins.test_out_proj_brute_force,
+]
 
 
 def _fold_wrong_rows(q_nope, wkv_b):
@@ -124,6 +130,25 @@ def _rmsnorm_sum_not_mean(x, w, eps):
     return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps) * np.asarray(w)
 
 
+def _out_proj_dim_major(o, w_o):
+    # flattens O value-dim-major instead of head-major
+    o = np.asarray(o, dtype=np.float64)
+    return np.swapaxes(o, 1, 2).reshape(o.shape[0], -1) @ np.asarray(w_o).T
+
+
+def _out_proj_drop_last_head(o, w_o):
+    o = np.array(o, dtype=np.float64)
+    o[:, -1, :] = 0.0
+    return o.reshape(o.shape[0], -1) @ np.asarray(w_o).T
+
+
+def _out_proj_untransposed(o, w_o):
+    # weight read [in, out] although it is stored [out, in]
+    o = np.asarray(o, dtype=np.float64)
+    w = np.asarray(w_o, dtype=np.float64)
+    return o.reshape(o.shape[0], -1) @ w.reshape(w.shape[1], w.shape[0])
+
+
 _orig_rope = om.rope
 
 MUTANTS = [
@@ -143,6 +168,9 @@ MUTANTS = [
     ("rope", _rope_swapped_pairs, ROPE_PINS),
     ("rmsnorm", _rmsnorm_no_sqrt, NORM_PINS),
     ("rmsnorm", _rmsnorm_sum_not_mean, NORM_PINS),
+    ("out_proj", _out_proj_dim_major, OUT_PROJ_PINS),
+    ("out_proj", _out_proj_drop_last_head, OUT_PROJ_PINS),
+    ("out_proj", _out_proj_untransposed, OUT_PROJ_PINS),
 ]
 
 

@@ -369,6 +369,61 @@ def test_cache_write_with_selection_weights():
 # numbers printed on the pages
 # ---------------------------------------------------------------------------
 
+def _out_proj_problem(seed, B=3, H=4, Dv=5, dim=7):
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal((B, H, Dv)), rng.standard_normal((dim, H * Dv))
+
+
+def test_out_proj_one_hot_selects_a_weight_column():
+    """A single 1 at head h, value dim d of O picks column h*Dv + d of W_O
+    ([out, in] storage, O flattened head-major as wo(x.flatten(2)) does)."""
+    _, w = _out_proj_problem(0)
+    B, H, Dv = 3, 4, 5
+    for b, h, d in [(0, 0, 0), (1, 2, 3), (2, 3, 4), (0, 1, 0)]:
+        o = np.zeros((B, H, Dv))
+        o[b, h, d] = 1.0
+        out = orc.out_proj(o, w)
+        assert np.array_equal(out[b], w[:, h * Dv + d])
+        others = [i for i in range(B) if i != b]
+        assert not out[others].any()
+
+
+def test_out_proj_is_linear():
+    o1, w = _out_proj_problem(1)
+    o2, _ = _out_proj_problem(2)
+    a = -1.75
+    lhs = orc.out_proj(a * o1 + o2, w)
+    rhs = a * orc.out_proj(o1, w) + orc.out_proj(o2, w)
+    assert np.abs(lhs - rhs).max() <= 1e-12 * (1 + np.abs(rhs).max())
+
+
+def test_out_proj_mixes_heads_under_a_joint_permutation_only():
+    """Renumbering the heads of O together with the matching column blocks of
+    W_O leaves Delta unchanged; renumbering O alone does not (the projection
+    is the step that mixes heads)."""
+    o, w = _out_proj_problem(3)
+    H, Dv = 4, 5
+    perm = np.array([2, 0, 3, 1])
+    cols = (perm[:, None] * Dv + np.arange(Dv)[None, :]).reshape(-1)
+    ref = orc.out_proj(o, w)
+    assert np.abs(orc.out_proj(o[:, perm, :], w[:, cols]) - ref).max() <= 1e-12 * np.abs(ref).max()
+    assert np.abs(orc.out_proj(o[:, perm, :], w) - ref).max() > 1e-3
+
+
+def test_out_proj_brute_force():
+    o, w = _out_proj_problem(4)
+    B, H, Dv = o.shape
+    want = np.zeros((B, w.shape[0]))
+    for b in range(B):
+        for n in range(w.shape[0]):
+            acc = 0.0
+            for h in range(H):
+                for d in range(Dv):
+                    acc += o[b, h, d] * w[n, h * Dv + d]
+            want[b, n] = acc
+    assert np.abs(orc.out_proj(o, w) - want).max() <= 1e-12 * (1 + np.abs(want).max())
+
+
 def test_parameter_counts_match_the_pages():
     gold = json.load(open(os.path.join(GOLD, "param_counts.json")))
     pc = orc.parameter_counts()
