@@ -226,6 +226,24 @@ int mla_gather_rows(const mla_bf16_t* c_kv, int64_t ckv_bstride, int ckv_rstride
 /* Number of key splits mla_decode uses for (B, k) on the current device. */
 int mla_decode_num_splits(int B, int k);
 
+/*
+ * Output projection of the attention block ("Mix and project" page: the
+ * output projection wo, the only step that mixes heads, 16,384 x 7,168
+ * weights; the decode excerpt applies it as wo(x.flatten(2))):
+ *   Delta[b, n] = sum over h, d of O[b, h, d] W_O[n, h * 128 + d]
+ *     O      bf16 [B, 128, 128]   (the mla_decode output; flattened head-major)
+ *     w_o    bf16 [7168, 16384]   ([out, in] storage)
+ *     delta  bf16 [B, 7168]
+ * fp32 accumulation.  A row tile of W_O whose K range is split between CTAs
+ * is summed from fp32 partials in a fixed order, so the result is the same
+ * on every run.  Requires 1 <= B <= 65535 and a caller-owned device
+ * workspace of at least mla_out_proj_workspace_bytes(B) bytes, 256-byte
+ * aligned (MLA_ERR_WORKSPACE otherwise).  status may be NULL (see above).
+ */
+size_t mla_out_proj_workspace_bytes(int B);
+int mla_out_proj(const mla_bf16_t* O, const mla_bf16_t* w_o, int B, mla_bf16_t* delta, void* ws,
+                 size_t ws_bytes, int32_t* status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -268,6 +268,16 @@ def make_cache_write(rows=32, T=64, write_pos=None, seed=0, device="cpu",
     return x, w_kva, norm_w, rope_table(T).to(device), write_pos
 
 
+def make_out_proj(B=8, seed=0, device="cpu", o_std=0.035):
+    """Inputs of the output projection: O [B,128,128] with the spread of the
+    decode outputs of the workloads (std ~0.035) and W_O [7168, 16384]
+    ([out, in]) with variance 1/16384."""
+    g = _gen(90_000 + seed, device)
+    o = _normal_bf16((B, H, DV), o_std, g, device)
+    w_o = _normal_bf16((DIM, H * DV), 1.0 / math.sqrt(H * DV), g, device)
+    return o, w_o
+
+
 def make_rope_input(B=2, S=5, Hx=128, seed=0, device="cpu"):
     g = _gen(80_000 + seed, device)
     return _normal_bf16((B, S, Hx, R), 1.0, g, device)

@@ -19,6 +19,8 @@ from ._lib import (  # noqa: F401
     mla_fold_wuk,
     mla_gather_rows,
     mla_index_mask,
+    mla_out_proj,
+    mla_out_proj_workspace_bytes,
     mla_rope,
     status_string,
 )

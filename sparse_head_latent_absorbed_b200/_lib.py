@@ -36,6 +36,8 @@ _SIGS = {
                                   _c_int, _c_int, _vp, _c_int, _vp, _c_int, _c_float, _vp, _vp,
                                   _c_size, _vp, _vp]),
     "mla_fold_wuk": (_c_int, [_vp, _vp, _c_int, _vp, _vp]),
+    "mla_out_proj_workspace_bytes": (_c_size, [_c_int]),
+    "mla_out_proj": (_c_int, [_vp, _vp, _c_int, _vp, _vp, _c_size, _vp, _vp]),
     "mla_index_mask": (_c_int, [_vp, _c_int, _c_int, _vp, _c_int, _vp, _vp, _vp]),
     "mla_gather_rows": (_c_int, [_vp, _c_i64, _c_int, _vp, _c_i64, _c_int, _c_int, _vp,
                                  _c_int, _c_int, _vp, _vp, _vp, _vp]),
@@ -136,6 +138,30 @@ def mla_cache_write(x: torch.Tensor, w_kva: torch.Tensor, norm_w: torch.Tensor, 
                                B, S, int(start_pos), _p(c_kv), cbs, crs, _p(k_pe), kbs, krs,
                                cache.shape[1], _p(ws), ws.numel(), _stream(x.device)),
            "mla_cache_write")
+
+
+def mla_out_proj_workspace_bytes(B: int) -> int:
+    return int(LIB.mla_out_proj_workspace_bytes(int(B)))
+
+
+def mla_out_proj(O: torch.Tensor, w_o: torch.Tensor, out: Optional[torch.Tensor] = None,
+                 ws: Optional[torch.Tensor] = None,
+                 status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Delta = flatten(O) W_O^T: O bf16 [B, 128, 128], w_o bf16 [7168, 16384]
+    ([out, in]) -> bf16 [B, 7168]."""
+    _need(O, torch.bfloat16, "O")
+    _need(w_o, torch.bfloat16, "w_o")
+    B = O.shape[0]
+    if out is None:
+        out = torch.empty(B, w_o.shape[0], dtype=torch.bfloat16, device=O.device)
+    need = mla_out_proj_workspace_bytes(B)
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=O.device)
+    _check(LIB.mla_out_proj(_p(O.contiguous()), _p(w_o.contiguous()), B, _p(out), _p(ws),
+                            ws.numel(), _p(status) if status is not None else None,
+                            _stream(O.device)),
+           "mla_out_proj")
+    return out
 
 
 NOALLOC_MAX_ROWS = 64

@@ -1,0 +1,322 @@
+// Output projection of the attention block ("Mix and project" page: the
+// output projection wo, the only step that mixes heads; its parameter table
+// gives 16,384 x 7,168 = 117,440,512 weights):
+//
+//   Delta[b, n] = sum_k x[b, k] W_O[n, k],   x = O[b] flattened head-major
+//
+// with O [B, 128, 128] bf16 (the decode output), W_O [7168, 16384] bf16 stored
+// [out, in], Delta [B, 7168] bf16.  The step reads 235 MB of weights for a
+// few MB of activations, so it is HBM-bound on W_O.
+//
+//   oproj_kernel     swap-AB GEMM on tcgen05: D^T[n, b] with 128 rows of W_O
+//                    as M, the batch as N (up to 128 per block), K = 16384 in
+//                    chunks of 64 through a 4-stage TMA ring.  Persistent CTAs
+//                    take equal slices of the flattened (row tile, K chunk)
+//                    list, so every SM streams the same number of weight
+//                    bytes; a slice covers the end of one row tile and the
+//                    start of the next, each part ("segment") ending with an
+//                    fp32 partial in its slot of the workspace.
+//   oproj_finalize   sums the slots of each row tile in slot order (a fixed
+//                    order: the result does not depend on timing) and rounds
+//                    to bf16.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "host_util.h"
+
+namespace shla {
+namespace oproj {
+
+constexpr int K_IN = 128 * 128;     // 16384 inputs: 128 heads x 128 value dims, head-major
+constexpr int N_OUT = 7168;         // model dimension
+constexpr int KC = 64;              // K per chunk: one 128-byte swizzle atom of bf16
+constexpr int NCHUNK = K_IN / KC;   // 256 chunks per row tile
+constexpr int MT = N_OUT / 128;     // 56 row tiles of W_O
+constexpr int NST = 4;              // ring depth
+constexpr int STAGE = 2 * 16384;    // A: 128 W_O rows x 64 k; B: up to 128 batch rows x 64 k
+constexpr int SMEM_BYTES = NST * STAGE + 1024;
+constexpr int NTHREADS = 192;       // warps 0-3 epilogue, warp 4 loads, warp 5 MMA + TMEM
+constexpr int kMaxSlots = 8;        // partial slots per row tile (a schedule bound)
+static_assert(K_IN % KC == 0 && N_OUT % 128 == 0, "tiling");
+
+// Slices of the flattened list of MT x NCHUNK units: CTA c owns units
+// [bnd(c), bnd(c+1)); row tile m covers units [m NCHUNK, (m+1) NCHUNK).
+struct Sched {
+  int tot;  // MT * NCHUNK
+  int nc;   // CTAs per batch block
+  __host__ __device__ int bnd(int c) const { return (int)((long long)c * tot / nc); }
+  // first / last CTA whose slice meets row tile m
+  __host__ __device__ int c_first(int m) const {
+    return (int)((((long long)m * NCHUNK + 1) * nc + tot - 1) / tot) - 1;
+  }
+  __host__ __device__ int c_last(int m) const {
+    return (int)((((long long)(m + 1) * NCHUNK) * nc + tot - 1) / tot) - 1;
+  }
+};
+
+// TMA tiled load of one box (no multicast) at (x, y), bytes counted on bar
+DEV void tma_load_tile(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+struct Bars {
+  uint64_t full[NST], empty[NST];
+  uint64_t seg_done;   // a segment's products have completed (MMA commit)
+  uint64_t tmem_free;  // the epilogue has read the accumulator (128 threads)
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+}  // namespace oproj
+
+// ---------------------------------------------------------------------------
+// D^T[n, b] = sum_k W_O[n, k] x[b, k] over this CTA's slice of (row tile,
+// K chunk) units, for batch rows [b0, b0 + 128).
+//   A = W_O rows (M = 128, K = 64 per chunk), K-major, 128-byte swizzle
+//   B = x rows   (N = 128 batch rows),         K-major, 128-byte swizzle
+// Rows of the B box beyond B hold stale data; only their own columns of D
+// are affected, and those are not stored.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(oproj::NTHREADS, 1)
+    oproj_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
+                 float* __restrict__ part, int B, int a_rows, oproj::Sched sch,
+                 int32_t* status) {
+  using namespace oproj;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));  // swizzle atoms: 1 KB aligned
+  const uint32_t sbase = smem_u32(smem);
+  __shared__ Bars bars;
+  volatile int* abort = &bars.abort;
+  const int c = blockIdx.x, b0 = blockIdx.y * 128;
+  const int u0 = sch.bnd(c), u1 = sch.bnd(c + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (warp == 5) {
+    tmem_alloc(&bars.tmem_base, 128);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&bars.full[s], 1);   // the loader's expect_tx arrival + bytes
+      mbar_init(&bars.empty[s], 1);  // MMA commit
+    }
+    mbar_init(&bars.seg_done, 1);
+    mbar_init(&bars.tmem_free, 128);
+    mbar_init(&bars.drain, 1);
+    bars.abort = 0;
+    fence_mbarrier_init_cluster();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars.tmem_base;
+
+  if (warp == 4) {
+    // ---------------- loads ----------------
+    if (lane == 0) {
+      int issued = 0;
+#pragma unroll 1
+      for (int u = u0; u < u1; ++u) {
+        const int i = u - u0, s = i % NST;
+        if (!mbar_wait(&bars.empty[s], ((i / NST) & 1) ^ 1, abort, status)) break;
+        mbar_arrive_expect_tx(&bars.full[s], 16384 + 128 * a_rows);
+        const int m = u / NCHUNK, ch = u - m * NCHUNK;
+        const uint32_t st = sbase + s * STAGE;
+        tma_load_tile(st, &map_w, ch * KC, m * 128, &bars.full[s]);
+        tma_load_tile(st + 16384, &map_x, ch * KC, b0, &bars.full[s]);
+        issued = i + 1;
+      }
+      // on an abort, loads still in flight land before the CTA can leave
+      for (int i = max(0, issued - NST); i < issued; ++i)
+        mbar_wait(&bars.full[i % NST], (i / NST) & 1, nullptr, nullptr);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t hi = desc_hi(1024, kSwizzle128B);
+      int seg = 0;
+#pragma unroll 1
+      for (int u = u0; u < u1; ++u) {
+        const int i = u - u0, s = i % NST;
+        const int ch = u % NCHUNK;
+        const bool first = u == u0 || ch == 0, last = u == u1 - 1 || ch == NCHUNK - 1;
+        if (!mbar_wait(&bars.full[s], (i / NST) & 1, abort, status)) break;
+        // a new segment overwrites the accumulator once the epilogue has read it
+        if (first && seg > 0 && !mbar_wait(&bars.tmem_free, (seg - 1) & 1, abort, status)) break;
+        tc_fence_after();
+        const uint32_t la = desc_lo(sbase + s * STAGE, 16), lb = desc_lo(sbase + s * STAGE + 16384, 16);
+        if (first)
+          tc_mma_c<false>(tmem, desc_join(la, hi), desc_join(lb, hi), idesc);
+        else
+          tc_mma_c<true>(tmem, desc_join(la, hi), desc_join(lb, hi), idesc);
+#pragma unroll
+        for (int ks = 1; ks < KC / 16; ++ks)
+          tc_mma_c<true>(tmem, desc_join(la + ks * 2, hi), desc_join(lb + ks * 2, hi), idesc);
+        tc_commit(&bars.empty[s]);
+        if (last) {
+          tc_commit(&bars.seg_done);
+          ++seg;
+        }
+      }
+      // everything issued so far has finished before TMEM is released
+      tc_commit(&bars.drain);
+      mbar_wait(&bars.drain, 0, nullptr, status);
+    }
+    __syncwarp();
+  } else if (u1 > u0) {
+    // ---------------- epilogue (warps 0-3: TMEM lane = row of the tile) ----------------
+    // segment k of the slice is row tile m0 + k; its partial goes to slot
+    // c - c_first(m) as part[m][slot][b][row], 32 consecutive rows per store
+    const int m0 = u0 / NCHUNK, m1 = (u1 - 1) / NCHUNK;
+    const int nl = warp * 32 + lane;
+#pragma unroll 1
+    for (int m = m0, seg = 0; m <= m1; ++m, ++seg) {
+      if (!warp_wait(&bars.seg_done, seg & 1, abort, status)) break;
+      tc_fence_after();
+      const int slot = c - sch.c_first(m);
+      float* dst = part + (size_t)(m * kMaxSlots + slot) * B * 128 + nl;
+#pragma unroll 1
+      for (int col = 0; col < 128; col += 16) {
+        uint32_t r[16];
+        tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + col, r);
+        tc_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int b = b0 + col + j;
+          if (b < B) dst[(size_t)b * 128] = __uint_as_float(r[j]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars.tmem_free);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// Delta[b, n0 .. n0+7] = bf16(sum over the slots of row tile n0 / 128, in
+// slot order).  grid (B, N_OUT / 1024), 128 threads of 8 outputs each.
+__global__ void __launch_bounds__(128) oproj_finalize(const float* __restrict__ part,
+                                                       oproj::Sched sch, int B,
+                                                       __nv_bfloat16* __restrict__ out) {
+  using namespace oproj;
+  const int b = blockIdx.x;
+  const int n0 = (blockIdx.y * 128 + threadIdx.x) * 8;
+  if (n0 >= N_OUT) return;
+  const int m = n0 / 128, nl = n0 % 128;
+  const int used = sch.c_last(m) - sch.c_first(m) + 1;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+  for (int s = 0; s < used; ++s) {
+    const float4* src =
+        reinterpret_cast<const float4*>(part + ((size_t)(m * kMaxSlots + s) * B + b) * 128 + nl);
+    const float4 v0 = src[0], v1 = src[1];
+    acc[0] += v0.x;
+    acc[1] += v0.y;
+    acc[2] += v0.z;
+    acc[3] += v0.w;
+    acc[4] += v1.x;
+    acc[5] += v1.y;
+    acc[6] += v1.z;
+    acc[7] += v1.w;
+  }
+  uint4 o;
+  o.x = pack_bf16x2(acc[0], acc[1]);
+  o.y = pack_bf16x2(acc[2], acc[3]);
+  o.z = pack_bf16x2(acc[4], acc[5]);
+  o.w = pack_bf16x2(acc[6], acc[7]);
+  *reinterpret_cast<uint4*>(out + (size_t)b * N_OUT + n0) = o;
+}
+
+// ---------------------------------------------------------------------------
+// host
+// ---------------------------------------------------------------------------
+typedef CUresult (*OprojEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static OprojEncodeFn oproj_encode() {
+  static OprojEncodeFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<OprojEncodeFn>(f);
+  }
+  return fn;
+}
+
+// 2-D map over a row-major [rows][16384] bf16 matrix, boxes of 64 x box_rows
+static int oproj_map(CUtensorMap* map, const void* base, int rows, int box_rows) {
+  OprojEncodeFn fn = oproj_encode();
+  if (!fn) return MLA_ERR_CUDA;
+  const cuuint64_t dims[2] = {(cuuint64_t)oproj::K_IN, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)oproj::K_IN * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)oproj::KC, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// CTAs per batch block: one per SM, at most 384 so that a row tile meets at
+// most kMaxSlots slices (slices of >= 37 units against 256 units per tile)
+static oproj::Sched oproj_sched(int sms) {
+  oproj::Sched s;
+  s.tot = oproj::MT * oproj::NCHUNK;
+  s.nc = sms < 1 ? 1 : (sms > 384 ? 384 : sms);
+  return s;
+}
+
+}  // namespace shla
+
+using namespace shla;
+
+extern "C" size_t mla_out_proj_workspace_bytes(int B) {
+  if (B < 1 || B > 65535) return 0;
+  return round_up((size_t)oproj::MT * oproj::kMaxSlots * B * 128 * sizeof(float), 256);
+}
+
+extern "C" int mla_out_proj(const mla_bf16_t* O, const mla_bf16_t* w_o, int B, mla_bf16_t* delta,
+                            void* ws, size_t ws_bytes, int32_t* status, void* stream) {
+  if (!O || !w_o || !delta) return MLA_ERR_NULL;
+  if (B < 1 || B > 65535) return MLA_ERR_SHAPE;
+  if (!aligned16(O) || !aligned16(w_o) || !aligned16(delta)) return MLA_ERR_ALIGN;
+  if (!ws || !aligned256(ws) || ws_bytes < mla_out_proj_workspace_bytes(B))
+    return MLA_ERR_WORKSPACE;
+  int sms = 0;
+  if (int e = check_device(&sms)) return e;
+  const oproj::Sched sch = oproj_sched(sms);
+  const int rows = B < 128 ? B : 128;
+  alignas(64) CUtensorMap map_w, map_x;
+  if (int e = oproj_map(&map_w, w_o, oproj::N_OUT, 128)) return e;
+  if (int e = oproj_map(&map_x, O, B, rows)) return e;
+  static unsigned long long attr_done = 0;
+  if (int e = ensure_smem_attr(oproj_kernel, oproj::SMEM_BYTES, &attr_done)) return e;
+  cudaStream_t st = as_stream(stream);
+  float* part = static_cast<float*>(ws);
+  oproj_kernel<<<dim3(sch.nc, (B + 127) / 128), oproj::NTHREADS, oproj::SMEM_BYTES, st>>>(
+      map_w, map_x, part, B, rows, sch, status);
+  if (int e = launch_status()) return e;
+  oproj_finalize<<<dim3(B, oproj::N_OUT / 1024), 128, 0, st>>>(
+      part, sch, B, reinterpret_cast<__nv_bfloat16*>(delta));
+  return launch_status();
+}

@@ -71,6 +71,14 @@ def test_null_and_shape_checks_before_any_cuda_call(lib):
     assert lib.mla_cache_write(dummy, dummy, dummy, 1e-6, dummy, 1, 1, 0, dummy, 0, 576,
                                dummy, 0, 576, 10, None, 0, None) == -4
     assert L.mla_cache_write_workspace_bytes(32) == 28 * 32 * 576 * 4
+    # output projection
+    assert lib.mla_out_proj(None, dummy, 1, dummy, dummy, 1 << 30, None, None) == -1
+    assert lib.mla_out_proj(dummy, dummy, 0, dummy, dummy, 1 << 30, None, None) == -2
+    assert lib.mla_out_proj(dummy, odd, 1, dummy, dummy, 1 << 30, None, None) == -3
+    assert lib.mla_out_proj(dummy, dummy, 4, dummy, dummy, 16, None, None) == -4
+    assert lib.mla_out_proj(dummy, dummy, 4, dummy, vp(4096 + 16), 1 << 30, None, None) == -4
+    assert L.mla_out_proj_workspace_bytes(0) == 0
+    assert L.mla_out_proj_workspace_bytes(128) >= 56 * 4 * 128 * 128 * 4
 
 
 def test_workspace_and_split_choice(lib):
