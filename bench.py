@@ -449,6 +449,34 @@ def run_ours(args):
         e_ms += a.elapsed_time(b_)
     e_ms = reduce_max(e_ms / n_e2e, world, dev)
 
+    # ---- the next row on the path: the output projection Delta = flatten(O) W_O^T ----
+    next_rows = {}
+    if not args.no_next_rows:
+        o_in, w_o = mi.make_out_proj(B=B, seed=1, device=dev)
+        d_out = torch.empty(B, 7168, dtype=torch.bfloat16, device=dev)
+        op_ws = torch.empty(shla.mla_out_proj_workspace_bytes(B), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            shla.mla_out_proj(o_in, w_o, out=d_out, ws=op_ws)
+        torch.cuda.synchronize()
+        op_ms = 0.0
+        n_op = max(3, min(args.steps, 100))
+        for _ in range(n_op):
+            flush_l2()
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            shla.mla_out_proj(o_in, w_o, out=d_out, ws=op_ws)
+            b_.record(stream)
+            torch.cuda.synchronize()
+            op_ms += a.elapsed_time(b_)
+        op_ms = reduce_max(op_ms / n_op, world, dev)
+        op_bytes = 7168 * 16384 * 2 + B * 16384 * 2 + B * 7168 * 2
+        next_rows["out_proj"] = {
+            "what": "Delta = flatten(O) W_O^T, W_O [7168, 16384] bf16 (oproj_kernel + finalize)",
+            "us": op_ms * 1e3, "bound": "hbm", "algorithmic_bytes": op_bytes,
+            "achieved": op_bytes / (op_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": op_bytes / (op_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+        del w_o
+
     units = B * k * HEADS
     value = world * units / (ms_per_step * 1e-3)
     line = {
@@ -466,6 +494,7 @@ def run_ours(args):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "algorithmic": dict(zip(("bytes_per_step", "flops_per_step"), algorithmic_work(B, k))),
+        "next_rows": next_rows,
     }
     # ---- CPU baseline: the oracle on a bounded sample, rank 0 at N=1 ----
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
@@ -494,6 +523,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="minimum seconds of oracle work in the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip the separate timing of the output projection")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
