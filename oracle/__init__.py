@@ -13,6 +13,7 @@ from .mla_oracle import (  # noqa: F401
     mix_latent,
     out_proj,
     parameter_counts,
+    query_proj,
     rmsnorm,
     rope,
     scores,

@@ -23,6 +23,8 @@ Sources (page title, section):
     embedding.
   * "Mix and project" (the output projection wo and its parameter count):
     Delta_attn = flatten(O) W_O^T.
+  * "Query rotary up-projection" (the MLA init and forward excerpts): the
+    query path wq_a -> q_norm -> wq_b -> split -> RoPE.
 
 Readings taken where the pages are silent:
   * index semantics follow the decode mask built by scatter of 0 into a -inf
@@ -240,6 +242,30 @@ def cache_write(x, w_kva, norm_w, eps, R_pos, C, interleaved=True):
     lat = rmsnorm(lat, norm_w, eps)
     pe = rope(pe[:, None, :], R_pos, interleaved)[:, 0, :]
     return lat, pe
+
+
+# ---------------------------------------------------------------------------
+# query path ("Query rotary up-projection": the MLA init and forward excerpts;
+# W_QR is output features Dn..Dn+Rr of each head's block in wq_b)
+# ---------------------------------------------------------------------------
+
+
+def query_proj(x, wq_a, q_norm_w, eps, wq_b, R_pos, n_heads, dn, interleaved=True):
+    """qr = RMSNorm(x wq_a^T) * w;  q = qr wq_b^T viewed [B, n_heads, dn + rr];
+    q_nope = q[..., :dn];  q_pe = RoPE(q[..., dn:]) at each row's position.
+
+    x [B, dim], wq_a [q_lora, dim] and wq_b [n_heads*(dn+rr), q_lora] stored
+    [out, in]; R_pos complex [B, rr/2] (the rotary coefficients of each row's
+    query position).  Returns (q_nope [B, n_heads, dn], q_pe [B, n_heads, rr])."""
+    t = np.asarray(x, dtype=np.float64) @ np.asarray(wq_a, dtype=np.float64).T
+    qr = rmsnorm(t, q_norm_w, eps)
+    q = qr @ np.asarray(wq_b, dtype=np.float64).T
+    B = q.shape[0]
+    q = q.reshape(B, n_heads, -1)
+    q_nope, q_pe = q[..., :dn], q[..., dn:]
+    # rope takes [..., S, Hx, Rr] with R [S, Rr/2]: treat the batch as positions
+    q_pe = rope(q_pe, np.asarray(R_pos), interleaved)
+    return q_nope, q_pe
 
 
 # ---------------------------------------------------------------------------

@@ -40,6 +40,12 @@ OUT_PROJ_PINS = [
     pins.test_out_proj_mixes_heads_under_a_joint_permutation_only,
     pins.test_out_proj_brute_force,
 ]
+QUERY_PINS = [
+    pins.test_query_proj_routes_heads_and_splits_nope_before_rope,
+    pins.test_query_proj_is_scale_invariant_through_the_norm,
+    pins.test_query_proj_position_moves_only_the_rotary_part,
+    pins.test_query_proj_brute_force,
+]
 
 
 def _fold_wrong_rows(q_nope, wkv_b):
@@ -149,6 +155,30 @@ def _out_proj_untransposed(o, w_o):
     return o.reshape(o.shape[0], -1) @ w.reshape(w.shape[1], w.shape[0])
 
 
+def _query_rope_first(x, wq_a, w, eps, wq_b, R_pos, n_heads, dn, interleaved=True):
+    # rotary part taken from the front of each head's block
+    qr = om.rmsnorm(np.asarray(x, dtype=np.float64) @ np.asarray(wq_a).T, w, eps)
+    q = (qr @ np.asarray(wq_b).T).reshape(qr.shape[0], n_heads, -1)
+    rr = q.shape[-1] - dn
+    return q[..., rr:], om.rope(q[..., :rr], np.asarray(R_pos), interleaved)
+
+
+def _query_norm_first(x, wq_a, w, eps, wq_b, R_pos, n_heads, dn, interleaved=True):
+    # normalises the input instead of the down-projection
+    xn = np.asarray(x, dtype=np.float64)
+    xn = xn / np.sqrt(np.mean(xn * xn, axis=-1, keepdims=True) + eps)
+    qr = (xn @ np.asarray(wq_a).T) * np.asarray(w)
+    q = (qr @ np.asarray(wq_b).T).reshape(qr.shape[0], n_heads, -1)
+    return q[..., :dn], om.rope(q[..., dn:], np.asarray(R_pos), interleaved)
+
+
+def _query_feature_major(x, wq_a, w, eps, wq_b, R_pos, n_heads, dn, interleaved=True):
+    # views the wq_b output feature-major instead of head-major
+    qr = om.rmsnorm(np.asarray(x, dtype=np.float64) @ np.asarray(wq_a).T, w, eps)
+    q = (qr @ np.asarray(wq_b).T).reshape(qr.shape[0], -1, n_heads).swapaxes(1, 2)
+    return q[..., :dn], om.rope(q[..., dn:], np.asarray(R_pos), interleaved)
+
+
 _orig_rope = om.rope
 
 MUTANTS = [
@@ -171,6 +201,9 @@ MUTANTS = [
     ("out_proj", _out_proj_dim_major, OUT_PROJ_PINS),
     ("out_proj", _out_proj_drop_last_head, OUT_PROJ_PINS),
     ("out_proj", _out_proj_untransposed, OUT_PROJ_PINS),
+    ("query_proj", _query_rope_first, QUERY_PINS),
+    ("query_proj", _query_norm_first, QUERY_PINS),
+    ("query_proj", _query_feature_major, QUERY_PINS),
 ]
 
 

@@ -424,6 +424,91 @@ def test_out_proj_brute_force():
     assert np.abs(orc.out_proj(o, w) - want).max() <= 1e-12 * (1 + np.abs(want).max())
 
 
+def _query_problem(seed, B=3, dim=10, ql=6, H=2, dn=4, rr=4):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((B, dim))
+    wa = rng.standard_normal((ql, dim))
+    w = 1.0 + 0.25 * rng.standard_normal(ql)
+    wb = rng.standard_normal((H * (dn + rr), ql))
+    R = np.exp(1j * rng.standard_normal((B, rr // 2)))
+    return x, wa, w, wb, R
+
+
+def test_query_proj_routes_heads_and_splits_nope_before_rope():
+    """wq_a = [I 0] and w = 1, eps = 0 make qr = x[:, :ql] / rms; a one-hot
+    wq_b sends qr[j] to (head h, feature e) of the head-major [H, dn + rr]
+    view; at position 0 (R = 1) features e < dn land in q_nope[h, e] and the
+    rest in q_pe[h, e - dn], exactly."""
+    B, dim, ql, H, dn, rr = 2, 9, 5, 3, 4, 6
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((B, dim))
+    wa = np.zeros((ql, dim))
+    wa[np.arange(ql), np.arange(ql)] = 1.0
+    t = x[:, :ql]
+    qr = t / np.sqrt(np.mean(t * t, axis=1, keepdims=True))
+    routes = [(0, 0, 0), (0, dn - 1, 1), (1, dn, 2), (2, dn + rr - 1, 4), (2, 1, 3)]
+    wb = np.zeros((H * (dn + rr), ql))
+    for h, e, j in routes:
+        wb[h * (dn + rr) + e, j] = 1.0
+    R0 = np.ones((B, rr // 2), dtype=complex)
+    qn, qp = orc.query_proj(x, wa, np.ones(ql), 0.0, wb, R0, H, dn)
+    assert qn.shape == (B, H, dn) and qp.shape == (B, H, rr)
+    want_n, want_p = np.zeros((B, H, dn)), np.zeros((B, H, rr))
+    for h, e, j in routes:
+        if e < dn:
+            want_n[:, h, e] = qr[:, j]
+        else:
+            want_p[:, h, e - dn] = qr[:, j]
+    assert np.abs(qn - want_n).max() <= 1e-12
+    assert np.abs(qp - want_p).max() <= 1e-12
+
+
+def test_query_proj_is_scale_invariant_through_the_norm():
+    """With eps = 0 the RMSNorm cancels any positive scale of x."""
+    x, wa, w, wb, R = _query_problem(6)
+    a = orc.query_proj(x, wa, w, 0.0, wb, R, 2, 4)
+    b = orc.query_proj(3.7 * x, wa, w, 0.0, wb, R, 2, 4)
+    for u, v in zip(a, b):
+        assert np.abs(u - v).max() <= 1e-12 * np.abs(u).max()
+
+
+def test_query_proj_position_moves_only_the_rotary_part():
+    x, wa, w, wb, R = _query_problem(7)
+    R2 = R * np.exp(1j * np.array([0.3, -1.1]))
+    n1, p1 = orc.query_proj(x, wa, w, 1e-6, wb, R, 2, 4)
+    n2, p2 = orc.query_proj(x, wa, w, 1e-6, wb, R2, 2, 4)
+    assert np.array_equal(n1, n2)
+    assert np.abs(p1 - p2).max() > 1e-3
+    pair = lambda p: p[..., 0::2] ** 2 + p[..., 1::2] ** 2  # noqa: E731
+    assert np.abs(pair(p1) - pair(p2)).max() <= 1e-12 * pair(p1).max()
+
+
+def test_query_proj_brute_force():
+    B, dim, ql, H, dn, rr = 2, 5, 4, 2, 3, 4
+    x, wa, w, wb, _ = _query_problem(8, B, dim, ql, H, dn, rr)
+    ang = np.random.default_rng(9).standard_normal((B, rr // 2))
+    R = np.cos(ang) + 1j * np.sin(ang)
+    eps = 1e-6
+    qn_want = np.zeros((B, H, dn))
+    qp_want = np.zeros((B, H, rr))
+    for b in range(B):
+        t = [sum(x[b, i] * wa[o, i] for i in range(dim)) for o in range(ql)]
+        ms = sum(v * v for v in t) / ql
+        qr = [t[o] / math.sqrt(ms + eps) * w[o] for o in range(ql)]
+        for h in range(H):
+            feats = [sum(qr[j] * wb[h * (dn + rr) + e, j] for j in range(ql)) for e in range(dn + rr)]
+            for e in range(dn):
+                qn_want[b, h, e] = feats[e]
+            for p in range(rr // 2):
+                x0, x1 = feats[dn + 2 * p], feats[dn + 2 * p + 1]
+                c, s_ = math.cos(ang[b, p]), math.sin(ang[b, p])
+                qp_want[b, h, 2 * p] = x0 * c - x1 * s_
+                qp_want[b, h, 2 * p + 1] = x0 * s_ + x1 * c
+    qn, qp = orc.query_proj(x, wa, w, eps, wb, R, H, dn)
+    assert np.abs(qn - qn_want).max() <= 1e-12 * (1 + np.abs(qn_want).max())
+    assert np.abs(qp - qp_want).max() <= 1e-12 * (1 + np.abs(qp_want).max())
+
+
 def test_parameter_counts_match_the_pages():
     gold = json.load(open(os.path.join(GOLD, "param_counts.json")))
     pc = orc.parameter_counts()
