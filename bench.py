@@ -476,6 +476,28 @@ def run_ours(args):
             "achieved": op_bytes / (op_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": op_bytes / (op_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
         del w_o
+        qx, wq_a, qn_w, wq_b, qrope, qpos = mi.make_query_proj(B=B, seed=1, device=dev)
+        q_ws = torch.empty(shla.mla_query_proj_workspace_bytes(B), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            shla.mla_query_proj(qx, wq_a, qn_w, 1e-6, wq_b, qrope, qpos, ws=q_ws)
+        torch.cuda.synchronize()
+        q_ms = 0.0
+        for _ in range(n_op):
+            flush_l2()
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            shla.mla_query_proj(qx, wq_a, qn_w, 1e-6, wq_b, qrope, qpos, ws=q_ws)
+            b_.record(stream)
+            torch.cuda.synchronize()
+            q_ms += a.elapsed_time(b_)
+        q_ms = reduce_max(q_ms / n_op, world, dev)
+        q_bytes = (1536 * 7168 + 24576 * 1536) * 2 + B * 7168 * 2 + B * 128 * 192 * 2
+        next_rows["query_proj"] = {
+            "what": "x -> wq_a -> RMSNorm -> wq_b -> split -> RoPE (2 x xwt_kernel + finishes)",
+            "us": q_ms * 1e3, "bound": "hbm", "algorithmic_bytes": q_bytes,
+            "achieved": q_bytes / (q_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": q_bytes / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+        del wq_a, wq_b
 
     units = B * k * HEADS
     value = world * units / (ms_per_step * 1e-3)
@@ -524,7 +546,7 @@ def main(argv=None):
                     help="minimum seconds of oracle work in the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-next-rows", action="store_true",
-                    help="skip the separate timing of the output projection")
+                    help="skip the separate timing of the output projection and query path")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

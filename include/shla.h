@@ -244,6 +244,31 @@ size_t mla_out_proj_workspace_bytes(int B);
 int mla_out_proj(const mla_bf16_t* O, const mla_bf16_t* w_o, int B, mla_bf16_t* delta, void* ws,
                  size_t ws_bytes, int32_t* status, void* stream);
 
+/*
+ * Query path ("Query rotary up-projection" page: the MLA init and forward
+ * excerpts; W_QR is output features 128-191 of each head's 192 in wq_b):
+ *   qr[b, :]   = RMSNorm(x[b] wq_a^T) * q_norm_w   (fp32 norm, qr rounded to bf16)
+ *   q[b, h, :] = (qr[b] wq_b^T)[192 h .. 192 h + 191]
+ *   q_nope[b, h, :] = q[b, h, 0:128]
+ *   q_pe[b, h, :]   = interleaved rotation of q[b, h, 128:192] by rope[pos[b]]
+ *     x        bf16 [B, 7168]
+ *     wq_a     bf16 [1536, 7168]       ([out, in])
+ *     q_norm_w bf16 [1536], eps >= 0   (RMSNorm y = x / sqrt(mean(x^2) + eps) * w)
+ *     wq_b     bf16 [24576, 1536]      ([out, in], 128 heads x (128 + 64))
+ *     rope     fp32 [T, 32, 2]         ((cos, sin) per position and pair)
+ *     pos      int32 [B]               (the query position of each row)
+ *     q_nope   bf16 [B, 128, 128], q_pe bf16 [B, 128, 64]: the mla_decode inputs
+ * A row whose pos is outside [0, T) gets q_pe = 0 and is counted in
+ * status[1].  Partials are summed in a fixed order (results identical on
+ * every run).  Requires 1 <= B <= 65535 and a device workspace of at least
+ * mla_query_proj_workspace_bytes(B) bytes, 256-byte aligned.
+ */
+size_t mla_query_proj_workspace_bytes(int B);
+int mla_query_proj(const mla_bf16_t* x, const mla_bf16_t* wq_a, const mla_bf16_t* q_norm_w,
+                   float eps, const mla_bf16_t* wq_b, const float* rope, int T,
+                   const int32_t* pos, int B, mla_bf16_t* q_nope, mla_bf16_t* q_pe, void* ws,
+                   size_t ws_bytes, int32_t* status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

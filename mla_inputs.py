@@ -30,6 +30,7 @@ DN = 128         # non-rotary query/key part per head (qk_nope_head_dim)
 DV = 128         # value width per head (v_head_dim)
 KROW = C + R     # 576 cached values per position
 DIM = 7168       # model width
+QL = 1536        # query latent width (q_lora_rank)
 THETA = 1.0e4    # rope_theta
 
 
@@ -276,6 +277,22 @@ def make_out_proj(B=8, seed=0, device="cpu", o_std=0.035):
     o = _normal_bf16((B, H, DV), o_std, g, device)
     w_o = _normal_bf16((DIM, H * DV), 1.0 / math.sqrt(H * DV), g, device)
     return o, w_o
+
+
+def make_query_proj(B=8, T=4096, seed=0, device="cpu"):
+    """Inputs of the query path: x [B, 7168] ~ N(0,1), wq_a [1536, 7168] with
+    variance 1/7168, q_norm weight 1, wq_b [24576, 1536] with variance 1/1536
+    (so qr and q are ~N(0,1)), the rope table [T, 32, 2] and one query
+    position per row drawn uniformly from [0, T)."""
+    g = _gen(95_000 + seed, device)
+    x = _normal_bf16((B, DIM), 1.0, g, device)
+    wq_a = _normal_bf16((QL, DIM), 1.0 / math.sqrt(DIM), g, device)
+    q_norm_w = torch.ones(QL, dtype=torch.bfloat16, device=device)
+    wq_b = _normal_bf16((H * (DN + R), QL), 1.0 / math.sqrt(QL), g, device)
+    gi = torch.Generator()
+    gi.manual_seed(96_000 + seed)
+    pos = torch.randint(0, T, (B,), generator=gi, dtype=torch.int32).to(device)
+    return x, wq_a, q_norm_w, wq_b, rope_table(T).to(device), pos
 
 
 def make_rope_input(B=2, S=5, Hx=128, seed=0, device="cpu"):

@@ -21,6 +21,8 @@ from ._lib import (  # noqa: F401
     mla_index_mask,
     mla_out_proj,
     mla_out_proj_workspace_bytes,
+    mla_query_proj,
+    mla_query_proj_workspace_bytes,
     mla_rope,
     status_string,
 )

@@ -38,6 +38,9 @@ _SIGS = {
     "mla_fold_wuk": (_c_int, [_vp, _vp, _c_int, _vp, _vp]),
     "mla_out_proj_workspace_bytes": (_c_size, [_c_int]),
     "mla_out_proj": (_c_int, [_vp, _vp, _c_int, _vp, _vp, _c_size, _vp, _vp]),
+    "mla_query_proj_workspace_bytes": (_c_size, [_c_int]),
+    "mla_query_proj": (_c_int, [_vp, _vp, _vp, _c_float, _vp, _vp, _c_int, _vp, _c_int, _vp,
+                                _vp, _vp, _c_size, _vp, _vp]),
     "mla_index_mask": (_c_int, [_vp, _c_int, _c_int, _vp, _c_int, _vp, _vp, _vp]),
     "mla_gather_rows": (_c_int, [_vp, _c_i64, _c_int, _vp, _c_i64, _c_int, _c_int, _vp,
                                  _c_int, _c_int, _vp, _vp, _vp, _vp]),
@@ -162,6 +165,32 @@ def mla_out_proj(O: torch.Tensor, w_o: torch.Tensor, out: Optional[torch.Tensor]
                             _stream(O.device)),
            "mla_out_proj")
     return out
+
+
+def mla_query_proj_workspace_bytes(B: int) -> int:
+    return int(LIB.mla_query_proj_workspace_bytes(int(B)))
+
+
+def mla_query_proj(x: torch.Tensor, wq_a: torch.Tensor, q_norm_w: torch.Tensor, eps: float,
+                   wq_b: torch.Tensor, rope: torch.Tensor, pos: torch.Tensor,
+                   ws: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None):
+    """x bf16 [B, 7168] -> (q_nope bf16 [B, 128, 128], q_pe bf16 [B, 128, 64])
+    with the rotation at pos (int32 [B]) from the fp32 table rope [T, 32, 2]."""
+    _need(x, torch.bfloat16, "x")
+    _need(pos, torch.int32, "pos")
+    _need(rope, torch.float32, "rope")
+    B = x.shape[0]
+    q_nope = torch.empty(B, 128, 128, dtype=torch.bfloat16, device=x.device)
+    q_pe = torch.empty(B, 128, 64, dtype=torch.bfloat16, device=x.device)
+    if ws is None:
+        ws = torch.empty(mla_query_proj_workspace_bytes(B), dtype=torch.uint8, device=x.device)
+    _check(LIB.mla_query_proj(_p(x.contiguous()), _p(wq_a.contiguous()), _p(q_norm_w),
+                              float(eps), _p(wq_b.contiguous()), _p(rope.contiguous()),
+                              rope.shape[0], _p(pos.contiguous()), B, _p(q_nope), _p(q_pe),
+                              _p(ws), ws.numel(), _p(status) if status is not None else None,
+                              _stream(x.device)),
+           "mla_query_proj")
+    return q_nope, q_pe
 
 
 NOALLOC_MAX_ROWS = 64

@@ -1,58 +1,39 @@
-// Output projection of the attention block ("Mix and project" page: the
-// output projection wo, the only step that mixes heads; its parameter table
-// gives 16,384 x 7,168 = 117,440,512 weights):
+// Weight-streaming projections of the attention block, and the output
+// projection ("Mix and project" page: the output projection wo, the only step
+// that mixes heads; its parameter table gives 16,384 x 7,168 = 117,440,512
+// weights):
 //
 //   Delta[b, n] = sum_k x[b, k] W_O[n, k],   x = O[b] flattened head-major
 //
 // with O [B, 128, 128] bf16 (the decode output), W_O [7168, 16384] bf16 stored
-// [out, in], Delta [B, 7168] bf16.  The step reads 235 MB of weights for a
-// few MB of activations, so it is HBM-bound on W_O.
+// [out, in], Delta [B, 7168] bf16.  These projections read a large weight for
+// a few MB of activations, so they are HBM-bound on the weight.
 //
-//   oproj_kernel     swap-AB GEMM on tcgen05: D^T[n, b] with 128 rows of W_O
-//                    as M, the batch as N (up to 128 per block), K = 16384 in
-//                    chunks of 64 through a 4-stage TMA ring.  Persistent CTAs
-//                    take equal slices of the flattened (row tile, K chunk)
-//                    list, so every SM streams the same number of weight
-//                    bytes; a slice covers the end of one row tile and the
-//                    start of the next, each part ("segment") ending with an
-//                    fp32 partial in its slot of the workspace.
-//   oproj_finalize   sums the slots of each row tile in slot order (a fixed
+//   xwt_kernel       swap-AB GEMM on tcgen05: D^T[n, b] with 128 rows of W as
+//                    M, the batch as N (up to 128 per block), K in chunks of 64
+//                    through a 4-stage TMA ring.  Persistent CTAs take equal
+//                    slices of the flattened (row tile, K chunk) list, so every
+//                    SM streams the same number of weight bytes; a slice covers
+//                    the end of one row tile and the start of the next, each
+//                    part ("segment") ending with an fp32 partial in its slot
+//                    of the workspace (see xwt.h).
+//   xwt_finish_bf16  sums the slots of each row tile in slot order (a fixed
 //                    order: the result does not depend on timing) and rounds
 //                    to bf16.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
 #include "host_util.h"
+#include "xwt.h"
 
 namespace shla {
-namespace oproj {
+namespace xwt {
 
-constexpr int K_IN = 128 * 128;     // 16384 inputs: 128 heads x 128 value dims, head-major
-constexpr int N_OUT = 7168;         // model dimension
 constexpr int KC = 64;              // K per chunk: one 128-byte swizzle atom of bf16
-constexpr int NCHUNK = K_IN / KC;   // 256 chunks per row tile
-constexpr int MT = N_OUT / 128;     // 56 row tiles of W_O
 constexpr int NST = 4;              // ring depth
-constexpr int STAGE = 2 * 16384;    // A: 128 W_O rows x 64 k; B: up to 128 batch rows x 64 k
+constexpr int STAGE = 2 * 16384;    // A: 128 W rows x 64 k; B: up to 128 batch rows x 64 k
 constexpr int SMEM_BYTES = NST * STAGE + 1024;
 constexpr int NTHREADS = 192;       // warps 0-3 epilogue, warp 4 loads, warp 5 MMA + TMEM
-constexpr int kMaxSlots = 8;        // partial slots per row tile (a schedule bound)
-static_assert(K_IN % KC == 0 && N_OUT % 128 == 0, "tiling");
-
-// Slices of the flattened list of MT x NCHUNK units: CTA c owns units
-// [bnd(c), bnd(c+1)); row tile m covers units [m NCHUNK, (m+1) NCHUNK).
-struct Sched {
-  int tot;  // MT * NCHUNK
-  int nc;   // CTAs per batch block
-  __host__ __device__ int bnd(int c) const { return (int)((long long)c * tot / nc); }
-  // first / last CTA whose slice meets row tile m
-  __host__ __device__ int c_first(int m) const {
-    return (int)((((long long)m * NCHUNK + 1) * nc + tot - 1) / tot) - 1;
-  }
-  __host__ __device__ int c_last(int m) const {
-    return (int)((((long long)(m + 1) * NCHUNK) * nc + tot - 1) / tot) - 1;
-  }
-};
 
 // TMA tiled load of one box (no multicast) at (x, y), bytes counted on bar
 DEV void tma_load_tile(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
@@ -72,21 +53,20 @@ struct Bars {
   int abort;
 };
 
-}  // namespace oproj
+}  // namespace xwt
 
 // ---------------------------------------------------------------------------
-// D^T[n, b] = sum_k W_O[n, k] x[b, k] over this CTA's slice of (row tile,
+// D^T[n, b] = sum_k W[n, k] X[b, k] over this CTA's slice of (row tile,
 // K chunk) units, for batch rows [b0, b0 + 128).
-//   A = W_O rows (M = 128, K = 64 per chunk), K-major, 128-byte swizzle
-//   B = x rows   (N = 128 batch rows),         K-major, 128-byte swizzle
+//   A = W rows (M = 128, K = 64 per chunk), K-major, 128-byte swizzle
+//   B = X rows (N = 128 batch rows),         K-major, 128-byte swizzle
 // Rows of the B box beyond B hold stale data; only their own columns of D
 // are affected, and those are not stored.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(oproj::NTHREADS, 1)
-    oproj_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
-                 float* __restrict__ part, int B, int a_rows, oproj::Sched sch,
-                 int32_t* status) {
-  using namespace oproj;
+__global__ void __launch_bounds__(xwt::NTHREADS, 1)
+    xwt_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
+               float* __restrict__ part, int B, int a_rows, XwtSched sch, int32_t* status) {
+  using namespace xwt;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));  // swizzle atoms: 1 KB aligned
@@ -95,6 +75,7 @@ __global__ void __launch_bounds__(oproj::NTHREADS, 1)
   volatile int* abort = &bars.abort;
   const int c = blockIdx.x, b0 = blockIdx.y * 128;
   const int u0 = sch.bnd(c), u1 = sch.bnd(c + 1);
+  const int nch = sch.nch;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (warp == 5) {
@@ -126,7 +107,7 @@ __global__ void __launch_bounds__(oproj::NTHREADS, 1)
         const int i = u - u0, s = i % NST;
         if (!mbar_wait(&bars.empty[s], ((i / NST) & 1) ^ 1, abort, status)) break;
         mbar_arrive_expect_tx(&bars.full[s], 16384 + 128 * a_rows);
-        const int m = u / NCHUNK, ch = u - m * NCHUNK;
+        const int m = u / nch, ch = u - m * nch;
         const uint32_t st = sbase + s * STAGE;
         tma_load_tile(st, &map_w, ch * KC, m * 128, &bars.full[s]);
         tma_load_tile(st + 16384, &map_x, ch * KC, b0, &bars.full[s]);
@@ -146,8 +127,8 @@ __global__ void __launch_bounds__(oproj::NTHREADS, 1)
 #pragma unroll 1
       for (int u = u0; u < u1; ++u) {
         const int i = u - u0, s = i % NST;
-        const int ch = u % NCHUNK;
-        const bool first = u == u0 || ch == 0, last = u == u1 - 1 || ch == NCHUNK - 1;
+        const int ch = u % nch;
+        const bool first = u == u0 || ch == 0, last = u == u1 - 1 || ch == nch - 1;
         if (!mbar_wait(&bars.full[s], (i / NST) & 1, abort, status)) break;
         // a new segment overwrites the accumulator once the epilogue has read it
         if (first && seg > 0 && !mbar_wait(&bars.tmem_free, (seg - 1) & 1, abort, status)) break;
@@ -174,15 +155,15 @@ __global__ void __launch_bounds__(oproj::NTHREADS, 1)
   } else if (u1 > u0) {
     // ---------------- epilogue (warps 0-3: TMEM lane = row of the tile) ----------------
     // segment k of the slice is row tile m0 + k; its partial goes to slot
-    // c - c_first(m) as part[m][slot][b][row], 32 consecutive rows per store
-    const int m0 = u0 / NCHUNK, m1 = (u1 - 1) / NCHUNK;
+    // c - c_first(m), 32 consecutive rows per store
+    const int m0 = u0 / nch, m1 = (u1 - 1) / nch;
     const int nl = warp * 32 + lane;
 #pragma unroll 1
     for (int m = m0, seg = 0; m <= m1; ++m, ++seg) {
       if (!warp_wait(&bars.seg_done, seg & 1, abort, status)) break;
       tc_fence_after();
       const int slot = c - sch.c_first(m);
-      float* dst = part + (size_t)(m * kMaxSlots + slot) * B * 128 + nl;
+      float* dst = part + (size_t)(m * sch.slots + slot) * B * 128 + nl;
 #pragma unroll 1
       for (int col = 0; col < 128; col += 16) {
         uint32_t r[16];
@@ -207,22 +188,21 @@ __global__ void __launch_bounds__(oproj::NTHREADS, 1)
   }
 }
 
-// Delta[b, n0 .. n0+7] = bf16(sum over the slots of row tile n0 / 128, in
-// slot order).  grid (B, N_OUT / 1024), 128 threads of 8 outputs each.
-__global__ void __launch_bounds__(128) oproj_finalize(const float* __restrict__ part,
-                                                       oproj::Sched sch, int B,
-                                                       __nv_bfloat16* __restrict__ out) {
-  using namespace oproj;
+// Y[b, n0 .. n0+7] = bf16(sum over the slots of row tile n0 / 128, in slot
+// order).  grid (B, ceil(n_out / 1024)), 128 threads of 8 outputs each.
+__global__ void __launch_bounds__(128) xwt_finish_bf16(const float* __restrict__ part,
+                                                        XwtSched sch, int B, int n_out,
+                                                        __nv_bfloat16* __restrict__ out) {
   const int b = blockIdx.x;
   const int n0 = (blockIdx.y * 128 + threadIdx.x) * 8;
-  if (n0 >= N_OUT) return;
+  if (n0 >= n_out) return;
   const int m = n0 / 128, nl = n0 % 128;
   const int used = sch.c_last(m) - sch.c_first(m) + 1;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
   for (int s = 0; s < used; ++s) {
     const float4* src =
-        reinterpret_cast<const float4*>(part + ((size_t)(m * kMaxSlots + s) * B + b) * 128 + nl);
+        reinterpret_cast<const float4*>(part + ((size_t)(m * sch.slots + s) * B + b) * 128 + nl);
     const float4 v0 = src[0], v1 = src[1];
     acc[0] += v0.x;
     acc[1] += v0.y;
@@ -238,37 +218,37 @@ __global__ void __launch_bounds__(128) oproj_finalize(const float* __restrict__ 
   o.y = pack_bf16x2(acc[2], acc[3]);
   o.z = pack_bf16x2(acc[4], acc[5]);
   o.w = pack_bf16x2(acc[6], acc[7]);
-  *reinterpret_cast<uint4*>(out + (size_t)b * N_OUT + n0) = o;
+  *reinterpret_cast<uint4*>(out + (size_t)b * n_out + n0) = o;
 }
 
 // ---------------------------------------------------------------------------
 // host
 // ---------------------------------------------------------------------------
-typedef CUresult (*OprojEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+typedef CUresult (*XwtEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-static OprojEncodeFn oproj_encode() {
-  static OprojEncodeFn fn = nullptr;
+static XwtEncodeFn xwt_encode() {
+  static XwtEncodeFn fn = nullptr;
   if (!fn) {
     void* f = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<OprojEncodeFn>(f);
+      fn = reinterpret_cast<XwtEncodeFn>(f);
   }
   return fn;
 }
 
-// 2-D map over a row-major [rows][16384] bf16 matrix, boxes of 64 x box_rows
-static int oproj_map(CUtensorMap* map, const void* base, int rows, int box_rows) {
-  OprojEncodeFn fn = oproj_encode();
+// 2-D map over a row-major [rows][cols] bf16 matrix, boxes of 64 x box_rows
+static int xwt_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
+  XwtEncodeFn fn = xwt_encode();
   if (!fn) return MLA_ERR_CUDA;
-  const cuuint64_t dims[2] = {(cuuint64_t)oproj::K_IN, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)oproj::K_IN * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)oproj::KC, (cuuint32_t)box_rows};
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)xwt::KC, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -277,14 +257,40 @@ static int oproj_map(CUtensorMap* map, const void* base, int rows, int box_rows)
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
-// CTAs per batch block: one per SM, at most 384 so that a row tile meets at
-// most kMaxSlots slices (slices of >= 37 units against 256 units per tile)
-static oproj::Sched oproj_sched(int sms) {
-  oproj::Sched s;
-  s.tot = oproj::MT * oproj::NCHUNK;
-  s.nc = sms < 1 ? 1 : (sms > 384 ? 384 : sms);
+XwtSched xwt_plan(int n_out, int k_in) {
+  XwtSched s;
+  s.nch = k_in / xwt::KC;
+  s.tot = (n_out / 128) * s.nch;
+  s.nc = s.tot < kXwtCtas ? s.tot : kXwtCtas;
+  s.slots = 1;
+  for (int m = 0; m < n_out / 128; ++m) {
+    const int used = s.c_last(m) - s.c_first(m) + 1;
+    if (used > s.slots) s.slots = used;
+  }
   return s;
 }
+
+size_t xwt_part_bytes(const XwtSched& plan, int n_out, int B) {
+  return (size_t)(n_out / 128) * plan.slots * B * 128 * sizeof(float);
+}
+
+int xwt_gemm(const void* w, int n_out, int k_in, const void* x, int B, float* part,
+             const XwtSched& plan, int32_t* status, cudaStream_t st) {
+  const int rows = B < 128 ? B : 128;
+  alignas(64) CUtensorMap map_w, map_x;
+  if (int e = xwt_map(&map_w, w, n_out, k_in, 128)) return e;
+  if (int e = xwt_map(&map_x, x, B, k_in, rows)) return e;
+  static unsigned long long attr_done = 0;
+  if (int e = ensure_smem_attr(xwt_kernel, xwt::SMEM_BYTES, &attr_done)) return e;
+  xwt_kernel<<<dim3(plan.nc, (B + 127) / 128), xwt::NTHREADS, xwt::SMEM_BYTES, st>>>(
+      map_w, map_x, part, B, rows, plan, status);
+  return launch_status();
+}
+
+namespace oproj {
+constexpr int K_IN = 128 * 128;  // 16384 inputs: 128 heads x 128 value dims, head-major
+constexpr int N_OUT = 7168;      // model dimension
+}  // namespace oproj
 
 }  // namespace shla
 
@@ -292,7 +298,8 @@ using namespace shla;
 
 extern "C" size_t mla_out_proj_workspace_bytes(int B) {
   if (B < 1 || B > 65535) return 0;
-  return round_up((size_t)oproj::MT * oproj::kMaxSlots * B * 128 * sizeof(float), 256);
+  const XwtSched plan = xwt_plan(oproj::N_OUT, oproj::K_IN);
+  return round_up(xwt_part_bytes(plan, oproj::N_OUT, B), 256);
 }
 
 extern "C" int mla_out_proj(const mla_bf16_t* O, const mla_bf16_t* w_o, int B, mla_bf16_t* delta,
@@ -302,21 +309,12 @@ extern "C" int mla_out_proj(const mla_bf16_t* O, const mla_bf16_t* w_o, int B, m
   if (!aligned16(O) || !aligned16(w_o) || !aligned16(delta)) return MLA_ERR_ALIGN;
   if (!ws || !aligned256(ws) || ws_bytes < mla_out_proj_workspace_bytes(B))
     return MLA_ERR_WORKSPACE;
-  int sms = 0;
-  if (int e = check_device(&sms)) return e;
-  const oproj::Sched sch = oproj_sched(sms);
-  const int rows = B < 128 ? B : 128;
-  alignas(64) CUtensorMap map_w, map_x;
-  if (int e = oproj_map(&map_w, w_o, oproj::N_OUT, 128)) return e;
-  if (int e = oproj_map(&map_x, O, B, rows)) return e;
-  static unsigned long long attr_done = 0;
-  if (int e = ensure_smem_attr(oproj_kernel, oproj::SMEM_BYTES, &attr_done)) return e;
+  if (int e = check_device()) return e;
+  const XwtSched plan = xwt_plan(oproj::N_OUT, oproj::K_IN);
   cudaStream_t st = as_stream(stream);
   float* part = static_cast<float*>(ws);
-  oproj_kernel<<<dim3(sch.nc, (B + 127) / 128), oproj::NTHREADS, oproj::SMEM_BYTES, st>>>(
-      map_w, map_x, part, B, rows, sch, status);
-  if (int e = launch_status()) return e;
-  oproj_finalize<<<dim3(B, oproj::N_OUT / 1024), 128, 0, st>>>(
-      part, sch, B, reinterpret_cast<__nv_bfloat16*>(delta));
+  if (int e = xwt_gemm(w_o, oproj::N_OUT, oproj::K_IN, O, B, part, plan, status, st)) return e;
+  xwt_finish_bf16<<<dim3(B, (oproj::N_OUT + 1023) / 1024), 128, 0, st>>>(
+      part, plan, B, oproj::N_OUT, reinterpret_cast<__nv_bfloat16*>(delta));
   return launch_status();
 }

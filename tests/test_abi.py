@@ -78,6 +78,21 @@ def test_null_and_shape_checks_before_any_cuda_call(lib):
     assert lib.mla_out_proj(dummy, dummy, 4, dummy, dummy, 16, None, None) == -4
     assert lib.mla_out_proj(dummy, dummy, 4, dummy, vp(4096 + 16), 1 << 30, None, None) == -4
     assert L.mla_out_proj_workspace_bytes(0) == 0
+    # query path
+    args = lambda **kw: [kw.get(n, dummy) for n in ("x", "wa", "w")] + [kw.get("eps", 1e-6)] + \
+        [kw.get(n, dummy) for n in ("wb", "rope")] + [kw.get("T", 16), kw.get("pos", dummy),
+                                                      kw.get("B", 2), dummy, dummy,
+                                                      kw.get("ws", dummy), kw.get("wsb", 1 << 30),
+                                                      None, None]  # noqa: E731
+    assert lib.mla_query_proj(*args(x=None)) == -1
+    assert lib.mla_query_proj(*args(pos=None)) == -1
+    assert lib.mla_query_proj(*args(B=0)) == -2
+    assert lib.mla_query_proj(*args(T=0)) == -2
+    assert lib.mla_query_proj(*args(eps=-1.0)) == -2
+    assert lib.mla_query_proj(*args(wb=odd)) == -3
+    assert lib.mla_query_proj(*args(wsb=64)) == -4
+    assert L.mla_query_proj_workspace_bytes(0) == 0
+    assert L.mla_query_proj_workspace_bytes(8) >= 8 * 1536 * 2
     assert L.mla_out_proj_workspace_bytes(128) >= 56 * 4 * 128 * 128 * 4
 
 
