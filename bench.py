@@ -471,7 +471,7 @@ def run_ours(args):
         op_ms = reduce_max(op_ms / n_op, world, dev)
         op_bytes = 7168 * 16384 * 2 + B * 16384 * 2 + B * 7168 * 2
         next_rows["out_proj"] = {
-            "what": "Delta = flatten(O) W_O^T, W_O [7168, 16384] bf16 (oproj_kernel + finalize)",
+            "what": "Delta = flatten(O) W_O^T, W_O [7168, 16384] bf16 (xwt_kernel + xwt_finish_bf16)",
             "us": op_ms * 1e3, "bound": "hbm", "algorithmic_bytes": op_bytes,
             "achieved": op_bytes / (op_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": op_bytes / (op_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}

@@ -47,6 +47,19 @@ DEV void report_timeout(int32_t* status) {
 }
 
 // ---------------------------------------------------------------------------
+// programmatic dependent launch
+// ---------------------------------------------------------------------------
+
+// wait until the previous kernel on the stream has completed and its memory
+// operations are visible (returns at once for a launch without the
+// programmatic-serialisation attribute)
+DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// let the next kernel on the stream be scheduled once every block of this
+// one has signalled (the first signal of a block counts)
+DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // mbarriers
 // ---------------------------------------------------------------------------
 

@@ -48,4 +48,28 @@ inline int ensure_smem_attr(F* fn, int bytes, unsigned long long* done_mask) {
 
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// once every block of the previous kernel on the stream has executed
+// griddepcontrol.launch_dependents (or exited), so its set-up overlaps that
+// kernel's tail.  The kernel must execute griddepcontrol.wait before it reads
+// or writes anything the previous kernel writes or reads.  Used only where
+// the previous kernel is one of this library's, launched by the same call.
+template <typename... KArgs, typename... Args>
+inline int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...) == cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
+}
+
 }  // namespace shla

@@ -46,8 +46,8 @@ DEV void tma_load_tile(uint32_t dst, const CUtensorMap* map, int x, int y, uint6
 
 struct Bars {
   uint64_t full[NST], empty[NST];
-  uint64_t seg_done;   // a segment's products have completed (MMA commit)
-  uint64_t tmem_free;  // the epilogue has read the accumulator (128 threads)
+  uint64_t seg_done[2];   // segment k's products in accumulator k & 1 have completed
+  uint64_t tmem_free[2];  // the epilogue has read accumulator k & 1 (128 threads)
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(xwt::NTHREADS, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (warp == 5) {
-    tmem_alloc(&bars.tmem_base, 128);
+    tmem_alloc(&bars.tmem_base, 256);  // two 128-column accumulators
     tmem_relinquish();
   }
   if (tid == 0) {
@@ -87,8 +87,10 @@ __global__ void __launch_bounds__(xwt::NTHREADS, 1)
       mbar_init(&bars.full[s], 1);   // the loader's expect_tx arrival + bytes
       mbar_init(&bars.empty[s], 1);  // MMA commit
     }
-    mbar_init(&bars.seg_done, 1);
-    mbar_init(&bars.tmem_free, 128);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.seg_done[i], 1);
+      mbar_init(&bars.tmem_free[i], 128);
+    }
     mbar_init(&bars.drain, 1);
     bars.abort = 0;
     fence_mbarrier_init_cluster();
@@ -102,16 +104,37 @@ __global__ void __launch_bounds__(xwt::NTHREADS, 1)
     // ---------------- loads ----------------
     if (lane == 0) {
       int issued = 0;
+      int m = u0 / nch, ch = u0 - m * nch, s = 0, ph = 0;  // tile, chunk, stage, its phase
+      // The weight is not written by the kernel before this one on the
+      // stream: the first stages' weight boxes load before waiting for it.
+      const int npre = min(NST, u1 - u0);
+      for (int i = 0, mm = m, cc = ch; i < npre; ++i) {
+        mbar_arrive_expect_tx(&bars.full[i], 16384 + 128 * a_rows);
+        tma_load_tile(sbase + i * STAGE, &map_w, cc * KC, mm * 128, &bars.full[i]);
+        if (++cc == nch) {
+          cc = 0;
+          ++mm;
+        }
+      }
+      pdl_wait();  // X may be the previous kernel's output
 #pragma unroll 1
       for (int u = u0; u < u1; ++u) {
-        const int i = u - u0, s = i % NST;
-        if (!mbar_wait(&bars.empty[s], ((i / NST) & 1) ^ 1, abort, status)) break;
-        mbar_arrive_expect_tx(&bars.full[s], 16384 + 128 * a_rows);
-        const int m = u / nch, ch = u - m * nch;
         const uint32_t st = sbase + s * STAGE;
-        tma_load_tile(st, &map_w, ch * KC, m * 128, &bars.full[s]);
+        if (u - u0 >= npre) {
+          if (!mbar_wait(&bars.empty[s], ph ^ 1, abort, status)) break;
+          mbar_arrive_expect_tx(&bars.full[s], 16384 + 128 * a_rows);
+          tma_load_tile(st, &map_w, ch * KC, m * 128, &bars.full[s]);
+        }
         tma_load_tile(st + 16384, &map_x, ch * KC, b0, &bars.full[s]);
-        issued = i + 1;
+        issued = u - u0 + 1;
+        if (++ch == nch) {
+          ch = 0;
+          ++m;
+        }
+        if (++s == NST) {
+          s = 0;
+          ph ^= 1;
+        }
       }
       // on an abort, loads still in flight land before the CTA can leave
       for (int i = max(0, issued - NST); i < issued; ++i)
@@ -123,30 +146,38 @@ __global__ void __launch_bounds__(xwt::NTHREADS, 1)
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t hi = desc_hi(1024, kSwizzle128B);
-      int seg = 0;
+      int seg = 0, ch = u0 % nch, s = 0, ph = 0;  // segment, chunk, stage, its phase
 #pragma unroll 1
       for (int u = u0; u < u1; ++u) {
-        const int i = u - u0, s = i % NST;
-        const int ch = u % nch;
         const bool first = u == u0 || ch == 0, last = u == u1 - 1 || ch == nch - 1;
-        if (!mbar_wait(&bars.full[s], (i / NST) & 1, abort, status)) break;
-        // a new segment overwrites the accumulator once the epilogue has read it
-        if (first && seg > 0 && !mbar_wait(&bars.tmem_free, (seg - 1) & 1, abort, status)) break;
+        const int acc = seg & 1;
+        if (!mbar_wait(&bars.full[s], ph, abort, status)) break;
+        // segment seg reuses accumulator seg & 1 once the epilogue has read
+        // segment seg - 2 from it
+        if (first && seg >= 2 && !mbar_wait(&bars.tmem_free[acc], ((seg >> 1) - 1) & 1, abort, status))
+          break;
         tc_fence_after();
         const uint32_t la = desc_lo(sbase + s * STAGE, 16), lb = desc_lo(sbase + s * STAGE + 16384, 16);
+        const uint32_t d = tmem + acc * 128;
         if (first)
-          tc_mma_c<false>(tmem, desc_join(la, hi), desc_join(lb, hi), idesc);
+          tc_mma_c<false>(d, desc_join(la, hi), desc_join(lb, hi), idesc);
         else
-          tc_mma_c<true>(tmem, desc_join(la, hi), desc_join(lb, hi), idesc);
+          tc_mma_c<true>(d, desc_join(la, hi), desc_join(lb, hi), idesc);
 #pragma unroll
         for (int ks = 1; ks < KC / 16; ++ks)
-          tc_mma_c<true>(tmem, desc_join(la + ks * 2, hi), desc_join(lb + ks * 2, hi), idesc);
+          tc_mma_c<true>(d, desc_join(la + ks * 2, hi), desc_join(lb + ks * 2, hi), idesc);
         tc_commit(&bars.empty[s]);
         if (last) {
-          tc_commit(&bars.seg_done);
+          tc_commit(&bars.seg_done[acc]);
           ++seg;
         }
+        if (++ch == nch) ch = 0;
+        if (++s == NST) {
+          s = 0;
+          ph ^= 1;
+        }
       }
+      pdl_trigger();  // all products issued: the finishing kernel may be scheduled
       // everything issued so far has finished before TMEM is released
       tc_commit(&bars.drain);
       mbar_wait(&bars.drain, 0, nullptr, status);
@@ -160,14 +191,15 @@ __global__ void __launch_bounds__(xwt::NTHREADS, 1)
     const int nl = warp * 32 + lane;
 #pragma unroll 1
     for (int m = m0, seg = 0; m <= m1; ++m, ++seg) {
-      if (!warp_wait(&bars.seg_done, seg & 1, abort, status)) break;
+      const int acc = seg & 1;
+      if (!warp_wait(&bars.seg_done[acc], (seg >> 1) & 1, abort, status)) break;
       tc_fence_after();
       const int slot = c - sch.c_first(m);
       float* dst = part + (size_t)(m * sch.slots + slot) * B * 128 + nl;
 #pragma unroll 1
       for (int col = 0; col < 128; col += 16) {
         uint32_t r[16];
-        tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + col, r);
+        tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + acc * 128 + col, r);
         tc_wait_ld();
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -176,7 +208,7 @@ __global__ void __launch_bounds__(xwt::NTHREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&bars.tmem_free);
+      mbar_arrive(&bars.tmem_free[acc]);
     }
   }
 
@@ -184,7 +216,7 @@ __global__ void __launch_bounds__(xwt::NTHREADS, 1)
   __syncthreads();
   if (warp == 5) {
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, 256);
   }
 }
 
@@ -198,6 +230,7 @@ __global__ void __launch_bounds__(128) xwt_finish_bf16(const float* __restrict__
   if (n0 >= n_out) return;
   const int m = n0 / 128, nl = n0 % 128;
   const int used = sch.c_last(m) - sch.c_first(m) + 1;
+  pdl_wait();  // the partials of the GEMM before this kernel
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
   for (int s = 0; s < used; ++s) {
@@ -275,15 +308,19 @@ size_t xwt_part_bytes(const XwtSched& plan, int n_out, int B) {
 }
 
 int xwt_gemm(const void* w, int n_out, int k_in, const void* x, int B, float* part,
-             const XwtSched& plan, int32_t* status, cudaStream_t st) {
+             const XwtSched& plan, int32_t* status, cudaStream_t st, bool pdl) {
   const int rows = B < 128 ? B : 128;
   alignas(64) CUtensorMap map_w, map_x;
   if (int e = xwt_map(&map_w, w, n_out, k_in, 128)) return e;
   if (int e = xwt_map(&map_x, x, B, k_in, rows)) return e;
   static unsigned long long attr_done = 0;
   if (int e = ensure_smem_attr(xwt_kernel, xwt::SMEM_BYTES, &attr_done)) return e;
-  xwt_kernel<<<dim3(plan.nc, (B + 127) / 128), xwt::NTHREADS, xwt::SMEM_BYTES, st>>>(
-      map_w, map_x, part, B, rows, plan, status);
+  const dim3 grid(plan.nc, (B + 127) / 128);
+  if (pdl)
+    return launch_pdl(xwt_kernel, grid, dim3(xwt::NTHREADS), xwt::SMEM_BYTES, st, map_w, map_x,
+                      part, B, rows, plan, status);
+  xwt_kernel<<<grid, xwt::NTHREADS, xwt::SMEM_BYTES, st>>>(map_w, map_x, part, B, rows, plan,
+                                                            status);
   return launch_status();
 }
 
@@ -313,8 +350,8 @@ extern "C" int mla_out_proj(const mla_bf16_t* O, const mla_bf16_t* w_o, int B, m
   const XwtSched plan = xwt_plan(oproj::N_OUT, oproj::K_IN);
   cudaStream_t st = as_stream(stream);
   float* part = static_cast<float*>(ws);
-  if (int e = xwt_gemm(w_o, oproj::N_OUT, oproj::K_IN, O, B, part, plan, status, st)) return e;
-  xwt_finish_bf16<<<dim3(B, (oproj::N_OUT + 1023) / 1024), 128, 0, st>>>(
-      part, plan, B, oproj::N_OUT, reinterpret_cast<__nv_bfloat16*>(delta));
-  return launch_status();
+  if (int e = xwt_gemm(w_o, oproj::N_OUT, oproj::K_IN, O, B, part, plan, status, st, false))
+    return e;
+  return launch_pdl(xwt_finish_bf16, dim3(B, (oproj::N_OUT + 1023) / 1024), dim3(128), 0, st,
+                    part, plan, B, oproj::N_OUT, reinterpret_cast<__nv_bfloat16*>(delta));
 }

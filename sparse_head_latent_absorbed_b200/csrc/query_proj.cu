@@ -36,6 +36,8 @@ __global__ void __launch_bounds__(192) qa_finish(const float* __restrict__ part,
   const int b = blockIdx.x, t = threadIdx.x;
   const int n0 = t * 8, m = n0 / 128, nl = n0 % 128;
   const int used = sch.c_last(m) - sch.c_first(m) + 1;
+  pdl_trigger();  // the second GEMM may set up and prefetch its weight now
+  pdl_wait();     // the partials of the first GEMM
   float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
   for (int s = 0; s < used; ++s) {
@@ -91,6 +93,7 @@ __global__ void __launch_bounds__(128) qb_finish(const float* __restrict__ part,
   const int h = n0 / (DN + RR), e = n0 - h * (DN + RR);
   const int m = n0 / 128, nl = n0 % 128;
   const int used = sch.c_last(m) - sch.c_first(m) + 1;
+  pdl_wait();  // the partials of the second GEMM
   float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
   for (int s = 0; s < used; ++s) {
@@ -166,14 +169,16 @@ extern "C" int mla_query_proj(const mla_bf16_t* x, const mla_bf16_t* wq_a,
   __nv_bfloat16* qr =
       reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + qproj_part_bytes(B));
   const XwtSched pa = xwt_plan(qproj::QL, qproj::DIM);
-  if (int e = xwt_gemm(wq_a, qproj::QL, qproj::DIM, x, B, part, pa, status, st)) return e;
-  qa_finish<<<B, 192, 0, st>>>(part, pa, B, reinterpret_cast<const __nv_bfloat16*>(q_norm_w), eps,
-                               qr);
-  if (int e = launch_status()) return e;
+  // the three kernels after the first are launched with programmatic
+  // serialisation: each prepares while its predecessor drains
+  if (int e = xwt_gemm(wq_a, qproj::QL, qproj::DIM, x, B, part, pa, status, st, false)) return e;
+  if (int e = launch_pdl(qa_finish, dim3(B), dim3(192), 0, st, part, pa, B,
+                         reinterpret_cast<const __nv_bfloat16*>(q_norm_w), eps, qr))
+    return e;
   const XwtSched pb = xwt_plan(qproj::QW, qproj::QL);
-  if (int e = xwt_gemm(wq_b, qproj::QW, qproj::QL, qr, B, part, pb, status, st)) return e;
-  qb_finish<<<dim3(B, qproj::QW / 1024), 128, 0, st>>>(
-      part, pb, B, reinterpret_cast<const float2*>(rope), T, pos,
-      reinterpret_cast<__nv_bfloat16*>(q_nope), reinterpret_cast<__nv_bfloat16*>(q_pe), status);
-  return launch_status();
+  if (int e = xwt_gemm(wq_b, qproj::QW, qproj::QL, qr, B, part, pb, status, st, true)) return e;
+  return launch_pdl(qb_finish, dim3(B, qproj::QW / 1024), dim3(128), 0, st, part, pb, B,
+                    reinterpret_cast<const float2*>(rope), T, pos,
+                    reinterpret_cast<__nv_bfloat16*>(q_nope),
+                    reinterpret_cast<__nv_bfloat16*>(q_pe), status);
 }

@@ -43,8 +43,10 @@ XwtSched xwt_plan(int n_out, int k_in);
 // fp32 partial bytes for B rows under `plan`
 size_t xwt_part_bytes(const XwtSched& plan, int n_out, int B);
 
-// enqueue the partials of Y = X W^T; returns MLA_OK or an MLA_ERR_* code
+// enqueue the partials of Y = X W^T; returns MLA_OK or an MLA_ERR_* code.
+// pdl: launch with programmatic serialisation after a kernel of the same call
+// (the weight must not be written by that kernel; X and part may be).
 int xwt_gemm(const void* w, int n_out, int k_in, const void* x, int B, float* part,
-             const XwtSched& plan, int32_t* status, cudaStream_t st);
+             const XwtSched& plan, int32_t* status, cudaStream_t st, bool pdl);
 
 }  // namespace shla
