@@ -11,7 +11,7 @@
 //
 //   xwt_kernel       swap-AB GEMM on tcgen05: D^T[n, b] with 128 rows of W as
 //                    M, the batch as N (up to 128 per block), K in chunks of 64
-//                    through a 4-stage TMA ring.  Persistent CTAs take equal
+//                    through a 6-stage TMA ring.  Persistent CTAs take equal
 //                    slices of the flattened (row tile, K chunk) list, so every
 //                    SM streams the same number of weight bytes; a slice covers
 //                    the end of one row tile and the start of the next, each
@@ -30,7 +30,7 @@ namespace shla {
 namespace xwt {
 
 constexpr int KC = 64;              // K per chunk: one 128-byte swizzle atom of bf16
-constexpr int NST = 4;              // ring depth
+constexpr int NST = 6;              // ring depth: 96 KB of weight in flight per SM
 constexpr int STAGE = 2 * 16384;    // A: 128 W rows x 64 k; B: up to 128 batch rows x 64 k
 constexpr int SMEM_BYTES = NST * STAGE + 1024;
 constexpr int NTHREADS = 192;       // warps 0-3 epilogue, warp 4 loads, warp 5 MMA + TMEM

@@ -26,21 +26,30 @@ constexpr int NH = 128, DN = 128, RR = 64;
 constexpr int QW = NH * (DN + RR);        // 24576 outputs of wq_b
 }  // namespace qproj
 
-// qr[b, :] = bf16(RMSNorm(sum of the slots) * w): one block of 192 threads per
-// row, 8 consecutive outputs per thread
-__global__ void __launch_bounds__(192) qa_finish(const float* __restrict__ part, XwtSched sch,
-                                                  int B, const __nv_bfloat16* __restrict__ norm_w,
-                                                  float eps, __nv_bfloat16* __restrict__ qr) {
+// qr[b, :] = bf16(RMSNorm(sum of the slots) * w): one block per row.  Thread
+// (g, i) of 4 groups x 192 sums slots g, g + 4, g + 8, ... of outputs
+// 8i .. 8i + 7 (four times the loads in flight of one thread per output
+// octet); group 0 adds the other groups' sums in group order, so the result
+// does not depend on timing.
+constexpr int QA_GROUPS = 4;
+constexpr int QA_THREADS = 192 * QA_GROUPS;
+
+__global__ void __launch_bounds__(QA_THREADS) qa_finish(const float* __restrict__ part,
+                                                        XwtSched sch, int B,
+                                                        const __nv_bfloat16* __restrict__ norm_w,
+                                                        float eps, __nv_bfloat16* __restrict__ qr) {
   using namespace qproj;
+  __shared__ __align__(16) float gsum[QA_GROUPS - 1][QL];
   __shared__ float red[6];
   const int b = blockIdx.x, t = threadIdx.x;
-  const int n0 = t * 8, m = n0 / 128, nl = n0 % 128;
+  const int g = t / 192, i = t - g * 192;
+  const int n0 = i * 8, m = n0 / 128, nl = n0 % 128;
   const int used = sch.c_last(m) - sch.c_first(m) + 1;
   pdl_trigger();  // the second GEMM may set up and prefetch its weight now
   pdl_wait();     // the partials of the first GEMM
   float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-  for (int s = 0; s < used; ++s) {
+  for (int s = g; s < used; s += QA_GROUPS) {
     const float4* src =
         reinterpret_cast<const float4*>(part + ((size_t)(m * sch.slots + s) * B + b) * 128 + nl);
     const float4 a = src[0], c = src[1];
@@ -53,13 +62,35 @@ __global__ void __launch_bounds__(192) qa_finish(const float* __restrict__ part,
     v[6] += c.z;
     v[7] += c.w;
   }
-  float ss = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) ss += v[i] * v[i];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if ((t & 31) == 0) red[t >> 5] = ss;
+  if (g > 0) {
+    float4* dst = reinterpret_cast<float4*>(&gsum[g - 1][n0]);
+    dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+    dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
   __syncthreads();
+  if (g == 0) {  // warps 0-5
+#pragma unroll
+    for (int h = 0; h < QA_GROUPS - 1; ++h) {
+      const float4* src = reinterpret_cast<const float4*>(&gsum[h][n0]);
+      const float4 a = src[0], c = src[1];
+      v[0] += a.x;
+      v[1] += a.y;
+      v[2] += a.z;
+      v[3] += a.w;
+      v[4] += c.x;
+      v[5] += c.y;
+      v[6] += c.z;
+      v[7] += c.w;
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) ss += v[k] * v[k];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if ((t & 31) == 0) red[t >> 5] = ss;
+  }
+  __syncthreads();
+  if (g != 0) return;
   float tot = 0.f;
 #pragma unroll
   for (int w = 0; w < 6; ++w) tot += red[w];  // fixed order in every thread
@@ -69,9 +100,9 @@ __global__ void __launch_bounds__(192) qa_finish(const float* __restrict__ part,
   uint4 o;
   uint32_t* op = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 wf = __bfloat1622float2(wp[i]);
-    op[i] = pack_bf16x2(v[2 * i] * inv * wf.x, v[2 * i + 1] * inv * wf.y);
+  for (int k = 0; k < 4; ++k) {
+    const float2 wf = __bfloat1622float2(wp[k]);
+    op[k] = pack_bf16x2(v[2 * k] * inv * wf.x, v[2 * k + 1] * inv * wf.y);
   }
   *reinterpret_cast<uint4*>(qr + (size_t)b * QL + n0) = o;
 }
@@ -172,7 +203,7 @@ extern "C" int mla_query_proj(const mla_bf16_t* x, const mla_bf16_t* wq_a,
   // the three kernels after the first are launched with programmatic
   // serialisation: each prepares while its predecessor drains
   if (int e = xwt_gemm(wq_a, qproj::QL, qproj::DIM, x, B, part, pa, status, st, false)) return e;
-  if (int e = launch_pdl(qa_finish, dim3(B), dim3(192), 0, st, part, pa, B,
+  if (int e = launch_pdl(qa_finish, dim3(B), dim3(QA_THREADS), 0, st, part, pa, B,
                          reinterpret_cast<const __nv_bfloat16*>(q_norm_w), eps, qr))
     return e;
   const XwtSched pb = xwt_plan(qproj::QW, qproj::QL);
