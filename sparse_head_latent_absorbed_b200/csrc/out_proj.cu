@@ -10,8 +10,9 @@
 // a few MB of activations, so they are HBM-bound on the weight.
 //
 //   xwt_kernel       swap-AB GEMM on tcgen05: D^T[n, b] with 128 rows of W as
-//                    M, the batch as N (up to 128 per block), K in chunks of 64
-//                    through a 6-stage TMA ring.  Persistent CTAs take equal
+//                    M, the batch as N (up to 128 per block), K in chunks of 128
+//                    (two 64-wide swizzle atoms, so each W row is read 256
+//                    contiguous bytes at a time) through a 3-stage TMA ring.  Persistent CTAs take equal
 //                    slices of the flattened (row tile, K chunk) list, so every
 //                    SM streams the same number of weight bytes; a slice covers
 //                    the end of one row tile and the start of the next, each
@@ -29,9 +30,12 @@
 namespace shla {
 namespace xwt {
 
-constexpr int KC = 64;              // K per chunk: one 128-byte swizzle atom of bf16
-constexpr int NST = 6;              // ring depth: 96 KB of weight in flight per SM
-constexpr int STAGE = 2 * 16384;    // A: 128 W rows x 64 k; B: up to 128 batch rows x 64 k
+constexpr int KA = 64;              // K per 128-byte swizzle atom of bf16 (one TMA box)
+constexpr int AT = 2;               // atoms per stage: 256 contiguous bytes of each W row
+constexpr int KC = KA * AT;         // K per chunk (one ring stage)
+constexpr int NST = 3;              // ring depth: 96 KB of weight in flight per SM
+constexpr int ATOM = 16384;         // 128 rows x 128 bytes
+constexpr int STAGE = 2 * AT * ATOM;  // W atoms (128 W rows x KC), then X atoms (128 batch rows)
 constexpr int SMEM_BYTES = NST * STAGE + 1024;
 constexpr int NTHREADS = 192;       // warps 0-3 epilogue, warp 4 loads, warp 5 MMA + TMEM
 
@@ -109,8 +113,11 @@ __global__ void __launch_bounds__(xwt::NTHREADS, 1)
       // stream: the first stages' weight boxes load before waiting for it.
       const int npre = min(NST, u1 - u0);
       for (int i = 0, mm = m, cc = ch; i < npre; ++i) {
-        mbar_arrive_expect_tx(&bars.full[i], 16384 + 128 * a_rows);
-        tma_load_tile(sbase + i * STAGE, &map_w, cc * KC, mm * 128, &bars.full[i]);
+        mbar_arrive_expect_tx(&bars.full[i], AT * (ATOM + 128 * a_rows));
+#pragma unroll
+        for (int a = 0; a < AT; ++a)
+          tma_load_tile(sbase + i * STAGE + a * ATOM, &map_w, cc * KC + a * KA, mm * 128,
+                        &bars.full[i]);
         if (++cc == nch) {
           cc = 0;
           ++mm;
@@ -122,10 +129,14 @@ __global__ void __launch_bounds__(xwt::NTHREADS, 1)
         const uint32_t st = sbase + s * STAGE;
         if (u - u0 >= npre) {
           if (!mbar_wait(&bars.empty[s], ph ^ 1, abort, status)) break;
-          mbar_arrive_expect_tx(&bars.full[s], 16384 + 128 * a_rows);
-          tma_load_tile(st, &map_w, ch * KC, m * 128, &bars.full[s]);
+          mbar_arrive_expect_tx(&bars.full[s], AT * (ATOM + 128 * a_rows));
+#pragma unroll
+          for (int a = 0; a < AT; ++a)
+            tma_load_tile(st + a * ATOM, &map_w, ch * KC + a * KA, m * 128, &bars.full[s]);
         }
-        tma_load_tile(st + 16384, &map_x, ch * KC, b0, &bars.full[s]);
+#pragma unroll
+        for (int a = 0; a < AT; ++a)
+          tma_load_tile(st + (AT + a) * ATOM, &map_x, ch * KC + a * KA, b0, &bars.full[s]);
         issued = u - u0 + 1;
         if (++ch == nch) {
           ch = 0;
@@ -157,15 +168,18 @@ __global__ void __launch_bounds__(xwt::NTHREADS, 1)
         if (first && seg >= 2 && !mbar_wait(&bars.tmem_free[acc], ((seg >> 1) - 1) & 1, abort, status))
           break;
         tc_fence_after();
-        const uint32_t la = desc_lo(sbase + s * STAGE, 16), lb = desc_lo(sbase + s * STAGE + 16384, 16);
+        const uint32_t la = desc_lo(sbase + s * STAGE, 16);
+        const uint32_t lb = desc_lo(sbase + s * STAGE + AT * ATOM, 16);
         const uint32_t d = tmem + acc * 128;
         if (first)
           tc_mma_c<false>(d, desc_join(la, hi), desc_join(lb, hi), idesc);
         else
           tc_mma_c<true>(d, desc_join(la, hi), desc_join(lb, hi), idesc);
 #pragma unroll
-        for (int ks = 1; ks < KC / 16; ++ks)
-          tc_mma_c<true>(d, desc_join(la + ks * 2, hi), desc_join(lb + ks * 2, hi), idesc);
+        for (int ks = 1; ks < KC / 16; ++ks) {  // atom ks / 4 (1024 in units of 16 B), K16 step ks % 4
+          const uint32_t off = (ks >> 2) * (ATOM >> 4) + (ks & 3) * 2;
+          tc_mma_c<true>(d, desc_join(la + off, hi), desc_join(lb + off, hi), idesc);
+        }
         tc_commit(&bars.empty[s]);
         if (last) {
           tc_commit(&bars.seg_done[acc]);
@@ -281,7 +295,7 @@ static int xwt_map(CUtensorMap* map, const void* base, int rows, int cols, int b
   if (!fn) return MLA_ERR_CUDA;
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)xwt::KC, (cuuint32_t)box_rows};
+  const cuuint32_t box[2] = {(cuuint32_t)xwt::KA, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,

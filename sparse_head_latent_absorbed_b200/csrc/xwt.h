@@ -3,7 +3,7 @@
 // computed as fp32 partials of D^T = W X^T (xwt_gemm, in out_proj.cu), to be
 // summed and finished by a per-projection kernel.
 //
-// Work split: row tile m (128 rows of W) and K chunk j (64 columns) form unit
+// Work split: row tile m (128 rows of W) and K chunk j (128 columns) form unit
 // m * nch + j; persistent CTA c takes units [bnd(c), bnd(c+1)) for each block
 // of 128 batch rows.  The part of a row tile one CTA holds ends in an fp32
 // partial at part[((m * slots + (c - c_first(m))) * B + b) * 128 + row]; a
@@ -37,7 +37,7 @@ struct XwtSched {
 // the device
 constexpr int kXwtCtas = 148;
 
-// plan for a [n_out, k_in] weight (n_out % 128 == 0, k_in % 64 == 0)
+// plan for a [n_out, k_in] weight (n_out % 128 == 0, k_in % 128 == 0)
 XwtSched xwt_plan(int n_out, int k_in);
 
 // fp32 partial bytes for B rows under `plan`
