@@ -260,7 +260,7 @@ def run_reference(args):
     import mla_inputs as mi
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     wl = mi.make_config(args.config, device=dev,
-                        batch=slice(0, min(8, {0: 1, 1: 8, 2: 64, 3: 128, 4: 32}[args.config])))
+                        batch=slice(0, min(8, mi.CONFIG_SPECS[args.config]["B"])))
     rows = list(range(wl.B))
     for _ in range(args.warmup):
         oracle_sample_rate(wl, rows[:1])
@@ -305,6 +305,86 @@ def workload_config(cid: int, world: int):
 # our arm
 # ---------------------------------------------------------------------------
 
+def time_next_rows(B, dev, stream, flush_l2, n_op, world, peaks):
+    """Times the two rows after the decode on the attention block's path at
+    batch B: the output projection and the query path, each call after an L2
+    flush, CUDA events on the launching stream, max over ranks."""
+    import torch
+
+    import mla_inputs as mi
+    import sparse_head_latent_absorbed_b200 as shla
+
+    next_rows = {}
+    o_in, w_o = mi.make_out_proj(B=B, seed=1, device=dev)
+    d_out = torch.empty(B, 7168, dtype=torch.bfloat16, device=dev)
+    op_ws = torch.empty(shla.mla_out_proj_workspace_bytes(B), dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        shla.mla_out_proj(o_in, w_o, out=d_out, ws=op_ws)
+    torch.cuda.synchronize()
+    op_ms = 0.0
+    for _ in range(n_op):
+        flush_l2()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        shla.mla_out_proj(o_in, w_o, out=d_out, ws=op_ws)
+        b_.record(stream)
+        torch.cuda.synchronize()
+        op_ms += a.elapsed_time(b_)
+    op_ms = reduce_max(op_ms / n_op, world, dev)
+    op_bytes = 7168 * 16384 * 2 + B * 16384 * 2 + B * 7168 * 2
+    next_rows["out_proj"] = {
+        "what": "Delta = flatten(O) W_O^T, W_O [7168, 16384] bf16 (xwt_kernel + xwt_finish_bf16)",
+        "us": op_ms * 1e3, "bound": "hbm", "algorithmic_bytes": op_bytes,
+        "achieved": op_bytes / (op_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        "frac": op_bytes / (op_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    del w_o
+    qx, wq_a, qn_w, wq_b, qrope, qpos = mi.make_query_proj(B=B, seed=1, device=dev)
+    q_ws = torch.empty(shla.mla_query_proj_workspace_bytes(B), dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        shla.mla_query_proj(qx, wq_a, qn_w, 1e-6, wq_b, qrope, qpos, ws=q_ws)
+    torch.cuda.synchronize()
+    q_ms = 0.0
+    for _ in range(n_op):
+        flush_l2()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        shla.mla_query_proj(qx, wq_a, qn_w, 1e-6, wq_b, qrope, qpos, ws=q_ws)
+        b_.record(stream)
+        torch.cuda.synchronize()
+        q_ms += a.elapsed_time(b_)
+    q_ms = reduce_max(q_ms / n_op, world, dev)
+    q_bytes = (1536 * 7168 + 24576 * 1536) * 2 + B * 7168 * 2 + B * 128 * 192 * 2
+    next_rows["query_proj"] = {
+        "what": "x -> wq_a -> RMSNorm -> wq_b -> split -> RoPE (2 x xwt_kernel + finishes)",
+        "us": q_ms * 1e3, "bound": "hbm", "algorithmic_bytes": q_bytes,
+        "achieved": q_bytes / (q_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        "frac": q_bytes / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    del wq_a, wq_b
+    return next_rows
+
+
+def run_next_rows_only(args, dev, world, rank):
+    """Times only the next rows (output projection, query path) at the
+    workload's batch, with no decode cache on the device: the small case
+    under which those kernels are profiled.  Prints one JSON line."""
+    import torch
+
+    import mla_inputs as mi
+    B = mi.CONFIG_SPECS[args.config]["B"]
+    flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def flush_l2():
+        flush_w.zero_()
+        flush_r.max()
+    rows = time_next_rows(B, dev, torch.cuda.current_stream(), flush_l2,
+                          max(3, min(args.steps, 100)), world, load_peaks())
+    if rank == 0:
+        print(json.dumps({"next_rows": rows, "batch": B, "n_gpus": world,
+                          "l2": "flushed before each call"}), flush=True)
+    return 0
+
+
 def run_ours(args):
     import torch
 
@@ -322,6 +402,8 @@ def run_ours(args):
     import mla_inputs as mi
     import sparse_head_latent_absorbed_b200 as shla
 
+    if args.only_next_rows:
+        return run_next_rows_only(args, dev, world, rank)
     wl = mi.make_config(args.config, device=dev)
     B, k = wl.B, wl.k
     ws = torch.empty(shla.mla_decode_workspace_bytes(B, k), dtype=torch.uint8, device=dev)
@@ -449,55 +531,11 @@ def run_ours(args):
         e_ms += a.elapsed_time(b_)
     e_ms = reduce_max(e_ms / n_e2e, world, dev)
 
-    # ---- the next row on the path: the output projection Delta = flatten(O) W_O^T ----
+    # ---- the next rows on the path: output projection and query path ----
     next_rows = {}
     if not args.no_next_rows:
-        o_in, w_o = mi.make_out_proj(B=B, seed=1, device=dev)
-        d_out = torch.empty(B, 7168, dtype=torch.bfloat16, device=dev)
-        op_ws = torch.empty(shla.mla_out_proj_workspace_bytes(B), dtype=torch.uint8, device=dev)
-        for _ in range(3):
-            shla.mla_out_proj(o_in, w_o, out=d_out, ws=op_ws)
-        torch.cuda.synchronize()
-        op_ms = 0.0
-        n_op = max(3, min(args.steps, 100))
-        for _ in range(n_op):
-            flush_l2()
-            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            shla.mla_out_proj(o_in, w_o, out=d_out, ws=op_ws)
-            b_.record(stream)
-            torch.cuda.synchronize()
-            op_ms += a.elapsed_time(b_)
-        op_ms = reduce_max(op_ms / n_op, world, dev)
-        op_bytes = 7168 * 16384 * 2 + B * 16384 * 2 + B * 7168 * 2
-        next_rows["out_proj"] = {
-            "what": "Delta = flatten(O) W_O^T, W_O [7168, 16384] bf16 (xwt_kernel + xwt_finish_bf16)",
-            "us": op_ms * 1e3, "bound": "hbm", "algorithmic_bytes": op_bytes,
-            "achieved": op_bytes / (op_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": op_bytes / (op_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
-        del w_o
-        qx, wq_a, qn_w, wq_b, qrope, qpos = mi.make_query_proj(B=B, seed=1, device=dev)
-        q_ws = torch.empty(shla.mla_query_proj_workspace_bytes(B), dtype=torch.uint8, device=dev)
-        for _ in range(3):
-            shla.mla_query_proj(qx, wq_a, qn_w, 1e-6, wq_b, qrope, qpos, ws=q_ws)
-        torch.cuda.synchronize()
-        q_ms = 0.0
-        for _ in range(n_op):
-            flush_l2()
-            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            shla.mla_query_proj(qx, wq_a, qn_w, 1e-6, wq_b, qrope, qpos, ws=q_ws)
-            b_.record(stream)
-            torch.cuda.synchronize()
-            q_ms += a.elapsed_time(b_)
-        q_ms = reduce_max(q_ms / n_op, world, dev)
-        q_bytes = (1536 * 7168 + 24576 * 1536) * 2 + B * 7168 * 2 + B * 128 * 192 * 2
-        next_rows["query_proj"] = {
-            "what": "x -> wq_a -> RMSNorm -> wq_b -> split -> RoPE (2 x xwt_kernel + finishes)",
-            "us": q_ms * 1e3, "bound": "hbm", "algorithmic_bytes": q_bytes,
-            "achieved": q_bytes / (q_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": q_bytes / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
-        del wq_a, wq_b
+        next_rows = time_next_rows(B, dev, stream, flush_l2, max(3, min(args.steps, 100)), world,
+                                   peaks)
 
     units = B * k * HEADS
     value = world * units / (ms_per_step * 1e-3)
@@ -547,6 +585,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-next-rows", action="store_true",
                     help="skip the separate timing of the output projection and query path")
+    ap.add_argument("--only-next-rows", action="store_true",
+                    help="time only the output projection and query path (no decode cache "
+                         "on the device; prints their next_rows object)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -133,6 +133,16 @@ CONFIG_NAMES = {
 }
 
 
+# the five headline workloads: batch rows, cache rows per batch row, top-k
+CONFIG_SPECS = {
+    0: dict(B=1, T=1001, k=1001),
+    1: dict(B=8, T=4096, k=2048),
+    2: dict(B=64, T=32768, k=2048),
+    3: dict(B=128, T=131072, k=2048),
+    4: dict(B=32, T=65536, k=2048),
+}
+
+
 def make_config(cid: int, device="cpu", batch: Optional[slice] = None) -> Workload:
     """Build one of the five headline workloads.
 
@@ -141,14 +151,7 @@ def make_config(cid: int, device="cpu", batch: Optional[slice] = None) -> Worklo
     those of the full workload because every per-row draw is seeded by the
     row's own batch index.
     """
-    specs = {
-        0: dict(B=1, T=1001, k=1001),
-        1: dict(B=8, T=4096, k=2048),
-        2: dict(B=64, T=32768, k=2048),
-        3: dict(B=128, T=131072, k=2048),
-        4: dict(B=32, T=65536, k=2048),
-    }
-    s = specs[cid]
+    s = CONFIG_SPECS[cid]
     B, T, k = s["B"], s["T"], s["k"]
     rows = range(B) if batch is None else range(B)[batch]
     return _make_rows(cid, list(rows), B, T, k, device)
