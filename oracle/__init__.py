@@ -8,11 +8,15 @@ from .mla_oracle import (  # noqa: F401
     cache_write,
     decode_absorbed,
     decode_materialised,
+    decode_multi_query,
+    expand_keys_values,
     fold_wuk,
     index_mask,
     mix_latent,
     out_proj,
     parameter_counts,
+    prefill_mask,
+    prefill_materialised,
     query_proj,
     rmsnorm,
     rope,

@@ -25,6 +25,10 @@ Sources (page title, section):
     Delta_attn = flatten(O) W_O^T.
   * "Query rotary up-projection" (the MLA init and forward excerpts): the
     query path wq_a -> q_norm -> wq_b -> split -> RoPE.
+  * "Mix and project" (the MHA prefill branch of the forward excerpt): sparse
+    prefill with expanded per-head keys and values under the index mask plus
+    the causal mask; multi-query decode is the decode definition applied to
+    several query rows that share one cache row.
 
 Readings taken where the pages are silent:
   * index semantics follow the decode mask built by scatter of 0 into a -inf
@@ -192,6 +196,83 @@ def decode_materialised(q_nope, q_pe, wkv_b, c_kv, k_pe, topk, end_pos, scale):
         p = p / p.sum(-1, keepdims=True)
         out[b] = np.einsum("ht,thd->hd", p, v)
     return out
+
+
+# ---------------------------------------------------------------------------
+# sparse prefill ("Mix and project", the MHA prefill branch of the forward
+# excerpt) and multi-query decode
+# ---------------------------------------------------------------------------
+
+
+def prefill_mask(topk_b, S):
+    """The prefill branch's mask for one sequence of S tokens: the index mask
+    (-inf everywhere, 0 at each token's listed positions inside [0, S)) plus
+    the causal mask (-inf where the key position is after the token) -> [S, S]."""
+    index_mask = np.full((S, S), -np.inf)
+    for s_ in range(S):
+        for t in np.asarray(topk_b[s_]).tolist():
+            if 0 <= t < S:
+                index_mask[s_, t] = 0.0
+    return index_mask + np.triu(np.full((S, S), -np.inf), 1)
+
+
+def expand_keys_values(c, pe, wkv_b, Dn):
+    """Per-head keys and values of the prefill branch from latent rows c [S, C]
+    and rotary keys pe [S, Rr]: kv = wkv_b(c) split into k_nope (first Dn
+    rows of each head) and v (the rest); k = [k_nope ; pe broadcast to every
+    head] -> (k [S, H, Dn+Rr], v [S, H, Dv])."""
+    kv = np.einsum("tc,hjc->thj", c, wkv_b)                    # [S, H, Dn+Dv]
+    k_nope, v = kv[:, :, :Dn], kv[:, :, Dn:]
+    Hh = wkv_b.shape[0]
+    k = np.concatenate([k_nope, np.broadcast_to(pe[:, None, :], (c.shape[0], Hh, pe.shape[1]))],
+                       -1)
+    return k, v
+
+
+def prefill_materialised(q_nope, q_pe, wkv_b, c_kv, k_pe, topk, scale):
+    """Prefill of a prompt of S tokens per sequence, cached at positions
+    0 .. S-1, following the prefill branch step by step:
+
+      q      = [q_nope ; q_pe]                              per token and head
+      k, v   = expand_keys_values(c_KV, k_pe)               expanded per head
+      scores = q . k * scale                                [S, H, S]
+      O      = softmax_t(scores + prefill_mask) . v
+
+    q_nope [B,S,H,Dn], q_pe [B,S,H,Rr], wkv_b [H, Dn+Dv, C], c_kv [B,T,C],
+    k_pe [B,T,Rr] with T >= S, topk [B,S,k] int (-1 = padding) ->
+    O [B,S,H,Dv] float64.  A token whose masked row has no finite entry
+    gets O = 0 (the reading taken for an empty selection in decode)."""
+    q_nope = np.asarray(q_nope, dtype=np.float64)
+    q_pe = np.asarray(q_pe, dtype=np.float64)
+    wkv_b = np.asarray(wkv_b, dtype=np.float64)
+    B, S, Hh, Dn = q_nope.shape
+    Dv = wkv_b.shape[1] - Dn
+    out = np.zeros((B, S, Hh, Dv))
+    for b in range(B):
+        c = np.asarray(c_kv[b, :S], dtype=np.float64)          # [S, C]
+        pe = np.asarray(k_pe[b, :S], dtype=np.float64)         # [S, Rr]
+        k, v = expand_keys_values(c, pe, wkv_b, Dn)
+        q = np.concatenate([q_nope[b], q_pe[b]], -1)           # [S, H, Dn+Rr]
+        mask = prefill_mask(topk[b], S)
+        sc = np.einsum("shd,thd->sht", q, k) * scale + mask[:, None, :]
+        for s_ in range(S):
+            if not np.isfinite(mask[s_]).any():
+                continue
+            row = sc[s_]                                        # [H, S]
+            p = np.exp(row - row.max(-1, keepdims=True))
+            p = p / p.sum(-1, keepdims=True)
+            out[b, s_] = np.einsum("ht,thd->hd", p, v)
+    return out
+
+
+def decode_multi_query(q_nope, q_pe, wkv_b, c_kv, k_pe, topk, end_pos, scale, queries_per_row):
+    """Absorbed decode of B query rows over B / queries_per_row cache rows:
+    query row r is scored against cache row r // queries_per_row with its own
+    selection topk[r] and limit end_pos[r] -- the decode definition applied to
+    each query row."""
+    rows = np.arange(np.asarray(q_nope).shape[0]) // int(queries_per_row)
+    return decode_absorbed(q_nope, q_pe, wkv_b, np.asarray(c_kv)[rows], np.asarray(k_pe)[rows],
+                           topk, end_pos, scale)
 
 
 # ---------------------------------------------------------------------------

@@ -179,6 +179,61 @@ def _query_feature_major(x, wq_a, w, eps, wq_b, R_pos, n_heads, dn, interleaved=
     return q[..., :dn], om.rope(q[..., dn:], np.asarray(R_pos), interleaved)
 
 
+PREFILL_PINS = [
+    pins.test_prefill_equals_absorbed_decode_per_token,
+    pins.test_prefill_first_token_sees_only_itself,
+    pins.test_prefill_ignores_future_and_unlisted_positions,
+    pins.test_prefill_brute_force,
+]
+MULTI_QUERY_PINS = [pins.test_multi_query_matches_materialised_per_query]
+
+
+def _prefill_mask_no_causal(topk_b, S):
+    # index mask only: listed positions after the token stay visible
+    m = np.full((S, S), -np.inf)
+    for s_ in range(S):
+        for t in np.asarray(topk_b[s_]).tolist():
+            if 0 <= t < S:
+                m[s_, t] = 0.0
+    return m
+
+
+def _prefill_mask_strict(topk_b, S):
+    # causal mask that also hides the token's own position
+    m = _prefill_mask_no_causal(topk_b, S)
+    return m + np.triu(np.full((S, S), -np.inf), 0)
+
+
+def _prefill_mask_dense(topk_b, S):
+    # causal mask only: the index selection is ignored
+    return np.triu(np.full((S, S), -np.inf), 1)
+
+
+_orig_expand = om.expand_keys_values
+
+
+def _expand_values_from_key_rows(c, pe, wkv_b, Dn):
+    # values taken from the first rows of each head (the key rows)
+    k, v = _orig_expand(c, pe, wkv_b, Dn)
+    kv = np.einsum("tc,hjc->thj", c, wkv_b)
+    return k, kv[:, :, :v.shape[-1]]
+
+
+def _expand_without_rotary_key(c, pe, wkv_b, Dn):
+    # the shared rotary key left out of every head's key
+    k, v = _orig_expand(c, pe, wkv_b, Dn)
+    k = k.copy()
+    k[..., Dn:] = 0.0
+    return k, v
+
+
+def _multi_query_modulo_rows(q_nope, q_pe, wkv_b, c_kv, k_pe, topk, end_pos, scale, qpr):
+    # query row r read from cache row r % (cache rows) instead of r // qpr
+    rows = np.arange(np.asarray(q_nope).shape[0]) % np.asarray(c_kv).shape[0]
+    return om.decode_absorbed(q_nope, q_pe, wkv_b, np.asarray(c_kv)[rows], np.asarray(k_pe)[rows],
+                              topk, end_pos, scale)
+
+
 _orig_rope = om.rope
 
 MUTANTS = [
@@ -204,6 +259,12 @@ MUTANTS = [
     ("query_proj", _query_rope_first, QUERY_PINS),
     ("query_proj", _query_norm_first, QUERY_PINS),
     ("query_proj", _query_feature_major, QUERY_PINS),
+    ("prefill_mask", _prefill_mask_no_causal, PREFILL_PINS),
+    ("prefill_mask", _prefill_mask_strict, PREFILL_PINS),
+    ("prefill_mask", _prefill_mask_dense, PREFILL_PINS),
+    ("expand_keys_values", _expand_values_from_key_rows, PREFILL_PINS),
+    ("expand_keys_values", _expand_without_rotary_key, PREFILL_PINS),
+    ("decode_multi_query", _multi_query_modulo_rows, MULTI_QUERY_PINS),
 ]
 
 

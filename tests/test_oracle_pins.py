@@ -564,3 +564,121 @@ def test_inputs_are_seeded_and_shapes_match():
     assert tuple(w3.topk.shape) == (8, 2048)
     for b_ in range(8):
         assert len(set(w3.topk[b_].tolist())) == 2048
+
+
+# ---------------------------------------------------------------------------
+# sparse prefill ("Mix and project", MHA prefill branch) and multi-query decode
+# ---------------------------------------------------------------------------
+
+def _prefill_problem(seed, B=2, S=9, H=3, Dn=4, Dv=3, C=6, Rr=4, k=5, future=True):
+    """Hand-sized prefill: each token lists up to k positions; with `future`
+    some listed positions lie after the token (the causal mask removes them)."""
+    rng = np.random.default_rng(seed)
+    qn = rng.standard_normal((B, S, H, Dn))
+    qp = rng.standard_normal((B, S, H, Rr))
+    wkv = rng.standard_normal((H, Dn + Dv, C)) / math.sqrt(C)
+    c = rng.standard_normal((B, S + 2, C))
+    pe = rng.standard_normal((B, S + 2, Rr))
+    topk = np.full((B, S, k), -1, dtype=np.int64)
+    for b in range(B):
+        for s in range(S):
+            hi = S if future else s + 1
+            pick = rng.choice(hi, size=min(k, hi), replace=False)
+            topk[b, s, :len(pick)] = pick
+    return qn, qp, wkv, c, pe, topk, 0.4
+
+
+def test_prefill_equals_absorbed_decode_per_token():
+    """The expanded-key prefill equals the absorbed decode of each token on its
+    own ("Key heads": folding W_UK into the query gives the same scores), with
+    the token's causal limit s + 1 as end_pos: listed positions after the
+    token are excluded in both."""
+    qn, qp, wkv, c, pe, topk, scale = _prefill_problem(31)
+    got = orc.prefill_materialised(qn, qp, wkv, c, pe, topk, scale)
+    B, S = qn.shape[:2]
+    for b in range(B):
+        want = orc.decode_absorbed(qn[b], qp[b], wkv, np.repeat(c[b:b + 1], S, 0),
+                                   np.repeat(pe[b:b + 1], S, 0), topk[b], np.arange(1, S + 1),
+                                   scale)
+        assert np.abs(got[b] - want).max() <= 1e-12
+
+
+def test_prefill_first_token_sees_only_itself():
+    """Token 0 may attend only to position 0: with 0 listed its output is the
+    value of position 0, W_UV[h] c[0], for every head (softmax of one key)."""
+    qn, qp, wkv, c, pe, topk, scale = _prefill_problem(32)
+    topk[:, 0, 0] = 0
+    got = orc.prefill_materialised(qn, qp, wkv, c, pe, topk, scale)
+    Dn = qn.shape[-1]
+    for b in range(qn.shape[0]):
+        want = np.einsum("hdc,c->hd", wkv[:, Dn:, :], c[b, 0])
+        assert np.abs(got[b, 0] - want).max() <= 1e-12
+
+
+def test_prefill_ignores_future_and_unlisted_positions():
+    """Changing the cache rows of positions after a token, or of positions it
+    does not list, leaves that token's output unchanged; changing a listed
+    earlier position changes it."""
+    qn, qp, wkv, c, pe, topk, scale = _prefill_problem(33)
+    base = orc.prefill_materialised(qn, qp, wkv, c, pe, topk, scale)
+    S = qn.shape[1]
+    s = S // 2
+    listed = sorted(t for t in topk[0, s].tolist() if 0 <= t <= s)
+    others = [t for t in range(S) if t > s or t not in listed]
+    c2, pe2 = c.copy(), pe.copy()
+    c2[0, others] += 3.0
+    pe2[0, others] -= 2.0
+    moved = orc.prefill_materialised(qn, qp, wkv, c2, pe2, topk, scale)
+    assert np.abs(moved[0, s] - base[0, s]).max() <= 1e-12
+    assert listed, "the token lists an earlier position"
+    c3 = c.copy()
+    c3[0, listed[0]] += 1.0
+    changed = orc.prefill_materialised(qn, qp, wkv, c3, pe, topk, scale)
+    assert np.abs(changed[0, s] - base[0, s]).max() > 1e-6
+
+
+def test_prefill_brute_force():
+    """Scalar loops over tokens, heads, listed earlier positions and
+    features on a tiny case."""
+    qn, qp, wkv, c, pe, topk, scale = _prefill_problem(34, B=1, S=5, H=2, Dn=2, Dv=2, C=3,
+                                                        Rr=2, k=4)
+    got = orc.prefill_materialised(qn, qp, wkv, c, pe, topk, scale)
+    S, H, Dn, Dv, C, Rr = 5, 2, 2, 2, 3, 2
+    for s in range(S):
+        keys = sorted(set(t for t in topk[0, s].tolist() if 0 <= t <= s))
+        for h in range(H):
+            if not keys:
+                assert np.abs(got[0, s, h]).max() == 0.0
+                continue
+            sc = []
+            for t in keys:
+                acc = 0.0
+                for d in range(Dn):
+                    kd = sum(wkv[h, d, j] * c[0, t, j] for j in range(C))
+                    acc += qn[0, s, h, d] * kd
+                for r in range(Rr):
+                    acc += qp[0, s, h, r] * pe[0, t, r]
+                sc.append(acc * scale)
+            m = max(sc)
+            e = [math.exp(x - m) for x in sc]
+            z = sum(e)
+            for d in range(Dv):
+                want = 0.0
+                for t, w in zip(keys, e):
+                    want += (w / z) * sum(wkv[h, Dn + d, j] * c[0, t, j] for j in range(C))
+                assert abs(got[0, s, h, d] - want) <= 1e-12
+
+
+def test_multi_query_matches_materialised_per_query():
+    """Several query rows per cache row: each row equals the expanded-key path
+    run on its own cache row (the cache repeated per query), with its own
+    selection and limit."""
+    rng = np.random.default_rng(35)
+    qn, qp, wkv, c, pe, topk, end_pos, scale = _rand_problem(rng, B=6, T=30, k=11)
+    q = 3
+    got = orc.decode_multi_query(qn, qp, wkv, c[:2], pe[:2], topk, end_pos, scale, q)
+    want = orc.decode_materialised(qn, qp, wkv, np.repeat(c[:2], q, 0), np.repeat(pe[:2], q, 0),
+                                   topk, end_pos, scale)
+    assert np.abs(got - want).max() <= 1e-12
+    other = orc.decode_multi_query(qn, qp, wkv, c[2:4], pe[2:4], topk, end_pos, scale, q)
+    assert np.abs(other - got).max() > 1e-6  # the cache rows are used
