@@ -363,6 +363,68 @@ def time_next_rows(B, dev, stream, flush_l2, n_op, world, peaks):
     return next_rows
 
 
+def time_multi_query_rows(wl, dev, stream, flush_l2, n_op, world, peaks):
+    """Times the rows built on mla_decode_mq, each call after an L2 flush:
+    sparse prefill of one 4096-token prompt (top-k 2048, causal) and, when a
+    decode workload `wl` is given, multi-query decode of two new tokens per
+    sequence on its cache.  Work counts only listed positions inside each
+    query row's causal limit."""
+    import torch
+
+    import mla_inputs as mi
+    import sparse_head_latent_absorbed_b200 as shla
+
+    def timed(w):
+        ws = torch.empty(shla.mla_decode_workspace_bytes(w.B, w.k), dtype=torch.uint8,
+                         device=dev)
+        out = torch.empty(w.B, HEADS, 128, dtype=torch.bfloat16, device=dev)
+
+        def call():
+            shla.mla_decode_mq(w.q_nope, w.q_pe, w.wkv_b, w.cache, w.topk, w.end_pos, w.scale,
+                               w.queries_per_row, out=out, ws=ws)
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        ms = 0.0
+        for _ in range(n_op):
+            flush_l2()
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            call()
+            b_.record(stream)
+            torch.cuda.synchronize()
+            ms += a.elapsed_time(b_)
+        ms = reduce_max(ms / n_op, world, dev)
+        valid = int(((w.topk >= 0) & (w.topk < w.end_pos[:, None])).sum().item())
+        return ms, valid
+
+    rows = {}
+    pf = mi.make_prefill(B=1, S=4096, k=2048, seed=1, device=dev)
+    ms, valid = timed(pf)
+    flops = valid * 278_528 + pf.B * 33_554_432  # per listed key (128 heads) + fold and W_UV
+    rows["prefill"] = {
+        "what": "sparse prefill, 1 prompt x 4096 tokens, top-k 2048, causal (mla_decode_mq, "
+                "query row = token, absorbed form); the 4.7 MB prompt cache stays in L2",
+        "us": ms * 1e3, "head_keys_per_s": valid * HEADS / (ms * 1e-3),
+        "listed_keys": valid, "bound": "tensor", "algorithmic_flops": flops,
+        "achieved": flops / (ms * 1e-3) / 1e12, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+        "frac": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"]}
+    del pf
+    if wl is not None:
+        mq = mi.make_multi_query(B=wl.B, S=2, T=wl.T, k=wl.k, seed=1, device=dev,
+                                 cache=wl.cache, end_pos=wl.end_pos, wkv_b=wl.wkv_b)
+        ms, valid = timed(mq)
+        nbytes = valid * 1156 + mq.B * (32768 + 16384 + 32768) + 33_554_432
+        rows["multi_query_decode"] = {
+            "what": f"multi-query decode, {wl.B} sequences x 2 new tokens, top-k {wl.k}, on the "
+                    "decode workload's cache (mla_decode_mq)",
+            "us": ms * 1e3, "head_keys_per_s": valid * HEADS / (ms * 1e-3),
+            "listed_keys": valid, "bound": "hbm", "algorithmic_bytes": nbytes,
+            "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    return rows
+
+
 def run_next_rows_only(args, dev, world, rank):
     """Times only the next rows (output projection, query path) at the
     workload's batch, with no decode cache on the device: the small case
@@ -377,8 +439,11 @@ def run_next_rows_only(args, dev, world, rank):
     def flush_l2():
         flush_w.zero_()
         flush_r.max()
-    rows = time_next_rows(B, dev, torch.cuda.current_stream(), flush_l2,
-                          max(3, min(args.steps, 100)), world, load_peaks())
+    n_op = max(3, min(args.steps, 100))
+    peaks = load_peaks()
+    rows = time_next_rows(B, dev, torch.cuda.current_stream(), flush_l2, n_op, world, peaks)
+    rows.update(time_multi_query_rows(None, dev, torch.cuda.current_stream(), flush_l2, n_op,
+                                      world, peaks))
     if rank == 0:
         print(json.dumps({"next_rows": rows, "batch": B, "n_gpus": world,
                           "l2": "flushed before each call"}), flush=True)
@@ -534,8 +599,9 @@ def run_ours(args):
     # ---- the next rows on the path: output projection and query path ----
     next_rows = {}
     if not args.no_next_rows:
-        next_rows = time_next_rows(B, dev, stream, flush_l2, max(3, min(args.steps, 100)), world,
-                                   peaks)
+        n_op = max(3, min(args.steps, 100))
+        next_rows = time_next_rows(B, dev, stream, flush_l2, n_op, world, peaks)
+        next_rows.update(time_multi_query_rows(wl, dev, stream, flush_l2, n_op, world, peaks))
 
     units = B * k * HEADS
     value = world * units / (ms_per_step * 1e-3)

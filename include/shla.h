@@ -176,6 +176,41 @@ int mla_decode(const mla_bf16_t* q_nope, const mla_bf16_t* q_pe, const mla_bf16_
                mla_bf16_t* O, void* ws, size_t ws_bytes, int32_t* status, void* stream);
 
 /*
+ * Several query rows per cache batch row: query row r (0 <= r < B) reads
+ * cache batch row r / queries_per_row, with its own q_nope[r], q_pe[r],
+ * topk[r, :] and end_pos[r]; everything else is mla_decode's definition
+ * (mla_decode is the case queries_per_row = 1).  Two uses:
+ *
+ *   multi-query decode: S new tokens of one sequence scored in one step
+ *   (speculative or multi-token-prediction tokens); row b * S + s holds token
+ *   s of sequence b, end_pos[b * S + s] its causal limit.
+ *
+ *   sparse prefill ("Mix and project" page, the MHA prefill branch of the
+ *   forward excerpt, with the index mask added to the causal mask): a prompt
+ *   of S tokens of sequence b, cached at positions 0 .. S-1, gives rows
+ *   b * S + s with end_pos = s + 1.  The prefill branch expands per-head keys
+ *   k = [c_KV W_UK[h] ; k_pe] and values c_KV W_UV[h] and scores every prompt
+ *   position under the mask; folding W_UK into the query and W_UV after the
+ *   mix gives the same result in exact arithmetic ("Key heads" page), and
+ *   only the selected positions are read.  Entries past the causal limit are
+ *   excluded as the mask excludes them (and counted in status[1] like any
+ *   entry outside [0, end_pos)); pass -1 for them to keep the count clean.
+ *
+ *   q_nope, q_pe, topk, end_pos, O: B query rows, layouts as mla_decode
+ *   c_kv, k_pe, strides, T: B / queries_per_row cache batch rows
+ *   ws: mla_decode_workspace_bytes(B, k) bytes
+ * Requires queries_per_row >= 1 dividing B, and every cache row in use
+ * addressable as a 32-bit row index: (B / queries_per_row - 1) *
+ * (ckv_bstride / ckv_rstride) + T <= 2^31 - 1 (else MLA_ERR_SHAPE).
+ */
+int mla_decode_mq(const mla_bf16_t* q_nope, const mla_bf16_t* q_pe, const mla_bf16_t* wkv_b,
+                  const mla_bf16_t* c_kv, int64_t ckv_bstride, int ckv_rstride,
+                  const mla_bf16_t* k_pe, int64_t kpe_bstride, int kpe_rstride, int T,
+                  const int32_t* topk, int k, const int32_t* end_pos, int B, int queries_per_row,
+                  float scale, mla_bf16_t* O, void* ws, size_t ws_bytes, int32_t* status,
+                  void* stream);
+
+/*
  * The same call split into its three phases, for timing one of them alone:
  *   phase 1: fold of W_UK into the queries (writes q~ into ws)
  *   phase 2: gather + scores + softmax + latent mix (reads q~; writes the

@@ -298,6 +298,85 @@ def make_query_proj(B=8, T=4096, seed=0, device="cpu"):
     return x, wq_a, q_norm_w, wq_b, rope_table(T).to(device), pos
 
 
+def _causal_topk(limits, k, gen, recent=None):
+    """One selection row per query row with causal limit L: min(k, L) distinct
+    positions from [0, L), shuffled, padded with -1 to k.  With `recent`
+    set and L >= recent + k, half of them come from the last `recent`
+    positions and half from the earlier ones (the long-context decode mix)."""
+    out = torch.full((len(limits), k), -1, dtype=torch.int64)
+    for i, L in enumerate(limits):
+        L = int(L)
+        if L <= k:
+            sel = torch.randperm(L, generator=gen)
+        elif recent and L >= recent + k:
+            r = torch.randperm(recent, generator=gen)[:k // 2] + (L - recent)
+            o = torch.randperm(L - recent, generator=gen)[:k - k // 2]
+            sel = torch.cat([r, o])
+            sel = sel[torch.randperm(k, generator=gen)]
+        else:
+            sel = torch.randperm(L, generator=gen)[:k]
+        out[i, :len(sel)] = sel
+    return out
+
+
+def make_prefill(B=1, S=256, k=64, seed=0, device="cpu") -> Workload:
+    """Sparse prefill of B prompts of S tokens, cached at positions 0 .. S-1:
+    query row b * S + s is token s of prompt b, with causal limit s + 1 and
+    min(k, s + 1) distinct listed positions from [0, s] (an indexer lists
+    only visible positions), padded with -1.  Cache rows, q_nope and q_pe
+    ~ N(0,1), wkv_b variance 1/512, as in the decode workloads.  The returned
+    workload has B * S query rows and `queries_per_row` = S."""
+    g = _gen(70_000 + seed, device)
+    cache = _normal_bf16((B, S, KROW), 1.0, g, device)
+    q_nope = _normal_bf16((B * S, H, DN), 1.0, g, device)
+    q_pe = _normal_bf16((B * S, H, R), 1.0, g, device)
+    wkv_b = _normal_bf16((H, DN + DV, C), 1.0 / math.sqrt(C), g, device)
+    gi = torch.Generator()
+    gi.manual_seed(71_000 + seed)
+    limits = [s + 1 for _ in range(B) for s in range(S)]
+    topk = _causal_topk(limits, k, gi).to(torch.int32).to(device)
+    end_pos = torch.tensor(limits, dtype=torch.int32).to(device)
+    wl = Workload(name=f"sparse prefill B={B} S={S} top-k={k}", B=B * S, T=S, k=k, cache=cache,
+                  q_nope=q_nope, q_pe=q_pe, wkv_b=wkv_b, topk=topk, end_pos=end_pos,
+                  scale=softmax_scale(1.0))
+    wl.queries_per_row = S
+    return wl
+
+
+def make_multi_query(B=4, S=2, T=2048, k=256, seed=0, device="cpu", cache=None, end_pos=None,
+                     wkv_b=None) -> Workload:
+    """Multi-query decode: S new tokens per sequence (speculative or
+    multi-token-prediction tokens) whose rows are the last S cached
+    positions.  With e_b the sequence's cached length, token s sees
+    positions [0, e_b - (S - 1 - s)); its selection follows _causal_topk
+    (the recent/older mix when T > 8192).  `cache`, `end_pos` (e_b per
+    sequence) and `wkv_b` may be passed in to reuse a decode workload's;
+    otherwise they are drawn as in the decode workloads with e_b ~ U[T/2, T].
+    The returned workload has B * S query rows and `queries_per_row` = S."""
+    g = _gen(72_000 + seed, device)
+    if cache is None:
+        cache = _normal_bf16((B, T, KROW), 1.0, g, device)
+    if wkv_b is None:
+        wkv_b = _normal_bf16((H, DN + DV, C), 1.0 / math.sqrt(C), g, device)
+    gi = torch.Generator()
+    gi.manual_seed(73_000 + seed)
+    if end_pos is None:
+        e = torch.randint(T // 2, T + 1, (B,), generator=gi)
+    else:
+        e = end_pos.to("cpu").to(torch.int64)
+    q_nope = _normal_bf16((B * S, H, DN), 1.0, g, device)
+    q_pe = _normal_bf16((B * S, H, R), 1.0, g, device)
+    limits = [int(e[b]) - (S - 1 - s) for b in range(B) for s in range(S)]
+    topk = _causal_topk(limits, k, gi, recent=4096 if T > 8192 else None)
+    wl = Workload(name=f"multi-query decode B={B} S={S} T={T} top-k={k}", B=B * S, T=T, k=k,
+                  cache=cache, q_nope=q_nope, q_pe=q_pe, wkv_b=wkv_b,
+                  topk=topk.to(torch.int32).to(device),
+                  end_pos=torch.tensor(limits, dtype=torch.int32).to(device),
+                  scale=softmax_scale(1.0))
+    wl.queries_per_row = S
+    return wl
+
+
 def make_rope_input(B=2, S=5, Hx=128, seed=0, device="cpu"):
     g = _gen(80_000 + seed, device)
     return _normal_bf16((B, S, Hx, R), 1.0, g, device)

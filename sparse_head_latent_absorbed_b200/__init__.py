@@ -13,6 +13,7 @@ from ._lib import (  # noqa: F401
     mla_cache_write_noalloc,
     mla_cache_write_workspace_bytes,
     mla_decode,
+    mla_decode_mq,
     mla_decode_num_splits,
     mla_decode_phase,
     mla_decode_workspace_bytes,

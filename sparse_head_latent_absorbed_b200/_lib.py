@@ -32,6 +32,9 @@ _SIGS = {
     "mla_decode_num_splits": (_c_int, [_c_int, _c_int]),
     "mla_decode": (_c_int, [_vp, _vp, _vp, _vp, _c_i64, _c_int, _vp, _c_i64, _c_int, _c_int,
                             _vp, _c_int, _vp, _c_int, _c_float, _vp, _vp, _c_size, _vp, _vp]),
+    "mla_decode_mq": (_c_int, [_vp, _vp, _vp, _vp, _c_i64, _c_int, _vp, _c_i64, _c_int, _c_int,
+                               _vp, _c_int, _vp, _c_int, _c_int, _c_float, _vp, _vp, _c_size,
+                               _vp, _vp]),
     "mla_decode_phase": (_c_int, [_c_int, _vp, _vp, _vp, _vp, _c_i64, _c_int, _vp, _c_i64,
                                   _c_int, _c_int, _vp, _c_int, _vp, _c_int, _c_float, _vp, _vp,
                                   _c_size, _vp, _vp]),
@@ -247,6 +250,38 @@ def mla_decode(q_nope: torch.Tensor, q_pe: torch.Tensor, wkv_b: torch.Tensor,
                           krs, cache.shape[1], _p(topk.contiguous()), k, _p(end_pos), B,
                           float(scale), _p(out), _p(ws), ws.numel(), _p(status),
                           _stream(q_nope.device)), "mla_decode")
+    return out
+
+
+def mla_decode_mq(q_nope: torch.Tensor, q_pe: torch.Tensor, wkv_b: torch.Tensor,
+                  cache: torch.Tensor, topk: torch.Tensor, end_pos: torch.Tensor, scale: float,
+                  queries_per_row: int, out: Optional[torch.Tensor] = None,
+                  ws: Optional[torch.Tensor] = None,
+                  status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Sparse decode of several query rows per cache row (multi-query decode,
+    sparse prefill).  q_nope [B,128,128], q_pe [B,128,64], topk int32 [B,k],
+    end_pos int32 [B] for B query rows; cache [B / queries_per_row, T, 576];
+    query row r reads cache row r // queries_per_row -> O bf16 [B,128,128]."""
+    for t, n in ((q_nope, "q_nope"), (q_pe, "q_pe"), (wkv_b, "wkv_b")):
+        _need(t, torch.bfloat16, n)
+        if not t.is_contiguous():
+            raise MLAError(f"{n} must be contiguous")
+    _need(topk, torch.int32, "topk")
+    _need(end_pos, torch.int32, "end_pos")
+    B = q_nope.shape[0]
+    k = topk.shape[1]
+    if queries_per_row < 1 or B % queries_per_row or cache.shape[0] != B // queries_per_row:
+        raise MLAError("cache must hold B / queries_per_row batch rows")
+    c_kv, cbs, crs, k_pe, kbs, krs = _split_cache(cache)
+    if out is None:
+        out = torch.empty(B, 128, 128, dtype=torch.bfloat16, device=q_nope.device)
+    if ws is None:
+        ws = torch.empty(mla_decode_workspace_bytes(B, k), dtype=torch.uint8,
+                         device=q_nope.device)
+    _check(LIB.mla_decode_mq(_p(q_nope), _p(q_pe), _p(wkv_b), _p(c_kv), cbs, crs, _p(k_pe), kbs,
+                             krs, cache.shape[1], _p(topk.contiguous()), k, _p(end_pos), B,
+                             int(queries_per_row), float(scale), _p(out), _p(ws), ws.numel(),
+                             _p(status), _stream(q_nope.device)), "mla_decode_mq")
     return out
 
 

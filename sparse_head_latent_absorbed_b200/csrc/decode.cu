@@ -280,6 +280,7 @@ struct Params {
   const __nv_bfloat16* q_tilde;   // [B][128][512]
   const __nv_bfloat16* q_pe;      // [B][128][64]
   long long rows_per_b;           // row-index distance between batch rows in the cache maps
+  int q_per_row;                  // query rows per cache batch row (query row r reads row r / q_per_row)
   int T;
   const int32_t* topk;
   int k;
@@ -402,6 +403,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     const int gw = warp - GATHER_WARP0;
     const int ng = (16 - gw + NGATHER - 1) / NGATHER;  // groups of this warp
     int bad = 0, issued = 0;
+    int base_bb = -1;      // query row whose cache base is in `base`
+    long long base = 0;    // first TMA row of that query row's cache batch row
     TileCur cur = first_cur();
     SHLA_TRACE_DECL
 #pragma unroll 1
@@ -410,8 +413,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       const bool oka = key_valid(cur.ilo, cur.lim), okb = key_valid(cur.ihi, cur.lim);
       if (rank == 0 && gw == 0) bad += (!oka && cur.ilo != -1) + (!okb && cur.ihi != -1);
       // TMA rows: valid keys map to their cache row, others to row -1 (zero fill)
-      const int ra = oka ? (int)((long long)cur.bb * p.rows_per_b + cur.ilo) : -1;
-      const int rb = okb ? (int)((long long)cur.bb * p.rows_per_b + cur.ihi) : -1;
+      if (cur.bb != base_bb) {
+        base_bb = cur.bb;
+        base = (long long)(cur.bb / p.q_per_row) * p.rows_per_b;
+      }
+      const int ra = oka ? (int)(base + cur.ilo) : -1;
+      const int rb = okb ? (int)(base + cur.ihi) : -1;
       if (i + 1 < n) cur = advance(cur);
       SHLA_T(1);
       if (!warp_wait(&bars.empty[s], ((i / NST) & 1) ^ 1, abort, p.status)) break;
@@ -1265,17 +1272,22 @@ extern "C" int mla_fold_wuk(const mla_bf16_t* q_nope, const mla_bf16_t* wkv_b, i
                      reinterpret_cast<__nv_bfloat16*>(q_tilde), B, nullptr, as_stream(stream));
 }
 
+// B query rows; query row r reads cache batch row r / q_per_row
 static int decode_impl(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_pe,
                        const mla_bf16_t* wkv_b, const mla_bf16_t* c_kv, int64_t ckv_bstride,
                        int ckv_rstride, const mla_bf16_t* k_pe, int64_t kpe_bstride,
                        int kpe_rstride, int T, const int32_t* topk, int k,
-                       const int32_t* end_pos, int B, float scale, mla_bf16_t* O, void* ws,
-                       size_t ws_bytes, int32_t* status, void* stream) {
+                       const int32_t* end_pos, int B, int q_per_row, float scale, mla_bf16_t* O,
+                       void* ws, size_t ws_bytes, int32_t* status, void* stream) {
   if (phase < 0 || phase > 3) return MLA_ERR_SHAPE;
+  if (q_per_row < 1 || B % q_per_row != 0) return MLA_ERR_SHAPE;
   if (!q_nope || !q_pe || !wkv_b || !topk || !end_pos || !O) return MLA_ERR_NULL;
   if (int e = check_cache_args(c_kv, ckv_bstride, ckv_rstride, k_pe, kpe_bstride, kpe_rstride, T))
     return e;
   if (B < 1 || B > 65535 || k < 1 || k > 65536) return MLA_ERR_SHAPE;
+  // the gather's 32-bit TMA row coordinate covers every cache row in use
+  if ((long long)(B / q_per_row - 1) * (ckv_bstride / ckv_rstride) + T > 0x7fffffffLL)
+    return MLA_ERR_SHAPE;
   if (!aligned16(q_nope) || !aligned16(q_pe) || !aligned16(wkv_b) || !aligned16(O))
     return MLA_ERR_ALIGN;
   if (!ws || !aligned256(ws)) return MLA_ERR_WORKSPACE;
@@ -1302,6 +1314,7 @@ static int decode_impl(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_
   p.q_tilde = q_tilde;
   p.q_pe = reinterpret_cast<const __nv_bfloat16*>(q_pe);
   p.rows_per_b = ckv_bstride / ckv_rstride;
+  p.q_per_row = q_per_row;
   p.T = T;
   p.topk = topk;
   p.k = k;
@@ -1316,7 +1329,8 @@ static int decode_impl(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_
   p.status = status;
   if (phase == 0 || phase == 2) {
     alignas(64) CUtensorMap map_c, map_r;
-    const unsigned long long rows = (unsigned long long)(B - 1) * p.rows_per_b + T;
+    const unsigned long long rows =
+        (unsigned long long)(B / q_per_row - 1) * p.rows_per_b + T;  // cache batch rows in use
     if (int e = make_row_map(&map_c, c_kv, kC, rows, ckv_rstride, 64, CU_TENSOR_MAP_SWIZZLE_128B))
       return e;
     if (int e = make_row_map(&map_r, k_pe, kR, rows, kpe_rstride, 32, CU_TENSOR_MAP_SWIZZLE_64B))
@@ -1344,7 +1358,19 @@ extern "C" int mla_decode(const mla_bf16_t* q_nope, const mla_bf16_t* q_pe,
                           const int32_t* end_pos, int B, float scale, mla_bf16_t* O, void* ws,
                           size_t ws_bytes, int32_t* status, void* stream) {
   return decode_impl(0, q_nope, q_pe, wkv_b, c_kv, ckv_bstride, ckv_rstride, k_pe, kpe_bstride,
-                     kpe_rstride, T, topk, k, end_pos, B, scale, O, ws, ws_bytes, status, stream);
+                     kpe_rstride, T, topk, k, end_pos, B, 1, scale, O, ws, ws_bytes, status, stream);
+}
+
+extern "C" int mla_decode_mq(const mla_bf16_t* q_nope, const mla_bf16_t* q_pe,
+                             const mla_bf16_t* wkv_b, const mla_bf16_t* c_kv, int64_t ckv_bstride,
+                             int ckv_rstride, const mla_bf16_t* k_pe, int64_t kpe_bstride,
+                             int kpe_rstride, int T, const int32_t* topk, int k,
+                             const int32_t* end_pos, int B, int queries_per_row, float scale,
+                             mla_bf16_t* O, void* ws, size_t ws_bytes, int32_t* status,
+                             void* stream) {
+  return decode_impl(0, q_nope, q_pe, wkv_b, c_kv, ckv_bstride, ckv_rstride, k_pe, kpe_bstride,
+                     kpe_rstride, T, topk, k, end_pos, B, queries_per_row, scale, O, ws, ws_bytes,
+                     status, stream);
 }
 
 extern "C" int mla_decode_phase(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_pe,
@@ -1354,7 +1380,7 @@ extern "C" int mla_decode_phase(int phase, const mla_bf16_t* q_nope, const mla_b
                                 int k, const int32_t* end_pos, int B, float scale, mla_bf16_t* O,
                                 void* ws, size_t ws_bytes, int32_t* status, void* stream) {
   return decode_impl(phase, q_nope, q_pe, wkv_b, c_kv, ckv_bstride, ckv_rstride, k_pe,
-                     kpe_bstride, kpe_rstride, T, topk, k, end_pos, B, scale, O, ws, ws_bytes,
+                     kpe_bstride, kpe_rstride, T, topk, k, end_pos, B, 1, scale, O, ws, ws_bytes,
                      status, stream);
 }
 

@@ -26,7 +26,8 @@ def lib():
 
 def test_header_declares_the_boundary():
     names = _declared()
-    for must in ("mla_rope", "mla_cache_write", "mla_decode", "mla_decode_workspace_bytes",
+    for must in ("mla_rope", "mla_cache_write", "mla_decode", "mla_decode_mq",
+                 "mla_decode_workspace_bytes",
                  "mla_index_mask", "mla_gather_rows", "mla_status_string"):
         assert must in names
 
@@ -94,6 +95,14 @@ def test_null_and_shape_checks_before_any_cuda_call(lib):
     assert L.mla_query_proj_workspace_bytes(0) == 0
     assert L.mla_query_proj_workspace_bytes(8) >= 8 * 1536 * 2
     assert L.mla_out_proj_workspace_bytes(128) >= 56 * 4 * 128 * 128 * 4
+    # several query rows per cache row: queries_per_row must divide B, and the
+    # cache rows in use must be addressable with 32-bit row indices
+    mq = lambda B, q, bstride=0: lib.mla_decode_mq(  # noqa: E731
+        dummy, dummy, dummy, dummy, bstride, 576, dummy, bstride, 576, 10, dummy, 4, dummy, B, q,
+        1.0, dummy, dummy, 1 << 30, None, None)
+    assert mq(4, 0) == -2
+    assert mq(3, 2) == -2
+    assert mq(2, 1, 576 << 31) == -2
 
 
 def test_workspace_and_split_choice(lib):
