@@ -304,6 +304,19 @@ int mla_query_proj(const mla_bf16_t* x, const mla_bf16_t* wq_a, const mla_bf16_t
                    const int32_t* pos, int B, mla_bf16_t* q_nope, mla_bf16_t* q_pe, void* ws,
                    size_t ws_bytes, int32_t* status, void* stream);
 
+/*
+ * Test hook (host only, no device call): the work split of the
+ * weight-streaming GEMM behind mla_out_proj and mla_query_proj for a
+ * [n_out, k_in] weight.  Row tile m (128 weight rows) and K chunk j (128
+ * columns) form unit m * nch + j; CTA c of a batch block takes units
+ * [c * tot / nc, (c + 1) * tot / nc).  Writes plan[0..3] = tot, nc, nch,
+ * slots, and for every row tile m first_last[2m], first_last[2m + 1] = the
+ * first and last CTA holding a unit of tile m (the partial of CTA c for tile
+ * m goes to slot c - first); first_last may be NULL.  Requires
+ * n_out % 128 == 0 and k_in % 128 == 0, both positive (else MLA_ERR_SHAPE).
+ */
+int mla_xwt_plan(int n_out, int k_in, int32_t* plan, int32_t* first_last);
+
 #ifdef __cplusplus
 }
 #endif

@@ -44,6 +44,7 @@ _SIGS = {
     "mla_query_proj_workspace_bytes": (_c_size, [_c_int]),
     "mla_query_proj": (_c_int, [_vp, _vp, _vp, _c_float, _vp, _vp, _c_int, _vp, _c_int, _vp,
                                 _vp, _vp, _c_size, _vp, _vp]),
+    "mla_xwt_plan": (_c_int, [_c_int, _c_int, _vp, _vp]),
     "mla_index_mask": (_c_int, [_vp, _c_int, _c_int, _vp, _c_int, _vp, _vp, _vp]),
     "mla_gather_rows": (_c_int, [_vp, _c_i64, _c_int, _vp, _c_i64, _c_int, _c_int, _vp,
                                  _c_int, _c_int, _vp, _vp, _vp, _vp]),

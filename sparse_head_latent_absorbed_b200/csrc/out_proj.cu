@@ -347,6 +347,23 @@ constexpr int N_OUT = 7168;      // model dimension
 
 using namespace shla;
 
+extern "C" int mla_xwt_plan(int n_out, int k_in, int32_t* plan, int32_t* first_last) {
+  if (!plan) return MLA_ERR_NULL;
+  if (n_out < 128 || k_in < xwt::KC || n_out % 128 || k_in % xwt::KC) return MLA_ERR_SHAPE;
+  const XwtSched s = xwt_plan(n_out, k_in);
+  plan[0] = s.tot;
+  plan[1] = s.nc;
+  plan[2] = s.nch;
+  plan[3] = s.slots;
+  if (first_last) {
+    for (int m = 0; m < n_out / 128; ++m) {
+      first_last[2 * m] = s.c_first(m);
+      first_last[2 * m + 1] = s.c_last(m);
+    }
+  }
+  return MLA_OK;
+}
+
 extern "C" size_t mla_out_proj_workspace_bytes(int B) {
   if (B < 1 || B > 65535) return 0;
   const XwtSched plan = xwt_plan(oproj::N_OUT, oproj::K_IN);
