@@ -64,6 +64,7 @@ __global__ void __launch_bounds__(128) fold_kernel(const __nv_bfloat16* __restri
   __shared__ uint32_t tmem_base;
   const int ct = blockIdx.x, h = blockIdx.y, b0 = blockIdx.z * NB;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_trigger();  // the attend kernel may start its set-up and first gathers
 
   if (warp == 0) {
     tmem_alloc(&tmem_base, NCOLS);
@@ -334,6 +335,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
   const int n = t_end - t_begin;  // tiles of this cluster (>= 1)
   const int nt = p.sch.nt;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // the merge / W_UV kernels may be scheduled; they take an SM only once
+  // this kernel's CTA has left it (it holds the whole register file)
+  pdl_trigger();
   const uint32_t sbase = smem_u32(smem);
   const int bb0 = t_begin / nt, jt0 = t_begin - bb0 * nt;  // row / tile-in-row of tile 0
   auto lim_of = [&](int bb) { return min(ld_global_nc_s32_early(p.end_pos + bb), p.T); };
@@ -732,6 +736,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     TileCur c1 = n > 1 ? advance(c0) : c0;
     TileCur c2 = c1;
     int prev_bb = c0.bb;
+    pdl_wait();  // q~ is the fold kernel's output (the other roles read only inputs)
     load_q(c0.bb);
 
     // one key tile: `cur` holds this thread's scaled partial scores of tile i
@@ -902,7 +907,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
                                                        __nv_bfloat16* __restrict__ omerged) {
   const int b = blockIdx.x;
   const int used = sch.c_last(b) - sch.c_first(b) + 1;
+  pdl_trigger();
   if (used <= 1) return;
+  pdl_wait();  // partial outputs of the attend kernel
   const int h = blockIdx.y * 16 + (threadIdx.x >> 4);
   const int c0 = (threadIdx.x & 15) * 8;  // chunks c0, c0 + 128, c0 + 256, c0 + 384
   const float* lse_b = lse + (size_t)b * slots * kH + h;
@@ -980,6 +987,7 @@ __global__ void __launch_bounds__(128) uv_kernel(const __nv_bfloat16* __restrict
     mbar_init(&bar[1], 1);
     fence_mbarrier_init_cluster();
   }
+  pdl_wait();  // O~ of the attend or combine kernel
   auto load_chunk = [&](int kc) {
     const uint32_t sA = s0 + (kc & 1) * BUF, sB = sA + 32768;
     for (int q = tid; q < 128 * 16; q += 128) {
@@ -1169,22 +1177,24 @@ static int launch_fold(const __nv_bfloat16* q_nope, const __nv_bfloat16* wkv_b,
 
 template <int NB>
 static int launch_uv_nb(const __nv_bfloat16* wkv_b, const __nv_bfloat16* omerged, int B,
-                        __nv_bfloat16* O, int32_t* status, cudaStream_t st) {
+                        __nv_bfloat16* O, int32_t* status, cudaStream_t st, bool pdl) {
   const int smem = 2 * (32768 + NB * 256) + 1024;
   static unsigned long long attr_done = 0;
   if (int e = ensure_smem_attr(uv_kernel<NB>, smem, &attr_done)) return e;
   dim3 grid(kH, (B + NB - 1) / NB);
+  if (pdl) return launch_pdl(uv_kernel<NB>, grid, dim3(128), smem, st, wkv_b, omerged, B, O, status);
   uv_kernel<NB><<<grid, 128, smem, st>>>(wkv_b, omerged, B, O, status);
   return launch_status();
 }
 
+// pdl: launched right after a kernel of the same call (programmatic serialisation)
 static int launch_uv(const __nv_bfloat16* wkv_b, const __nv_bfloat16* omerged, int B,
-                     __nv_bfloat16* O, int32_t* status, cudaStream_t st) {
-  if (B <= 16) return launch_uv_nb<16>(wkv_b, omerged, B, O, status, st);
-  if (B <= 32) return launch_uv_nb<32>(wkv_b, omerged, B, O, status, st);
-  if (B <= 64) return launch_uv_nb<64>(wkv_b, omerged, B, O, status, st);
-  if (B <= 128) return launch_uv_nb<128>(wkv_b, omerged, B, O, status, st);
-  return launch_uv_nb<256>(wkv_b, omerged, B, O, status, st);
+                     __nv_bfloat16* O, int32_t* status, cudaStream_t st, bool pdl) {
+  if (B <= 16) return launch_uv_nb<16>(wkv_b, omerged, B, O, status, st, pdl);
+  if (B <= 32) return launch_uv_nb<32>(wkv_b, omerged, B, O, status, st, pdl);
+  if (B <= 64) return launch_uv_nb<64>(wkv_b, omerged, B, O, status, st, pdl);
+  if (B <= 128) return launch_uv_nb<128>(wkv_b, omerged, B, O, status, st, pdl);
+  return launch_uv_nb<256>(wkv_b, omerged, B, O, status, st, pdl);
 }
 
 // The number of clusters is capped so that no batch row meets more than
@@ -1337,16 +1347,31 @@ static int decode_impl(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_
       return e;
     static unsigned long long core_attr = 0;
     if (int e = ensure_smem_attr(core_kernel, core::SMEM_BYTES, &core_attr)) return e;
-    core_kernel<<<dim3(2 * sch.nc), core::NTHREADS, core::SMEM_BYTES, st>>>(p, map_c, map_r);
-    if (int e = launch_status()) return e;
+    // In the full call the fold precedes it: programmatic serialisation lets
+    // its set-up and first gathers (which read only the caller's inputs)
+    // overlap the fold's tail.  Launched alone it waits for the stream.
+    if (phase == 0) {
+      if (int e = launch_pdl(core_kernel, dim3(2 * sch.nc), dim3(core::NTHREADS),
+                             core::SMEM_BYTES, st, p, map_c, map_r))
+        return e;
+    } else {
+      core_kernel<<<dim3(2 * sch.nc), core::NTHREADS, core::SMEM_BYTES, st>>>(p, map_c, map_r);
+      if (int e = launch_status()) return e;
+    }
   }
   if (phase == 0 || phase == 3) {
     if (slots > 1) {
-      combine_kernel<<<dim3(B, kH / 16), 256, 0, st>>>(opart, lse, sch, slots, omerged);
-      if (int e = launch_status()) return e;
+      if (phase == 0) {
+        if (int e = launch_pdl(combine_kernel, dim3(B, kH / 16), dim3(256), 0, st, opart, lse,
+                               sch, slots, omerged))
+          return e;
+      } else {
+        combine_kernel<<<dim3(B, kH / 16), 256, 0, st>>>(opart, lse, sch, slots, omerged);
+        if (int e = launch_status()) return e;
+      }
     }
     return launch_uv(reinterpret_cast<const __nv_bfloat16*>(wkv_b), omerged, B,
-                     reinterpret_cast<__nv_bfloat16*>(O), status, st);
+                     reinterpret_cast<__nv_bfloat16*>(O), status, st, phase == 0 || slots > 1);
   }
   return MLA_OK;
 }
