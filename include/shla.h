@@ -167,6 +167,13 @@ int mla_cache_write_noalloc(const mla_bf16_t* x, const mla_bf16_t* w_kva,
  * Requires 1 <= B <= 65535 and 1 <= k <= 65536; scores, softmax and
  * accumulations are fp32; q~, the softmax weights and per-split partial
  * outputs are rounded to bf16 as tensor-core operands.
+ *
+ * The call enqueues three or four kernels on `stream`.  The first waits for
+ * the stream's earlier work as usual.  The later ones use programmatic
+ * dependent launch: each may start its set-up while its predecessor drains,
+ * and reads that predecessor's results only once it has finished.  For the
+ * caller nothing changes: work enqueued after the call starts when the call's
+ * last kernel has finished, and the inputs must not be modified before then.
  */
 size_t mla_decode_workspace_bytes(int B, int k);
 int mla_decode(const mla_bf16_t* q_nope, const mla_bf16_t* q_pe, const mla_bf16_t* wkv_b,

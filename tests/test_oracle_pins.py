@@ -682,3 +682,30 @@ def test_multi_query_matches_materialised_per_query():
     assert np.abs(got - want).max() <= 1e-12
     other = orc.decode_multi_query(qn, qp, wkv, c[2:4], pe[2:4], topk, end_pos, scale, q)
     assert np.abs(other - got).max() > 1e-6  # the cache rows are used
+
+
+def test_prefill_and_multi_query_inputs_are_causal_and_seeded():
+    """Each query row lists distinct positions inside its causal limit, as
+    many as the limit allows up to k, with -1 padding only after them; the
+    draws repeat under the same seed."""
+    pf = mi.make_prefill(B=2, S=70, k=40, seed=3)
+    again = mi.make_prefill(B=2, S=70, k=40, seed=3)
+    assert torch.equal(pf.topk, again.topk) and torch.equal(pf.q_nope, again.q_nope)
+    assert pf.queries_per_row == 70 and pf.B == 140 and tuple(pf.cache.shape) == (2, 70, 576)
+    for r in range(pf.B):
+        lim = int(pf.end_pos[r])
+        assert lim == r % 70 + 1
+        row = pf.topk[r].tolist()
+        n = min(40, lim)
+        assert all(0 <= t < lim for t in row[:n]) and len(set(row[:n])) == n
+        assert all(t == -1 for t in row[n:])
+    mq = mi.make_multi_query(B=3, S=2, T=9000, k=64, seed=4)
+    assert mq.queries_per_row == 2 and tuple(mq.cache.shape) == (3, 9000, 576)
+    for r in range(mq.B):
+        lim = int(mq.end_pos[r])
+        row = mq.topk[r].tolist()
+        assert all(0 <= t < lim for t in row) and len(set(row)) == 64
+        if r % 2 == 0:
+            assert lim == int(mq.end_pos[r + 1]) - 1  # token 0 sees one position less
+        recent = sum(t >= lim - 4096 for t in row)
+        assert recent >= 32  # half from the last 4096 positions (T > 8192)
