@@ -281,6 +281,9 @@ int mla_decode_num_splits(int B, int k);
  * on every run.  Requires 1 <= B <= 65535 and a caller-owned device
  * workspace of at least mla_out_proj_workspace_bytes(B) bytes, 256-byte
  * aligned (MLA_ERR_WORKSPACE otherwise).  status may be NULL (see above).
+ * Two kernels are enqueued; the second uses programmatic dependent launch
+ * (as described for mla_decode), with the same stream semantics for the
+ * caller.
  */
 size_t mla_out_proj_workspace_bytes(int B);
 int mla_out_proj(const mla_bf16_t* O, const mla_bf16_t* w_o, int B, mla_bf16_t* delta, void* ws,
@@ -303,7 +306,9 @@ int mla_out_proj(const mla_bf16_t* O, const mla_bf16_t* w_o, int B, mla_bf16_t* 
  * A row whose pos is outside [0, T) gets q_pe = 0 and is counted in
  * status[1].  Partials are summed in a fixed order (results identical on
  * every run).  Requires 1 <= B <= 65535 and a device workspace of at least
- * mla_query_proj_workspace_bytes(B) bytes, 256-byte aligned.
+ * mla_query_proj_workspace_bytes(B) bytes, 256-byte aligned.  Four kernels
+ * are enqueued; the last three use programmatic dependent launch (as
+ * described for mla_decode), with the same stream semantics for the caller.
  */
 size_t mla_query_proj_workspace_bytes(int B);
 int mla_query_proj(const mla_bf16_t* x, const mla_bf16_t* wq_a, const mla_bf16_t* q_norm_w,
