@@ -39,7 +39,7 @@ constexpr int STAGE = 2 * AT * ATOM;  // W atoms (128 W rows x KC), then X atoms
 constexpr int SMEM_BYTES = NST * STAGE + 1024;
 constexpr int NTHREADS = 192;       // warps 0-3 epilogue, warp 4 loads, warp 5 MMA + TMEM
 
-// TMA tiled load of one box (no multicast) at (x, y), bytes counted on bar
+// TMA tiled load of one box into this CTA's shared memory at (x, y), bytes counted on bar
 DEV void tma_load_tile(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
