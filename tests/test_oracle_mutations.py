@@ -184,8 +184,10 @@ PREFILL_PINS = [
     pins.test_prefill_first_token_sees_only_itself,
     pins.test_prefill_ignores_future_and_unlisted_positions,
     pins.test_prefill_brute_force,
+    pins.test_prefill_and_multi_query_degenerate_cases,
 ]
-MULTI_QUERY_PINS = [pins.test_multi_query_matches_materialised_per_query]
+MULTI_QUERY_PINS = [pins.test_multi_query_matches_materialised_per_query,
+                    pins.test_prefill_and_multi_query_degenerate_cases]
 
 
 def _prefill_mask_no_causal(topk_b, S):

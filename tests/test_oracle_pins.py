@@ -709,3 +709,25 @@ def test_prefill_and_multi_query_inputs_are_causal_and_seeded():
             assert lim == int(mq.end_pos[r + 1]) - 1  # token 0 sees one position less
         recent = sum(t >= lim - 4096 for t in row)
         assert recent >= 32  # half from the last 4096 positions (T > 8192)
+
+
+def test_prefill_and_multi_query_degenerate_cases():
+    """A one-token prompt is that token attending to itself (the value of
+    position 0); one query per cache row is plain decode; a prefill token
+    whose list holds only positions after it gets O = 0."""
+    qn, qp, wkv, c, pe, topk, scale = _prefill_problem(36, B=2, S=1, k=3)
+    topk[:] = -1
+    topk[:, 0, 0] = 0
+    got = orc.prefill_materialised(qn, qp, wkv, c, pe, topk, scale)
+    Dn = qn.shape[-1]
+    for b in range(2):
+        assert np.abs(got[b, 0] - np.einsum("hdc,c->hd", wkv[:, Dn:, :], c[b, 0])).max() <= 1e-12
+    rng = np.random.default_rng(37)
+    qn1, qp1, wkv1, c1, pe1, topk1, end1, scale1 = _rand_problem(rng, B=3, T=25, k=9)
+    a = orc.decode_multi_query(qn1, qp1, wkv1, c1, pe1, topk1, end1, scale1, 1)
+    b_ = orc.decode_materialised(qn1, qp1, wkv1, c1, pe1, topk1, end1, scale1)
+    assert np.abs(a - b_).max() <= 1e-12
+    qn, qp, wkv, c, pe, topk, scale = _prefill_problem(38, B=1, S=6, k=2)
+    topk[0, 2] = [4, 5]  # token 2 lists only later positions
+    got = orc.prefill_materialised(qn, qp, wkv, c, pe, topk, scale)
+    assert np.abs(got[0, 2]).max() == 0.0
