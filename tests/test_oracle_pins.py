@@ -731,3 +731,18 @@ def test_prefill_and_multi_query_degenerate_cases():
     topk[0, 2] = [4, 5]  # token 2 lists only later positions
     got = orc.prefill_materialised(qn, qp, wkv, c, pe, topk, scale)
     assert np.abs(got[0, 2]).max() == 0.0
+
+
+def test_workload_tensors_have_the_printed_sizes():
+    """The tensors the GPU tests and the bench feed the kernels have the
+    sizes the pages print: W_O 117,440,512 weights, the rotary rows of wq_b
+    12,582,912, wkv_b twice W_UK (8,388,608 each), 576 cached values per
+    position."""
+    gold = json.load(open(os.path.join(GOLD, "param_counts.json")))
+    _, w_o = mi.make_out_proj(B=1, seed=0)
+    assert w_o.numel() == gold["W_O"]["value"]
+    x, wq_a, qn_w, wq_b, tab, pos = mi.make_query_proj(B=1, T=8, seed=0)
+    assert wq_b.view(128, 192, 1536)[:, 128:, :].numel() == gold["W_QR"]["value"]
+    wl = mi.make_small(B=1, T=40, k=8, seed=0)
+    assert wl.wkv_b.numel() == 2 * gold["W_UK"]["value"]
+    assert wl.cache.shape[-1] == gold["cache_per_position"]["value"]
