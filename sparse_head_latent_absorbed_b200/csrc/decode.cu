@@ -5,35 +5,18 @@
 //   core_kernel      persistent 2-CTA clusters over equal ranges of the
 //                    (batch row, key tile) list: TMA gather of the selected
 //                    cache rows, S = Q~ K^T with the 128 heads as M, fp32
-//                    online softmax, O~ += P V.  CTA r of the pair owns latent
-//                    columns [256r, 256r+256) and rotary columns [32r, 32r+32);
-//                    the two partial score tiles are summed through
-//                    distributed shared memory.
+//                    online softmax, O~ += P V.  CTA r of the pair holds latent
+//                    columns [256r, 256r+256) and rotary columns [32r, 32r+32)
+//                    and runs the softmax of half of the heads; partial scores
+//                    and P cross between the two through distributed shared
+//                    memory.
 //   combine_kernel   log-sum-exp merge of the rows split across clusters
 //   uv_kernel        O = O~ W_UV^T per head on the merged O~ (tcgen05, value
 //                    dim as M, batch as N)
-#include <cuda_fp16.h>
 #include <math.h>
 
 #include "common.cuh"
 #include "host_util.h"
-
-// Optional per-role cycle accounting of the attend kernel (build with
-// -DSHLA_TRACE; the default build compiles the hooks away).  Each hook adds
-// the cycles since the previous hook to one bucket.
-#ifdef SHLA_TRACE
-namespace shla {
-__device__ unsigned long long g_trace[512][3][16];
-}
-#define SHLA_TRACE_DECL unsigned long long tr_[16] = {}; unsigned long long tp_ = clock64();
-#define SHLA_T(i) do { const unsigned long long n_ = clock64(); tr_[i] += n_ - tp_; tp_ = n_; } while (0)
-#define SHLA_TRACE_FLUSH(role) do { if (blockIdx.x < 512) for (int i_ = 0; i_ < 16; ++i_) \
-    atomicAdd(&shla::g_trace[blockIdx.x][role][i_], tr_[i_]); } while (0)
-#else
-#define SHLA_TRACE_DECL
-#define SHLA_T(i) do { } while (0)
-#define SHLA_TRACE_FLUSH(role) do { } while (0)
-#endif
 
 namespace shla {
 
@@ -155,112 +138,73 @@ __global__ void __launch_bounds__(128) fold_kernel(const __nv_bfloat16* __restri
 // normalised by its own sum, plus its log-sum-exp) that the combine kernel
 // merges.
 //
-// CTA r of the pair owns latent columns [256r, 256r+256) and rotary columns
-// [32r, 32r+32) of Q~ and of every selected cache row; both CTAs hold all 128
-// heads.  Per key tile (KT keys):
-//   S (partial)  = Q~_half K_half^T       M=128 heads, N=KT, K=288   (tcgen05)
-//   S            = S(own) + S(peer)      partials scaled to log2 units (invalid
-//                                        keys -inf), rounded to fp16 and
-//                                        exchanged through DSMEM; added, maxed
-//                                        and exponentiated as fp16 pairs
-//   P            = 2^(S - m)             running max m, lazily raised; row
-//                                        sum l on the CUDA cores
-//   O_half      += P V_half              M=128, N=256, K=KT          (tcgen05)
+// CTA r of the pair holds latent columns [256r, 256r+256) and rotary columns
+// [32r, 32r+32) of Q~ and of every selected cache row, for all 128 heads, and
+// runs the softmax of the 64 heads in TMEM lane quarters 2r and 2r+1.  Per key
+// tile (KT keys):
+//   S_r  = Q~_r K_r^T        partial scores, M=128 heads, N=KT, K=288 (tcgen05)
+//   the peer's heads' partial scores go to the peer in fp32 (st.async); the
+//   owner adds the two halves in fp32, scales to log2 units, sets invalid keys
+//   to -inf and runs the online softmax in fp32: running maximum m (raised
+//   lazily, once the tile maximum exceeds it by more than 8), P = 2^(s - m)
+//   rounded to bf16, row sum l of the fp32 P
+//   the owner's P rows go to both CTAs' shared memory, with (alpha, l, m) per
+//   row; alpha = 2^(m_old - m_new) rescales that row of O~ in both CTAs
+//   O_r += P V_r             M=128, N=256, K=KT, A = P from shared memory
 // V is the same shared-memory tile as K, read MN-major.
 //
-// Warp roles (512 threads; setmaxnreg gives the softmax warps 176 registers
-// and the others 80):
-//   warps 0-7   softmax: warp w covers head rows [32(w%4) + 16(w/4), +16)
-//               through 16x256b TMEM fragments, four threads per row.  They
-//               also load this CTA's half of Q~ at each segment start and
-//               write the segment outputs
-//   warps 8-14  gather: TMA tile::gather4 of the selected rows (4 rows per
-//               instruction); group g of four keys goes to warp 8 + g % 7
+// Warp roles (512 threads) in CTA r; q = warp % 4 is a warp's TMEM lane quarter:
+//   warps 0-3   quarter q owned (q / 2 == r): softmax of its 32 heads
+//               otherwise: sends its 32 heads' partial scores to the peer
+//               (all four load their rows of this CTA's half of Q~ at each
+//               segment start)
+//   warps 4-7   quarter q owned: gather; otherwise: receives the peer's
+//               (alpha, l, m) of its 32 heads, rescales and writes out their
+//               rows of this CTA's half of O~
+//   warps 8-13  gather: TMA tile::gather4 of the selected rows, two groups of
+//               four keys per gather warp and tile
+//   warp 14     L2 prefetch of the selected rows a few tiles ahead
 //   warp 15     TMEM owner and MMA issuer (one thread)
-// TMEM (512 columns): latent half of Q~ [0,128) as bf16 pairs, S [128,192),
-// two P buffers [192,256) as bf16 pairs, O half [256,512) fp32.  The rotary
-// half of Q sits in shared memory (64 B swizzle).
+// TMEM (512 columns): latent half of Q~ [0,128) as bf16 pairs, two score
+// tiles [128,256), O~ (latent half, fp32) [256,512).
 // ===========================================================================
-// packed fp16 pair helpers (low half = first element)
-DEV uint32_t f16x2_from_f32_sat(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-DEV uint32_t hadd2_u(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("add.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-DEV uint32_t hsub2_u(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("sub.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-DEV uint32_t hmax2_u(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("max.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-DEV uint32_t hex2_u(uint32_t a) {  // 2^x of both halves (special-function unit)
-  uint32_t r;
-  asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(a));
-  return r;
-}
-DEV float2 f16x2_to_f32x2(uint32_t h) {
-  float lo, hi;
-  asm("{.reg .f16 l, h; mov.b32 {l, h}, %2; cvt.f32.f16 %0, l; cvt.f32.f16 %1, h;}"
-      : "=f"(lo), "=f"(hi)
-      : "r"(h));
-  return make_float2(lo, hi);
-}
-DEV uint32_t bf16x2_from_f32(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-DEV uint32_t f16x2_splat(float v) {  // v exactly representable in fp16
-  const __half hv = __float2half_rn(v);
-  const uint16_t b = *reinterpret_cast<const uint16_t*>(&hv);
-  return (uint32_t)b | ((uint32_t)b << 16);
-}
+DEV uint32_t f2u(float x) { return __float_as_uint(x); }
+DEV float u2f(uint32_t x) { return __uint_as_float(x); }
 
 namespace core {
 constexpr int KT = 64;                       // keys per tile
 constexpr int NST = 4;                       // gather ring depth
-constexpr int NSOFT = 8;                     // softmax warps (two per TMEM lane quarter)
-constexpr int NGATHER = 7;                   // gather warps
-constexpr int GATHER_WARP0 = NSOFT;
-constexpr int MMA_WARP = NSOFT + NGATHER;
-constexpr int NTHREADS = 32 * (MMA_WARP + 1);  // 512
-// Register split (setmaxnreg; the launch gives 128 per thread): the eight
-// softmax warps take 176, the gather and MMA warps keep 80:
-// 8 x 32 x 176 + 8 x 32 x 80 = 65536.
-constexpr int REGS_SOFTMAX = 176, REGS_OTHER = 80;
-static_assert(NSOFT * 32 * REGS_SOFTMAX + (NTHREADS - 32 * NSOFT) * REGS_OTHER <= 65536,
-              "register split");
+constexpr int NGATHER = 8;                   // gather warps
+constexpr int PF_WARP = 14, MMA_WARP = 15;
+constexpr int NTHREADS = 512;
+constexpr int PF_AHEAD = 4;                  // prefetch distance, tiles ahead of the score products
 constexpr int ST_ATOM = KT * 128;            // one 64-column latent atom of a tile
 constexpr int ST_KR = 4 * ST_ATOM;           // rotary part of a tile (64 B swizzle)
 constexpr int ST_BYTES = ST_KR + KT * 64;    // 36864
 constexpr int OFF_ST = 0;
 constexpr int OFF_QR = OFF_ST + NST * ST_BYTES;  // rotary half of Q: 128 rows x 64 B, 64 B swizzle
-constexpr int OFF_XS = OFF_QR + 128 * 64;        // two buffers of exchanged partial scores
-constexpr int XS_BYTES = 128 * KT * 2;           // per softmax warp 4 chunks x 32 lanes x 16 B
-constexpr int OFF_BIAS = OFF_XS + 2 * XS_BYTES;  // per softmax warp: 0 / -inf per key of the tile
-constexpr int OFF_END = OFF_BIAS + NSOFT * KT * 4;
+constexpr int OFF_XS = OFF_QR + 128 * 64;        // received partial scores, two buffers
+constexpr int XS_BYTES = 2 * 16 * 32 * 16;       // [2 quarters][16 chunks][32 lanes][16 B]
+constexpr int OFF_P = OFF_XS + 2 * XS_BYTES;     // P of all 128 heads, two buffers
+constexpr int P_BYTES = 128 * 128;               // [128 rows][64 keys] bf16, 128 B swizzle, K-major
+constexpr int PA_BYTES = 128 * 16;               // per row: alpha, l, m (fp32)
+constexpr int PBUF = P_BYTES + PA_BYTES;
+constexpr int OFF_END = OFF_P + 2 * PBUF;
 constexpr int SMEM_BYTES = OFF_END + 1024;       // + alignment slack
-constexpr uint32_t XS_TX_BYTES = XS_BYTES;       // partial scores received per tile
+constexpr uint32_t XS_TX = XS_BYTES;             // partial scores received per tile
+constexpr uint32_t PP_TX = 64 * (128 + 16);      // P rows and (alpha, l, m) received per tile
 constexpr uint32_t GROUP_TX_BYTES = ST_BYTES / 16;  // bytes of one group of four keys
 constexpr uint32_t TMEM_COLS = 512;
-// TMEM: Q~ latent half (bf16 pairs), the score tile, two P tiles (bf16
-// pairs), O~ (latent half, fp32)
-constexpr uint32_t T_Q = 0, T_S = 128, T_P = 192, T_O = 256;
+constexpr uint32_t T_Q = 0, T_S = 128, T_O = 256;
+constexpr int REGS_WG0 = 152, REGS_REST = 120;
+static_assert(128 * (REGS_WG0 + 3 * REGS_REST) <= 65536, "register split");
 constexpr float kRescaleThreshold = 8.0f;        // log2 units
-static_assert(ST_BYTES % 1024 == 0 && OFF_QR % 1024 == 0 && OFF_XS % 16 == 0, "alignment");
+static_assert(ST_BYTES % 1024 == 0 && OFF_QR % 1024 == 0 && OFF_P % 1024 == 0 &&
+                  PBUF % 1024 == 0 && OFF_XS % 16 == 0,
+              "alignment");
 static_assert(SMEM_BYTES + 512 <= 232448, "shared memory budget");
-static_assert(T_Q + 128 <= T_S && T_S + KT <= T_P && T_P + KT <= T_O && T_O + 256 <= TMEM_COLS,
-              "TMEM plan");
-static_assert(KT / 4 == 16, "sixteen groups of four keys per tile");
+static_assert(T_Q + 128 <= T_S && T_S + 2 * KT <= T_O && T_O + 256 <= TMEM_COLS, "TMEM plan");
+static_assert(KT / 4 == 2 * NGATHER, "two groups of four keys per gather warp and tile");
 
 // Schedule: tiles [bnd(c), bnd(c+1)) of the flattened list belong to cluster c.
 struct Sched {
@@ -280,6 +224,9 @@ struct Sched {
 struct Params {
   const __nv_bfloat16* q_tilde;   // [B][128][512]
   const __nv_bfloat16* q_pe;      // [B][128][64]
+  const __nv_bfloat16* ckv;       // latent part of cache row 0 (prefetch addresses)
+  const __nv_bfloat16* kpe;       // rotary part of cache row 0
+  int ckv_rs, kpe_rs;             // row strides in elements
   long long rows_per_b;           // row-index distance between batch rows in the cache maps
   int q_per_row;                  // query rows per cache batch row (query row r reads row r / q_per_row)
   int T;
@@ -298,14 +245,19 @@ struct Params {
 
 struct Bars {
   uint64_t full[NST], empty[NST];  // gather ring
-  uint64_t s_full, s_empty;        // score tile in TMEM / read by all softmax threads
-  uint64_t p_full[2];              // P of tile t is in TMEM buffer t & 1 (all softmax threads)
-  uint64_t o_done[2];              // the value product of tile t has completed
+  uint64_t s_full[2], s_free[2];   // score tile t & 1 in TMEM / read by warps 0-3
+  uint64_t xs_full[2], xs_free[2]; // peer's partial scores landed / this CTA's buffer read by the peer
+  uint64_t p_own[2];               // this CTA's P rows of tile t & 1 written
+  uint64_t pp_full[2];             // the peer's P rows and (alpha, l, m) landed
+  uint64_t peer_ok[2];             // the peer's rows of O~ rescaled for tile t & 1
+  uint64_t o_done[2];              // this CTA's value product of tile t has completed
+  uint64_t pv_both[2];             // both CTAs' value products of tile t have completed
   uint64_t q_ready;                // the segment's Q~ is in TMEM / shared memory
-  uint64_t xs_full[2], xs_free[2]; // exchange buffers (peer's partial scores)
   uint64_t drain;
+  unsigned long long mask[NST];    // valid keys of the tile in each ring stage
   uint32_t tmem_base;
   int abort;
+  int prog;                        // score products issued (read by the prefetch warp)
 };
 
 DEV bool key_valid(int v, int lim) { return v >= 0 && v < lim; }
@@ -315,6 +267,10 @@ DEV bool key_valid(int v, int lim) { return v >= 0 && v < lim; }
 // valid-position limit and the tile's indices (lane l: keys l and 32 + l).
 struct TileCur {
   int bb, jt, lim, ilo, ihi;
+};
+// The same position without the indices.
+struct Pos {
+  int bb, jt;
 };
 
 }  // namespace core
@@ -369,6 +325,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     c.ilo = c.ihi = -1;
     return advance(c);
   };
+  auto next_pos = [&](Pos c) {
+    if (++c.jt == nt) {
+      c.jt = 0;
+      ++c.bb;
+    }
+    return c;
+  };
+
+  const int q4 = warp & 3;                    // TMEM lane quarter of warps 0-7
+  const bool owned = (q4 >> 1) == (int)rank;  // the quarter's heads are this CTA's
+  const int ql = q4 & 1;                      // index of the quarter within its CTA's pair
+  const bool is_gather = warp >= 8 ? warp < 8 + 6 : (warp >= 4 && owned);
+  const int gw = warp >= 8 ? warp - 8 : 6 + ql;  // gather warp index (0..7)
 
   if (warp == MMA_WARP) {
     tmem_alloc(&bars.tmem_base, TMEM_COLS);
@@ -380,42 +349,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       mbar_init(&bars.empty[s], 1);       // MMA commit after the tile's value product
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.p_full[i], 32 * NSOFT);
+      mbar_init(&bars.s_full[i], 1);
+      mbar_init(&bars.s_free[i], 4);
+      mbar_init(&bars.xs_full[i], 1);   // own expect_tx arrival + the peer's st.async bytes
+      mbar_init(&bars.xs_free[i], 2);   // one arrival per softmax warp of the peer
+      mbar_init(&bars.p_own[i], 2);
+      mbar_init(&bars.pp_full[i], 1);   // own expect_tx arrival + the peer's st.async bytes
+      mbar_init(&bars.peer_ok[i], 2);
       mbar_init(&bars.o_done[i], 1);
-      mbar_init(&bars.xs_full[i], 1);      // own expect_tx arrival + the peer's st.async bytes
-      mbar_init(&bars.xs_free[i], NSOFT);  // one arrival per softmax warp of the peer
+      mbar_init(&bars.pv_both[i], 2);   // this CTA's and the peer's value-product commits
     }
-    mbar_init(&bars.s_full, 1);
-    mbar_init(&bars.s_empty, 32 * NSOFT);
-    mbar_init(&bars.q_ready, 32 * NSOFT);
+    mbar_init(&bars.q_ready, 4);
     mbar_init(&bars.drain, 1);
     bars.abort = 0;
+    bars.prog = 0;
     fence_mbarrier_init_cluster();
-    mbar_arrive_expect_tx(&bars.xs_full[0], XS_TX_BYTES);
-    mbar_arrive_expect_tx(&bars.xs_full[1], XS_TX_BYTES);
+    for (int i = 0; i < 2 && i < n; ++i) {
+      mbar_arrive_expect_tx(&bars.xs_full[i], XS_TX);
+      mbar_arrive_expect_tx(&bars.pp_full[i], PP_TX);
+    }
   }
   tc_fence_before();
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
+  // Register split (the launch gives 128 per thread): warps 0-3 take
+  // REGS_WG0, every other warp REGS_REST; each role branch below starts with
+  // its warpgroup's setmaxnreg (warps 4-7 mix two roles with the same value).
+#define SHLA_REGS_DEC asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_REST))
+#define SHLA_REGS_INC asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_WG0))
 
-  if (warp >= GATHER_WARP0 && warp < MMA_WARP) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_OTHER));
+  if (is_gather) {
+    SHLA_REGS_DEC;
     // ---------------- gather (TMA tile::gather4) ----------------
-    // lane l holds the index of key l and key 32 + l of the tile; lanes
-    // 0..ng-1 each issue the five loads of one group of four keys
-    const int gw = warp - GATHER_WARP0;
-    const int ng = (16 - gw + NGATHER - 1) / NGATHER;  // groups of this warp
+    // lane l holds the index of key l and key 32 + l of the tile; lanes 0
+    // and 1 each issue the five loads of one group of four keys
     int bad = 0, issued = 0;
     int base_bb = -1;      // query row whose cache base is in `base`
     long long base = 0;    // first TMA row of that query row's cache batch row
     TileCur cur = first_cur();
-    SHLA_TRACE_DECL
 #pragma unroll 1
     for (int i = 0; i < n; ++i) {
       const int s = i % NST;
       const bool oka = key_valid(cur.ilo, cur.lim), okb = key_valid(cur.ihi, cur.lim);
       if (rank == 0 && gw == 0) bad += (!oka && cur.ilo != -1) + (!okb && cur.ihi != -1);
+      const uint32_t vlo = __ballot_sync(0xffffffffu, oka), vhi = __ballot_sync(0xffffffffu, okb);
       // TMA rows: valid keys map to their cache row, others to row -1 (zero fill)
       if (cur.bb != base_bb) {
         base_bb = cur.bb;
@@ -424,13 +402,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       const int ra = oka ? (int)(base + cur.ilo) : -1;
       const int rb = okb ? (int)(base + cur.ihi) : -1;
       if (i + 1 < n) cur = advance(cur);
-      SHLA_T(1);
       if (!warp_wait(&bars.empty[s], ((i / NST) & 1) ^ 1, abort, p.status)) break;
-      SHLA_T(0);
-      if (lane == 0) mbar_arrive_expect_tx(&bars.full[s], ng * GROUP_TX_BYTES);
+      if (lane == 0) {
+        if (gw == 0) bars.mask[s] = (unsigned long long)vlo | ((unsigned long long)vhi << 32);
+        mbar_arrive_expect_tx(&bars.full[s], 2 * GROUP_TX_BYTES);
+      }
       __syncwarp();
-      const int g = gw + NGATHER * (lane < ng ? lane : 0);  // this lane's group
-      const int k0 = 4 * g;                                 // its first key (0..60)
+      const int g = gw + NGATHER * (lane & 1);  // this lane's group (lanes 0 and 1 issue)
+      const int k0 = 4 * g;                     // its first key (0..60)
       const int src = k0 & 31;
       const int y0 = __shfl_sync(0xffffffffu, ra, src);
       const int y0b = __shfl_sync(0xffffffffu, rb, src);
@@ -440,7 +419,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       const int y2b = __shfl_sync(0xffffffffu, rb, src + 2);
       const int y3 = __shfl_sync(0xffffffffu, ra, src + 3);
       const int y3b = __shfl_sync(0xffffffffu, rb, src + 3);
-      if (lane < ng) {
+      if (lane < 2) {
         const bool hi = k0 >= 32;
         const int r0 = hi ? y0b : y0, r1 = hi ? y1b : y1, r2 = hi ? y2b : y2, r3 = hi ? y3b : y3;
         const uint32_t stage = sbase + OFF_ST + s * ST_BYTES;
@@ -451,70 +430,101 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
         tma_gather4(stage + ST_KR + k0 * 64, &map_r, rank * 32, r0, r1, r2, r3, &bars.full[s]);
       }
       issued = i + 1;
-      SHLA_T(2);
     }
     // on an abort, the loads still in flight land before the CTA can leave
     // (the waits are bounded and already complete on the normal path)
     for (int t = max(0, issued - NST); t < issued; ++t)
       warp_wait(&bars.full[t % NST], (t / NST) & 1, nullptr, nullptr);
-    if (lane == 0 && gw == 0) SHLA_TRACE_FLUSH(1);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);
     if (lane == 0 && bad && p.status) atomicAdd(p.status + 1, bad);
+  } else if (warp == PF_WARP) {
+    SHLA_REGS_DEC;
+    // ---------------- L2 prefetch of the rows PF_AHEAD tiles ahead ----------------
+    // lines of this CTA's part of each valid selected row (latent half and
+    // rotary half); they land in L2 before the gather asks for them
+    TileCur cur = first_cur();
+    const uint64_t t0 = globaltimer_ns();
+#pragma unroll 1
+    for (int i = 0; i < n; ++i) {
+      bool late = false;
+      while (*(volatile int*)&bars.prog < i - PF_AHEAD) {
+        if (*abort || globaltimer_ns() - t0 > kWaitLimitNs) {
+          late = true;
+          break;
+        }
+        __nanosleep(256);
+      }
+      if (late) break;
+      const long long base = (long long)(cur.bb / p.q_per_row) * p.rows_per_b;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int v = e ? cur.ihi : cur.ilo;
+        if (!key_valid(v, cur.lim)) continue;
+        const long long row = base + v;
+        const char* lat = reinterpret_cast<const char*>(p.ckv + row * p.ckv_rs + rank * 256);
+        const char* rot = reinterpret_cast<const char*>(p.kpe + row * p.kpe_rs + rank * 32);
+#pragma unroll
+        for (int l = 0; l < 4; ++l) prefetch_l2(lat + l * 128);
+        prefetch_l2(lat + 511);
+        prefetch_l2(rot);
+        prefetch_l2(rot + 63);
+      }
+      if (i + 1 < n) cur = advance(cur);
+    }
   } else if (warp == MMA_WARP) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_OTHER));
+    SHLA_REGS_DEC;
     // ---------------- MMA issuer ----------------
-    // Event loop.  A value product (A = P of tile t from TMEM buffer t & 1)
-    // goes first whenever its P is ready; a score product as soon as its keys
-    // have landed, the previous score tile has been read and this segment's
-    // Q~ is in place.
+    // Event loop.  A value product (A = P of tile t from shared memory
+    // buffer t & 1) goes first whenever both CTAs' P rows and rescales are
+    // in place; a score product as soon as its keys have landed, its score
+    // buffer has been read and this segment's Q~ is in place.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, KT, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, 0, 1);
-      // descriptors: a stage's low word plus a constant per K-step
-      constexpr uint32_t hi_k128 = desc_hi(1024, kSwizzle128B);  // K-major, 128 B swizzle
-      constexpr uint32_t hi_k64 = desc_hi(512, kSwizzle64B);     // K-major, 64 B swizzle
+      // descriptors: a buffer's low word plus a constant per K-step
+      constexpr uint32_t hi_k128 = desc_hi(1024, kSwizzle128B);  // 128 B swizzle, 8-row groups 1 KB apart
+      constexpr uint32_t hi_k64 = desc_hi(512, kSwizzle64B);     // 64 B swizzle
       const uint32_t lo_qr = desc_lo(sbase + OFF_QR, 16);        // rotary half of Q
       int qk = 0, pv = 0, idle = 0, qseg = -1;
       int qs = 0, qph = 0, ps = 0;  // stage of the next score product (and its phase), value product
       int jq = jt0, jp = jt0;  // tile-in-row of the next score / value product
-      bool alive = true;
       uint64_t t_idle = 0;  // when the current idle stretch was first checked (0: not yet)
-      SHLA_TRACE_DECL
 #pragma unroll 1
-      while (alive && pv < n) {
+      while (pv < n) {
         bool did = false;
-        if (pv < qk && mbar_test(&bars.p_full[pv & 1], (pv >> 1) & 1)) {
+        if (pv < qk && mbar_test(&bars.p_own[pv & 1], (pv >> 1) & 1) &&
+            mbar_test(&bars.peer_ok[pv & 1], (pv >> 1) & 1)) {
           tc_fence_after();
-          const int s = ps;
-          const uint32_t lo = desc_lo(sbase + OFF_ST + s * ST_BYTES, ST_ATOM);  // V, MN-major
-          const uint32_t tp = tmem + T_P + (pv & 1) * (KT / 2);
+          const int b = pv & 1;
+          const uint32_t lo_p = desc_lo(sbase + OFF_P + b * PBUF, 16);              // P, K-major
+          const uint32_t lo_v = desc_lo(sbase + OFF_ST + ps * ST_BYTES, ST_ATOM);  // V, MN-major
           const bool first = pv == 0 || jp == 0;
           if (first)
-            tc_mma_tmem_a_c<false>(tmem + T_O, tp, desc_join(lo, hi_k128), idesc_pv);
+            tc_mma_c<false>(tmem + T_O, desc_join(lo_p, hi_k128), desc_join(lo_v, hi_k128), idesc_pv);
           else
-            tc_mma_tmem_a_c<true>(tmem + T_O, tp, desc_join(lo, hi_k128), idesc_pv);
+            tc_mma_c<true>(tmem + T_O, desc_join(lo_p, hi_k128), desc_join(lo_v, hi_k128), idesc_pv);
 #pragma unroll
           for (int ks = 1; ks < KT / 16; ++ks)
-            tc_mma_tmem_a_c<true>(tmem + T_O, tp + ks * 8, desc_join(lo + ks * (2048 >> 4), hi_k128),
-                                  idesc_pv);
-          tc_commit(&bars.o_done[pv & 1]);
-          tc_commit(&bars.empty[s]);
+            tc_mma_c<true>(tmem + T_O, desc_join(lo_p + ks * 2, hi_k128),
+                           desc_join(lo_v + ks * (2048 >> 4), hi_k128), idesc_pv);
+          tc_commit(&bars.o_done[b]);
+          tc_commit(&bars.empty[ps]);
+          tc_commit_mc(&bars.pv_both[b], 3);
           ++pv;
           if (++ps == NST) ps = 0;
           if (++jp == nt) jp = 0;
           did = true;
-          SHLA_T(1);
         }
         if (qk < n && mbar_test(&bars.full[qs], qph) &&
-            (qk == 0 || mbar_test(&bars.s_empty, (qk - 1) & 1))) {
+            (qk < 2 || mbar_test(&bars.s_free[qk & 1], ((qk - 2) >> 1) & 1))) {
           const int seg = (qk == 0 || jq == 0) ? qseg + 1 : qseg;
           if (seg == qseg || mbar_test(&bars.q_ready, seg & 1)) {
             qseg = seg;
             tc_fence_after();
             const uint32_t st = sbase + OFF_ST + qs * ST_BYTES;
             const uint32_t lo = desc_lo(st, 16), lo_r = desc_lo(st + ST_KR, 16);
-            const uint32_t ts = tmem + T_S;
+            const uint32_t ts = tmem + T_S + (qk & 1) * KT;
             tc_mma_tmem_a_c<false>(ts, tmem + T_Q, desc_join(lo, hi_k128), idesc_qk);
 #pragma unroll
             for (int ks = 1; ks < 16; ++ks)
@@ -525,18 +535,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
             for (int ks = 0; ks < 2; ++ks)
               tc_mma_c<true>(ts, desc_join(lo_qr + ks * 2, hi_k64), desc_join(lo_r + ks * 2, hi_k64),
                              idesc_qk);
-            tc_commit(&bars.s_full);
+            tc_commit(&bars.s_full[qk & 1]);
             ++qk;
+            *(volatile int*)&bars.prog = qk;
             if (++qs == NST) {
               qs = 0;
               qph ^= 1;
             }
             if (++jq == nt) jq = 0;
             did = true;
-            SHLA_T(2);
           }
         }
-        SHLA_T(0);
         // the time limit runs from the first check of an idle stretch (the
         // timer is read only while nothing is ready)
         if (did) {
@@ -555,334 +564,290 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
           }
         }
       }
-      SHLA_TRACE_FLUSH(2);
       // everything issued so far has finished before TMEM is released
       tc_commit(&bars.drain);
       mbar_wait(&bars.drain, 0, nullptr, p.status);
+      // the peer's commits of its last value products land on this CTA's
+      // barriers before it leaves (bounded; complete on the normal path)
+      for (int t = max(0, pv - 2); t < pv; ++t)
+        mbar_wait(&bars.pv_both[t & 1], (t >> 1) & 1, nullptr, nullptr);
     }
     __syncwarp();
   } else {
-    // ---------------- softmax (four threads per head row) ----------------
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
-    // Warp w covers the 16 head rows [32q + 16s, +16) (q = w & 3 its TMEM
-    // lane quarter, s = w >> 2).  Through the 16x256b TMEM shape thread t
-    // holds rows r0 = t/4 and r0 + 8 of them and, of each 8-key block j, the
-    // keys 8j + 2c and 8j + 2c + 1 (c = t % 4): a row's 64 keys sit in four
-    // adjacent lanes, so its maxima and sums take two shuffles.  Score pair u
-    // of a thread is block u/2 of row r0 (u even) or of row r0 + 8 (u odd).
-    const int quarter = warp & 3, sub = warp >> 2;
-    const int c4 = lane & 3;
-    const int row0 = quarter * 32 + sub * 16 + (lane >> 2);  // second row: row0 + 8
-    const uint32_t frag_base = (uint32_t)(quarter * 32 + sub * 16) << 16;
-    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;  // 32x32b (Q~ load)
-    const int h = quarter * 32 + lane;  // this thread's row in 32x32b accesses
-    constexpr int NP = KT / 4;          // fp16 score pairs per thread per tile
-    // this CTA's half of Q~ for batch row bb: latent values [128 s, +128) of
-    // the CTA's 256 into TMEM as bf16 pairs (row h), rotary values [16 s, +16)
-    // of its 32 into the swizzled shared tile; then q_ready
+    // ---------------- TMEM warps: softmax / sender (0-3), receiver (4-7) ----------------
+    const int h = q4 * 32 + lane;                                // this thread's head row
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    const bool wg0 = warp < 4;
+    const uint32_t xs_off = ql * (XS_BYTES / 2) + lane * 16;    // + buffer + chunk * 512
+    const uint32_t p_peer = mapa_shared(sbase + OFF_P, peer);
+    const uint32_t pp_full_peer = mapa_shared(smem_u32(&bars.pp_full[0]), peer);
+    const uint32_t xs_full_peer = mapa_shared(smem_u32(&bars.xs_full[0]), peer);
+    const uint32_t xs_free_peer = mapa_shared(smem_u32(&bars.xs_free[0]), peer);
+    bool alive = true;
+
+    // this warp's 32 rows of this CTA's half of Q~ for batch row bb: latent
+    // values into TMEM as bf16 pairs, rotary values into the swizzled shared tile
     auto load_q = [&](int bb) {
-      const __nv_bfloat16* qrow = p.q_tilde + ((size_t)bb * kH + h) * kC + rank * 256 + sub * 128;
-      const __nv_bfloat16* rrow = p.q_pe + ((size_t)bb * kH + h) * kR + rank * 32 + sub * 16;
-      uint4 q[4][4], rq[2];
+      const __nv_bfloat16* qrow = p.q_tilde + ((size_t)bb * kH + h) * kC + rank * 256;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint4 v[8];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+        for (int i = 0; i < 8; ++i) v[i] = ld_global_nc_v4(qrow + c * 64 + i * 8);
+        uint32_t r[32];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) q[c][i] = ld_global_nc_v4(qrow + c * 32 + i * 8);
-      rq[0] = ld_global_nc_v4(rrow);
-      rq[1] = ld_global_nc_v4(rrow + 8);
+        for (int i = 0; i < 8; ++i) {
+          r[4 * i] = v[i].x;
+          r[4 * i + 1] = v[i].y;
+          r[4 * i + 2] = v[i].z;
+          r[4 * i + 3] = v[i].w;
+        }
+        tmem_st32(tmem + lane_base + T_Q + c * 32, r);
+      }
+      const __nv_bfloat16* rrow = p.q_pe + ((size_t)bb * kH + h) * kR + rank * 32;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t r[16];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          r[4 * i] = q[c][i].x;
-          r[4 * i + 1] = q[c][i].y;
-          r[4 * i + 2] = q[c][i].z;
-          r[4 * i + 3] = q[c][i].w;
-        }
-        tmem_st16(tmem + lane_base + T_Q + sub * 64 + c * 16, r);
+        const uint4 v = ld_global_nc_v4(rrow + c * 8);
+        st_shared_v4(sbase + OFF_QR + sw64_off(h, c), v.x, v.y, v.z, v.w);
       }
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-        st_shared_v4(sbase + OFF_QR + sw64_off(h, 2 * sub + c), rq[c].x, rq[c].y, rq[c].z,
-                     rq[c].w);
       fence_proxy_async_smem();
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars.q_ready);
-    };
-
-    // exchange buffer i of this warp: 4 chunks x 32 lanes x 16 bytes at
-    // +i*XS_BYTES (same offsets in both CTAs); a thread's 16 pairs are its
-    // chunks 0..3
-    const uint32_t xs_own0 = sbase + OFF_XS + warp * (XS_BYTES / NSOFT) + lane * 16;
-    const uint32_t xs_peer0 = mapa_shared(xs_own0, peer);
-    const uint32_t xs_full_peer0 = mapa_shared(smem_u32(&bars.xs_full[0]), peer);
-    const uint32_t xs_free_peer0 = mapa_shared(smem_u32(&bars.xs_free[0]), peer);
-    int nx = 0;  // next tile whose exchange buffer this CTA consumes
-    const uint32_t bias_w = sbase + OFF_BIAS + warp * (KT * 4);  // this warp's copy of the tile's key biases
-    float m_used[2] = {-INFINITY, -INFINITY};  // running maxima of rows r0, r0 + 8 (log2 units)
-    float l_run[2] = {0.f, 0.f};               // this thread's parts of their row sums
-    uint32_t sa[NP], sb[NP];  // scaled partial scores as fp16 pairs: current, next
-    bool alive = true;
-    SHLA_TRACE_DECL
-
-    // own partial of tile t (position ct): TMEM -> x scale + (0 | -inf) per
-    // key -> fp16 pairs -> the peer's exchange buffer.  When the next tile
-    // (position cn) starts a new batch row, its Q~ replaces this one.
-    auto fetch_send = [&](int t, uint32_t (&dst)[NP], const TileCur& ct, const TileCur& cn) -> bool {
-      const int b2 = t & 1;
       __syncwarp();
-      asm volatile("st.shared.f32 [%0], %1;" ::"r"(bias_w + lane * 4),
-                   "f"(key_valid(ct.ilo, ct.lim) ? 0.f : -INFINITY)
-                   : "memory");
-      asm volatile("st.shared.f32 [%0], %1;" ::"r"(bias_w + (32 + lane) * 4),
-                   "f"(key_valid(ct.ihi, ct.lim) ? 0.f : -INFINITY)
-                   : "memory");
-      __syncwarp();
-      SHLA_T(11);
-      if (!warp_wait(&bars.s_full, t & 1, abort, p.status)) return false;
-      SHLA_T(0);
-      tc_fence_after();
-      {
-        uint32_t r[32];
-        tmem_ld_16x256b_x8(tmem + frag_base + T_S, r);
-        tc_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float2 bv;
-          asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];"
-                       : "=f"(bv.x), "=f"(bv.y)
-                       : "r"(bias_w + (8 * j + 2 * c4) * 4));
-          const float x00 = fmaf(__uint_as_float(r[4 * j]), p.scale_log2, bv.x);
-          const float x01 = fmaf(__uint_as_float(r[4 * j + 1]), p.scale_log2, bv.y);
-          const float x10 = fmaf(__uint_as_float(r[4 * j + 2]), p.scale_log2, bv.x);
-          const float x11 = fmaf(__uint_as_float(r[4 * j + 3]), p.scale_log2, bv.y);
-          dst[2 * j] = f16x2_from_f32_sat(x00, x01);
-          dst[2 * j + 1] = f16x2_from_f32_sat(x10, x11);
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&bars.s_empty);
-      // (the score tile just read was the last product that used the old Q~)
-      if (t + 1 < n && cn.jt == 0) load_q(cn.bb);
-      SHLA_T(1);
-      if (!warp_wait<true>(&bars.xs_free[b2], ((t >> 1) & 1) ^ 1, abort, p.status)) return false;
-      SHLA_T(2);
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        st_async_v4(xs_peer0 + b2 * XS_BYTES + k * 512, __uint_as_float(dst[4 * k]),
-                    __uint_as_float(dst[4 * k + 1]), __uint_as_float(dst[4 * k + 2]),
-                    __uint_as_float(dst[4 * k + 3]), xs_full_peer0 + b2 * 8);
-      SHLA_T(3);
-      return true;
+      if (lane == 0) mbar_arrive(&bars.q_ready);
     };
-
-    // the value product of tile t has completed.  Sound because the softmax
-    // waits for the product of tile t - 2 (same barrier, previous phase)
-    // before it writes tile t's P, so at most one phase of each barrier is
-    // ever outstanding when it is tested.
+    // the value product of tile t has completed in this CTA
     auto wait_pv = [&](int t) -> bool {
       if (!warp_wait(&bars.o_done[t & 1], (t >> 1) & 1, abort, p.status)) return false;
       tc_fence_after();
       return true;
     };
-
-    // epilogue of a segment: rows r0 and r0 + 8 of the CTA's latent half of
-    // O~ / l into the row's output (a row held by one cluster) or the
-    // segment's slot, and (rank 0) the segment's log-sum-exps
-    auto flush = [&](int i_last, int bb) -> bool {
-      float l[2];
+    // this thread's row of O~ (this CTA's latent half) times a
+    auto rescale_o = [&](float a) {
+#pragma unroll 1
+      for (int cc = 0; cc < 256; cc += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_base + T_O + cc, r);
+        tc_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        l[e] = l_run[e] + __shfl_xor_sync(0xffffffffu, l_run[e], 1);
-        l[e] += __shfl_xor_sync(0xffffffffu, l[e], 2);
+        for (int j = 0; j < 32; ++j) r[j] = f2u(u2f(r[j]) * a);
+        tmem_st32(tmem + lane_base + T_O + cc, r);
       }
+      tc_wait_st();
+    };
+    // epilogue of a segment: this thread's row of this CTA's half of O~ / l
+    // into the row's output (a row held by one cluster) or the segment's slot
+    auto flush = [&](int i_last, int bb, float l, float m, bool write_lse) -> bool {
       if (!wait_pv(i_last)) return false;
       const int cf = p.sch.c_first(bb);
       const int used = p.sch.c_last(bb) - cf + 1;  // clusters holding a segment of row bb
       const int slot = cid - cf;
-      const float inv0 = l[0] > 0.f ? 1.f / l[0] : 0.f;
-      const float inv1 = l[1] > 0.f ? 1.f / l[1] : 0.f;
-      __nv_bfloat16* dst0 =
-          (used == 1 ? p.omerged + ((size_t)bb * kH + row0) * kC
-                     : p.opart + (((size_t)bb * p.slots + slot) * kH + row0) * kC) +
-          rank * 256 + 2 * c4;
-      __nv_bfloat16* dst1 = dst0 + 8 * kC;
-      uint32_t r[16];
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* dst = (used == 1 ? p.omerged + ((size_t)bb * kH + h) * kC
+                                      : p.opart + (((size_t)bb * p.slots + slot) * kH + h) * kC) +
+                           rank * 256;
 #pragma unroll 1
       for (int cc = 0; cc < 256; cc += 32) {
-        tmem_ld_16x256b_x4(tmem + frag_base + T_O + cc, r);
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_base + T_O + cc, r);
         tc_wait_ld();
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          *reinterpret_cast<uint32_t*>(dst0 + cc + 8 * j) =
-              pack_bf16x2(__uint_as_float(r[4 * j]) * inv0, __uint_as_float(r[4 * j + 1]) * inv0);
-          *reinterpret_cast<uint32_t*>(dst1 + cc + 8 * j) =
-              pack_bf16x2(__uint_as_float(r[4 * j + 2]) * inv1, __uint_as_float(r[4 * j + 3]) * inv1);
+          uint4 o;
+          o.x = pack_bf16x2(u2f(r[8 * j]) * inv, u2f(r[8 * j + 1]) * inv);
+          o.y = pack_bf16x2(u2f(r[8 * j + 2]) * inv, u2f(r[8 * j + 3]) * inv);
+          o.z = pack_bf16x2(u2f(r[8 * j + 4]) * inv, u2f(r[8 * j + 5]) * inv);
+          o.w = pack_bf16x2(u2f(r[8 * j + 6]) * inv, u2f(r[8 * j + 7]) * inv);
+          *reinterpret_cast<uint4*>(dst + cc + 8 * j) = o;
         }
       }
       tc_fence_before();
-      if (used > 1 && rank == 0 && c4 == 0) {
-        float* lse = p.lse + ((size_t)bb * p.slots + slot) * kH + row0;
-        lse[0] = l[0] > 0.f ? m_used[0] + log2f(l[0]) : -INFINITY;
-        lse[8] = l[1] > 0.f ? m_used[1] + log2f(l[1]) : -INFINITY;
-      }
+      if (write_lse && used > 1)
+        p.lse[((size_t)bb * p.slots + slot) * kH + h] = l > 0.f ? m + log2f(l) : -INFINITY;
       return true;
     };
 
-    // tile positions: c0 = tile i, c1 = tile i + 1, c2 = tile i + 2
-    TileCur c0 = first_cur();
-    TileCur c1 = n > 1 ? advance(c0) : c0;
-    TileCur c2 = c1;
-    int prev_bb = c0.bb;
-    pdl_wait();  // q~ is the fold kernel's output (the other roles read only inputs)
-    load_q(c0.bb);
-
-    // one key tile: `cur` holds this thread's scaled partial scores of tile i
-    // on entry; the next tile's partial is fetched into `nxt` and sent first
-    auto step = [&](int i, uint32_t (&cur)[NP], uint32_t (&nxt)[NP]) -> bool {
-      if (i + 1 < n) {
-        c2 = i + 2 < n ? advance(c1) : c1;
-        SHLA_T(12);
-        if (!fetch_send(i + 1, nxt, c1, c2)) return false;
-      }
-      // add the peer's partial scores (other latent half) of this tile
-      const int b2 = i & 1;
-      SHLA_T(11);
-      if (!warp_wait<true>(&bars.xs_full[b2], (i >> 1) & 1, abort, p.status)) return false;
-      nx = i + 1;
-      SHLA_T(4);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        uint4 o;
-        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(o.x), "=r"(o.y), "=r"(o.z), "=r"(o.w)
-                     : "r"(xs_own0 + b2 * XS_BYTES + k * 512));
-        cur[4 * k] = hadd2_u(cur[4 * k], o.x);
-        cur[4 * k + 1] = hadd2_u(cur[4 * k + 1], o.y);
-        cur[4 * k + 2] = hadd2_u(cur[4 * k + 2], o.z);
-        cur[4 * k + 3] = hadd2_u(cur[4 * k + 3], o.w);
-      }
-      // next use of this buffer (tile i + 2): expect the peer's bytes again
-      if (tid == 0 && i + 2 < n) mbar_arrive_expect_tx(&bars.xs_full[b2], XS_TX_BYTES);
-      // row maxima of the tile: the thread's pairs, then its row's four lanes
-      float mt[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        uint32_t mx2 = hmax2_u(hmax2_u(cur[e], cur[e + 2]), hmax2_u(cur[e + 4], cur[e + 6]));
-        mx2 = hmax2_u(mx2, hmax2_u(hmax2_u(cur[e + 8], cur[e + 10]), hmax2_u(cur[e + 12], cur[e + 14])));
-        const float2 f = f16x2_to_f32x2(mx2);
-        mt[e] = fmaxf(f.x, f.y);
-        mt[e] = fmaxf(mt[e], __shfl_xor_sync(0xffffffffu, mt[e], 1));
-        mt[e] = fmaxf(mt[e], __shfl_xor_sync(0xffffffffu, mt[e], 2));
-      }
-      SHLA_T(5);
-
-      // a new segment: write out the previous one and restart the running max
-      const bool first = i == 0 || c0.jt == 0;
-      if (first && i > 0) {
-        if (!flush(i - 1, prev_bb)) return false;
-        m_used[0] = m_used[1] = -INFINITY;
-        l_run[0] = l_run[1] = 0.f;
-      }
-      float m_new[2];
-      bool rescale[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        m_new[e] = fmaxf(m_used[e], mt[e]);
-        rescale[e] = m_new[e] > m_used[e] + kRescaleThreshold;
-      }
-      SHLA_T(6);
-      if (!first && __any_sync(0xffffffffu, rescale[0] || rescale[1])) {
-        // O~ must hold the value product of tile i - 1 before it is scaled;
-        // warp-collective over the warp's 16 rows x 256 accumulator columns:
-        // rows that keep their maximum scale by 1
-        if (!wait_pv(i - 1)) return false;
-        const float a0 = rescale[0] ? fast_exp2(m_used[0] - m_new[0]) : 1.f;
-        const float a1 = rescale[1] ? fast_exp2(m_used[1] - m_new[1]) : 1.f;
-        l_run[0] *= a0;
-        l_run[1] *= a1;
-        uint32_t r[16];
+    if (wg0) {
+      SHLA_REGS_INC;
+      pdl_wait();  // q~ is the fold kernel's output (the other roles read only inputs)
+      load_q(bb0);
+    } else {
+      SHLA_REGS_DEC;
+    }
+    Pos c = {bb0, jt0};
+    int prev_bb = bb0;
+    if (wg0 && !owned) {
+      // ---------------- sender of the peer's heads' partial scores ----------------
+      const uint32_t xs_peer = mapa_shared(sbase + OFF_XS + xs_off, peer);
 #pragma unroll 1
-        for (int cc = 0; cc < 256; cc += 32) {
-          const uint32_t ta = tmem + frag_base + T_O + cc;
-          tmem_ld_16x256b_x4(ta, r);
+      for (int i = 0; i < n; ++i) {
+        const int b = i & 1;
+        if (!warp_wait(&bars.s_full[b], (i >> 1) & 1, abort, p.status)) { alive = false; break; }
+        tc_fence_after();
+        uint32_t s[64];
+        tmem_ld32(tmem + lane_base + T_S + b * KT, *reinterpret_cast<uint32_t(*)[32]>(s));
+        tmem_ld32(tmem + lane_base + T_S + b * KT + 32, *reinterpret_cast<uint32_t(*)[32]>(s + 32));
+        tc_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.s_free[b]);
+        // (the score tile just read was the last product that used this Q~)
+        if (c.jt == nt - 1 && i + 1 < n) load_q(c.bb + 1);
+        if (!warp_wait<true>(&bars.xs_free[b], ((i >> 1) & 1) ^ 1, abort, p.status)) { alive = false; break; }
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          st_async_u4(xs_peer + b * XS_BYTES + k * 512, s[4 * k], s[4 * k + 1], s[4 * k + 2],
+                      s[4 * k + 3], xs_full_peer + b * 8);
+        c = next_pos(c);
+      }
+    } else if (wg0) {
+      // ---------------- softmax of this CTA's heads ----------------
+      const uint32_t xs_own = sbase + OFF_XS + xs_off;
+      float m_used = -INFINITY;  // running maximum of the row (log2 units)
+      float l = 0.f;             // running sum of the row
+      int nx = 0;                // next tile whose exchange buffer this warp consumes
+#pragma unroll 1
+      for (int i = 0; i < n; ++i) {
+        const int b = i & 1;
+        const bool first = i == 0 || c.jt == 0;
+        if (!warp_wait(&bars.s_full[b], (i >> 1) & 1, abort, p.status)) { alive = false; break; }
+        tc_fence_after();
+        float s[64];
+        {
+          uint32_t r[64];
+          tmem_ld32(tmem + lane_base + T_S + b * KT, *reinterpret_cast<uint32_t(*)[32]>(r));
+          tmem_ld32(tmem + lane_base + T_S + b * KT + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
           tc_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            r[4 * j] = __float_as_uint(__uint_as_float(r[4 * j]) * a0);
-            r[4 * j + 1] = __float_as_uint(__uint_as_float(r[4 * j + 1]) * a0);
-            r[4 * j + 2] = __float_as_uint(__uint_as_float(r[4 * j + 2]) * a1);
-            r[4 * j + 3] = __float_as_uint(__uint_as_float(r[4 * j + 3]) * a1);
-          }
-          tmem_st_16x256b_x4(ta, r);
+          for (int j = 0; j < 64; ++j) s[j] = u2f(r[j]);
         }
-      }
-#pragma unroll
-      for (int e = 0; e < 2; ++e)
-        if (rescale[e]) m_used[e] = m_new[e];
-      SHLA_T(7);
-      // P buffer b2 was last read by the value product of tile i - 2
-      if (i >= 2 && !wait_pv(i - 2)) return false;
-      SHLA_T(8);
-      // P = 2^(s - m) on fp16 pairs, to TMEM buffer b2 as bf16 pairs (pair u
-      // lands in P column 4(u/2) + c of its row); the tile's row sums are
-      // added on fp16 pairs in a tree (each P <= 2^8 under the lazy rescale,
-      // so a thread's part of a row stays <= 2^12)
-      {
-        const bool live0 = m_used[0] != -INFINITY, live1 = m_used[1] != -INFINITY;
-        const uint32_t m20 = live0 ? f16x2_splat(m_used[0]) : 0u;
-        const uint32_t m21 = live1 ? f16x2_splat(m_used[1]) : 0u;
-        uint32_t w[NP], e[NP];
-#pragma unroll
-        for (int u = 0; u < NP; ++u) {
-          const bool live = (u & 1) ? live1 : live0;
-          e[u] = live ? hex2_u(hsub2_u(cur[u], (u & 1) ? m21 : m20)) : 0u;
-          const float2 f = f16x2_to_f32x2(e[u]);
-          w[u] = bf16x2_from_f32(f.x, f.y);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.s_free[b]);
+        if (c.jt == nt - 1 && i + 1 < n) load_q(c.bb + 1);
+        // a new segment: write out the previous one and restart the running state
+        if (first && i > 0) {
+          if (!flush(i - 1, prev_bb, l, m_used, true)) { alive = false; break; }
+          m_used = -INFINITY;
+          l = 0.f;
         }
+        // valid keys of the tile (its stage stays in place until the tile's value product)
+        if (!warp_wait(&bars.full[i % NST], (i / NST) & 1, abort, p.status)) { alive = false; break; }
+        const unsigned long long vmask = *reinterpret_cast<volatile unsigned long long*>(&bars.mask[i % NST]);
+        // the peer's partial scores of these rows (the other latent half)
+        if (!warp_wait<true>(&bars.xs_full[b], (i >> 1) & 1, abort, p.status)) { alive = false; break; }
+        nx = i + 1;
 #pragma unroll
-        for (int d = 2; d < NP; d *= 2)
+        for (int k = 0; k < 16; ++k) {
+          const uint4 v = ld_shared_v4(xs_own + b * XS_BYTES + k * 512);
+          s[4 * k] += u2f(v.x);
+          s[4 * k + 1] += u2f(v.y);
+          s[4 * k + 2] += u2f(v.z);
+          s[4 * k + 3] += u2f(v.w);
+        }
+        __syncwarp();
+        if (lane == 0) {
+          // next use of this buffer (tile i + 2): expect the peer's bytes again,
+          // then let the peer write them
+          if (ql == 0 && i + 2 < n) mbar_arrive_expect_tx(&bars.xs_full[b], XS_TX);
+          mbar_arrive_cluster(xs_free_peer + b * 8);
+        }
+        // scale to log2 units, mask, tile maximum (fp32)
+        float mt = -INFINITY;
 #pragma unroll
-          for (int u = 0; u < NP; u += 2 * d) {
-            e[u] = hadd2_u(e[u], e[u + d]);
-            e[u + 1] = hadd2_u(e[u + 1], e[u + 1 + d]);
+        for (int j = 0; j < 64; ++j) {
+          s[j] = ((vmask >> j) & 1ull) ? s[j] * p.scale_log2 : -INFINITY;
+          mt = fmaxf(mt, s[j]);
+        }
+        const bool resc = mt > m_used + kRescaleThreshold;
+        const float alpha = (resc && !first) ? fast_exp2(m_used - mt) : 1.f;
+        if (!first && __any_sync(0xffffffffu, resc)) {
+          // O~ must hold the value product of tile i - 1 before it is scaled
+          if (!wait_pv(i - 1)) { alive = false; break; }
+          rescale_o(alpha);
+        }
+        if (resc) {
+          l *= alpha;
+          m_used = mt;
+        }
+        // P buffer b was last read by both CTAs' value products of tile i - 2
+        if (i >= 2 && !warp_wait<true>(&bars.pv_both[b], ((i - 2) >> 1) & 1, abort, p.status)) {
+          alive = false;
+          break;
+        }
+        // P = 2^(s - m) in fp32, rounded to bf16 into both CTAs' P buffer b
+        const bool live = m_used != -INFINITY;
+        const uint32_t p_loc = sbase + OFF_P + b * PBUF;
+        const uint32_t p_rem = p_peer + b * PBUF;
+        float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+        for (int j8 = 0; j8 < 8; ++j8) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = live ? fast_exp2(s[8 * j8 + 2 * e] - m_used) : 0.f;
+            const float x1 = live ? fast_exp2(s[8 * j8 + 2 * e + 1] - m_used) : 0.f;
+            ls0 += x0;
+            ls1 += x1;
+            w[e] = pack_bf16x2(x0, x1);
           }
-        const float2 l0 = f16x2_to_f32x2(e[0]), l1 = f16x2_to_f32x2(e[1]);
-        l_run[0] += l0.x + l0.y;
-        l_run[1] += l1.x + l1.y;
-        tmem_st_16x128b_x8(tmem + frag_base + T_P + b2 * (KT / 2), w);
+          const uint32_t off = sw128_off(h, j8);
+          st_shared_v4(p_loc + off, w[0], w[1], w[2], w[3]);
+          st_async_u4(p_rem + off, w[0], w[1], w[2], w[3], pp_full_peer + b * 8);
+        }
+        l += ls0 + ls1;
+        st_async_u4(p_rem + P_BYTES + h * 16, f2u(alpha), f2u(l), f2u(m_used), 0u,
+                    pp_full_peer + b * 8);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.p_own[b]);
+        prev_bb = c.bb;
+        c = next_pos(c);
       }
-      tc_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bars.p_full[b2]);
-      // this tile's exchange buffer can take the peer's tile i + 2 (its reads
-      // completed above)
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster_relaxed(xs_free_peer0 + b2 * 8);
-      prev_bb = c0.bb;
-      c0 = c1;
-      c1 = c2;
-      SHLA_T(9);
-      return true;
-    };
-
-    alive = fetch_send(0, sa, c0, c1);
+      if (__all_sync(0xffffffffu, alive) && !*abort) flush(n - 1, prev_bb, l, m_used, true);
+      // on an abort, partial scores the peer may still be sending land before
+      // the CTA can leave: the armed, unconsumed phases (bounded waits; none
+      // remain on the normal path)
+      for (int t = nx; t < n && t < nx + 2; ++t)
+        warp_wait<true>(&bars.xs_full[t & 1], (t >> 1) & 1, nullptr, nullptr);
+    } else {
+      // ---------------- receiver of the peer's P rows for these heads ----------------
+      float l_r = 0.f, m_r = -INFINITY;  // the owner's running state after the last tile
+      int nx = 0;
 #pragma unroll 1
-    for (int i = 0; i < n && alive; ++i) {
-      if (!step(i, sa, sb)) { alive = false; break; }
-#pragma unroll
-      for (int u = 0; u < NP; ++u) sa[u] = sb[u];
+      for (int i = 0; i < n; ++i) {
+        const int b = i & 1;
+        const bool first = i == 0 || c.jt == 0;
+        if (first && i > 0) {
+          if (!flush(i - 1, prev_bb, l_r, m_r, false)) { alive = false; break; }
+        }
+        if (!warp_wait<true>(&bars.pp_full[b], (i >> 1) & 1, abort, p.status)) { alive = false; break; }
+        nx = i + 1;
+        const uint4 a = ld_shared_v4(sbase + OFF_P + b * PBUF + P_BYTES + h * 16);
+        // the P rows that landed are read next by the value product (async proxy)
+        fence_proxy_async_smem();
+        __syncwarp();
+        // next use of this buffer (tile i + 2): the peer writes it only after
+        // this CTA's value product of tile i, which waits for this warp
+        if (lane == 0 && ql == 0 && i + 2 < n) mbar_arrive_expect_tx(&bars.pp_full[b], PP_TX);
+        const float alpha = u2f(a.x);
+        if (!first && __any_sync(0xffffffffu, alpha != 1.f)) {
+          if (!wait_pv(i - 1)) { alive = false; break; }
+          rescale_o(alpha);
+        }
+        l_r = u2f(a.y);
+        m_r = u2f(a.z);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.peer_ok[b]);
+        prev_bb = c.bb;
+        c = next_pos(c);
+      }
+      if (__all_sync(0xffffffffu, alive) && !*abort) flush(n - 1, prev_bb, l_r, m_r, false);
+      for (int t = nx; t < n && t < nx + 2; ++t)
+        warp_wait<true>(&bars.pp_full[t & 1], (t >> 1) & 1, nullptr, nullptr);
     }
-    SHLA_T(10);
-    if (lane == 0) SHLA_TRACE_FLUSH(0);
-    if (__all_sync(0xffffffffu, alive && !*abort)) flush(n - 1, prev_bb);
-    // on an abort, partial scores the peer may still be sending land before
-    // the CTA can leave: the armed, unconsumed phases (bounded waits; none
-    // remain on the normal path)
-    for (int t = nx; t < n && t < nx + 2; ++t)
-      warp_wait<true>(&bars.xs_full[t & 1], (t >> 1) & 1, nullptr, nullptr);
   }
 
   tc_fence_before();
@@ -893,6 +858,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
   }
   // neither CTA leaves while its peer may still touch its shared memory
   cluster_sync_all();
+#undef SHLA_REGS_DEC
+#undef SHLA_REGS_INC
 }
 
 // ===========================================================================
@@ -1323,6 +1290,10 @@ static int decode_impl(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_
   core::Params p;
   p.q_tilde = q_tilde;
   p.q_pe = reinterpret_cast<const __nv_bfloat16*>(q_pe);
+  p.ckv = reinterpret_cast<const __nv_bfloat16*>(c_kv);
+  p.kpe = reinterpret_cast<const __nv_bfloat16*>(k_pe);
+  p.ckv_rs = ckv_rstride;
+  p.kpe_rs = kpe_rstride;
   p.rows_per_b = ckv_bstride / ckv_rstride;
   p.q_per_row = q_per_row;
   p.T = T;
@@ -1408,14 +1379,3 @@ extern "C" int mla_decode_phase(int phase, const mla_bf16_t* q_nope, const mla_b
                      kpe_bstride, kpe_rstride, T, topk, k, end_pos, B, 1, scale, O, ws, ws_bytes,
                      status, stream);
 }
-
-#ifdef SHLA_TRACE
-extern "C" int mla_trace_read(void* host, size_t bytes) {
-  if (bytes < sizeof(shla::g_trace)) return MLA_ERR_SHAPE;
-  return cudaMemcpyFromSymbol(host, shla::g_trace, sizeof(shla::g_trace)) == cudaSuccess ? 0 : MLA_ERR_CUDA;
-}
-extern "C" int mla_trace_clear() {
-  static unsigned long long z[512][3][16];
-  return cudaMemcpyToSymbol(shla::g_trace, z, sizeof(z)) == cudaSuccess ? 0 : MLA_ERR_CUDA;
-}
-#endif
