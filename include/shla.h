@@ -128,7 +128,9 @@ int mla_cache_write(const mla_bf16_t* x, const mla_bf16_t* w_kva, const mla_bf16
  *
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
- * capture.  All calls share the array and it keeps the last call's contents;
+ * capture.  The address belongs to the device's context: a call made after
+ * the context was replaced (cudaDeviceReset and a new context) looks it up
+ * again.  All calls share the array and it keeps the last call's contents;
  * every value a call reads from it is written earlier in the same call, so
  * nothing needs clearing, but calls that can overlap on the GPU (different
  * streams, or different host threads) race on it and must be serialised by

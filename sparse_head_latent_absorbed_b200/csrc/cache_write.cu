@@ -157,7 +157,7 @@ template <int NB>
 static int launch_cw_gemm(const __nv_bfloat16* x, const __nv_bfloat16* w, int rows, float* part,
                           cudaStream_t st) {
   const int smem = 65536 + NB * 512 + 1024;
-  static unsigned long long attr_done = 0;
+  static std::atomic<unsigned long long> attr_done{0};
   if (int e = ensure_smem_attr(cw_gemm_kernel<NB>, smem, &attr_done)) return e;
   dim3 grid(cw::MT, cw::NKCH, (rows + NB - 1) / NB);
   cw_gemm_kernel<NB><<<grid, 128, smem, st>>>(x, w, rows, part, nullptr);
@@ -222,7 +222,9 @@ extern "C" int mla_cache_write(const mla_bf16_t* x, const mla_bf16_t* w_kva,
 // (28 x 64 x 576 floats = 4,128,768 bytes) on every GPU that loads this
 // library, until the process exits.  Its host-side name is only a stand-in:
 // the device address is looked up with cudaGetSymbolAddress once per device,
-// by the first call made with that device current.
+// by the first call made with that device current, and looked up again when
+// the device's context is no longer the one the address was taken in (after
+// cudaDeviceReset, the old address points at freed memory).
 // ---------------------------------------------------------------------------
 namespace shla {
 namespace noalloc {
@@ -231,19 +233,55 @@ static __device__ __align__(256) float g_scratch[cw::NKCH * kMaxRows * cw::kOut]
 
 static std::mutex g_mu;
 static float* g_addr[64] = {nullptr};
+static unsigned long long g_ctx_id[64] = {0};  // context the address belongs to
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// unique id of the calling thread's current context (0 when there is none);
+// driver ids are never reused within a process
+static unsigned long long current_context_id() {
+  static const CtxGetCurrentFn get_current = []() -> CtxGetCurrentFn {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<CtxGetCurrentFn>(f);
+    cudaGetLastError();
+    return nullptr;
+  }();
+  static const CtxGetIdFn get_id = []() -> CtxGetIdFn {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<CtxGetIdFn>(f);
+    cudaGetLastError();
+    return nullptr;
+  }();
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 // device address of g_scratch for the current device (set-up on first use)
 static int scratch_for_current_device(float** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MLA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_addr[dev]) {
+  const unsigned long long id = current_context_id();
+  if (!g_addr[dev] || id == 0 || id != g_ctx_id[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || !p) {
       cudaGetLastError();
       return MLA_ERR_CUDA;
     }
     g_addr[dev] = static_cast<float*>(p);
+    // the symbol lookup made the device's context current if none was
+    g_ctx_id[dev] = current_context_id();
   }
   *out = g_addr[dev];
   return MLA_OK;

@@ -134,6 +134,21 @@ DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
                : "memory");
 }
 
+// Relaxed forms, for arrivals that need no ordering of this thread's earlier
+// memory accesses beyond what has visibly completed (values already loaded
+// and consumed, tcgen05 loads waited for).  A release arrive would also wait
+// for the thread's earlier stores to other CTAs' shared memory.
+DEV void mbar_arrive_relaxed(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+DEV void mbar_arrive_expect_tx_relaxed(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.relaxed.cta.shared::cta.b64 _, [%0], %1;" ::"r"(
+                   smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
 // Bounded wait for the phase with the given parity to complete.  Returns
 // false (after flagging ``*abort`` and the status word) when the limit
 // expires or when another thread of the CTA has already aborted.

@@ -139,34 +139,30 @@ __global__ void __launch_bounds__(128) fold_kernel(const __nv_bfloat16* __restri
 // merges.
 //
 // CTA r of the pair holds latent columns [256r, 256r+256) and rotary columns
-// [32r, 32r+32) of Q~ and of every selected cache row, for all 128 heads, and
-// runs the softmax of the 64 heads in TMEM lane quarters 2r and 2r+1.  Per key
-// tile (KT keys):
+// [32r, 32r+32) of Q~ and of every selected cache row, for all 128 heads.  Per
+// key tile (KT keys):
 //   S_r  = Q~_r K_r^T        partial scores, M=128 heads, N=KT, K=288 (tcgen05)
-//   the peer's heads' partial scores go to the peer in fp32 (st.async); the
-//   owner adds the two halves in fp32, scales to log2 units, sets invalid keys
-//   to -inf and runs the online softmax in fp32: running maximum m (raised
-//   lazily, once the tile maximum exceeds it by more than 8), P = 2^(s - m)
-//   rounded to bf16, row sum l of the fp32 P
-//   the owner's P rows go to both CTAs' shared memory, with (alpha, l, m) per
-//   row; alpha = 2^(m_old - m_new) rescales that row of O~ in both CTAs
-//   O_r += P V_r             M=128, N=256, K=KT, A = P from shared memory
+//   each CTA sends its partial scores to the peer in fp32 (st.async) and adds
+//   the peer's to its own, a + b in one CTA and b + a in the other, which are
+//   the same fp32 numbers: both CTAs then scale to log2 units, set invalid
+//   keys to -inf and run the same fp32 online softmax, bit for bit (running
+//   maximum m, raised lazily once the tile maximum exceeds it by more than 8;
+//   P = 2^(s - m) rounded to bf16; row sum l of the fp32 P), so nothing else
+//   crosses between them
+//   O_r += P V_r             M=128, N=256, K=KT, A = P from TMEM
 // V is the same shared-memory tile as K, read MN-major.
 //
-// Warp roles (512 threads) in CTA r; q = warp % 4 is a warp's TMEM lane quarter:
-//   warps 0-3   quarter q owned (q / 2 == r): softmax of its 32 heads
-//               otherwise: sends its 32 heads' partial scores to the peer
-//               (all four load their rows of this CTA's half of Q~ at each
-//               segment start)
-//   warps 4-7   quarter q owned: gather; otherwise: receives the peer's
-//               (alpha, l, m) of its 32 heads, rescales and writes out their
-//               rows of this CTA's half of O~
-//   warps 8-13  gather: TMA tile::gather4 of the selected rows, two groups of
-//               four keys per gather warp and tile
-//   warp 14     L2 prefetch of the selected rows a few tiles ahead
-//   warp 15     TMEM owner and MMA issuer (one thread)
-// TMEM (512 columns): latent half of Q~ [0,128) as bf16 pairs, two score
-// tiles [128,256), O~ (latent half, fp32) [256,512).
+// Warp roles (640 threads):
+//   warps 0-7   softmax: warp w takes the 16 rows [32q + 16h, +16) of lane
+//               quarter q = w % 4, h = w / 4, and all keys of a tile, four
+//               threads per row (16x256b TMEM fragments).  They also load
+//               Q~ at each segment start.
+//   warps 8-11  send the partial scores of lane quarter w - 8 to the peer
+//   warps 12-18 gather: TMA tile::gather4 of the selected rows
+//   warp 19     TMEM owner and MMA issuer (one thread)
+// TMEM (512 columns): latent half of Q~ [0,128) as bf16 pairs, the score
+// tile [128,192), two P tiles [192,256) as bf16 pairs, O~ (latent half,
+// fp32) [256,512).
 // ===========================================================================
 DEV uint32_t f2u(float x) { return __float_as_uint(x); }
 DEV float u2f(uint32_t x) { return __uint_as_float(x); }
@@ -174,37 +170,34 @@ DEV float u2f(uint32_t x) { return __uint_as_float(x); }
 namespace core {
 constexpr int KT = 64;                       // keys per tile
 constexpr int NST = 4;                       // gather ring depth
-constexpr int NGATHER = 8;                   // gather warps
-constexpr int PF_WARP = 14, MMA_WARP = 15;
-constexpr int NTHREADS = 512;
-constexpr int PF_AHEAD = 4;                  // prefetch distance, tiles ahead of the score products
+constexpr int NSOFT = 8;                     // softmax warps
+constexpr int SEND_WARP0 = 8;                // sender warps 8-11
+constexpr int GATHER_WARP0 = 12;
+constexpr int NGATHER = 7;                   // gather warps 12-18
+constexpr int MMA_WARP = 19;
+constexpr int NTHREADS = 32 * (MMA_WARP + 1);  // 640
 constexpr int ST_ATOM = KT * 128;            // one 64-column latent atom of a tile
 constexpr int ST_KR = 4 * ST_ATOM;           // rotary part of a tile (64 B swizzle)
 constexpr int ST_BYTES = ST_KR + KT * 64;    // 36864
 constexpr int OFF_ST = 0;
 constexpr int OFF_QR = OFF_ST + NST * ST_BYTES;  // rotary half of Q: 128 rows x 64 B, 64 B swizzle
-constexpr int OFF_XS = OFF_QR + 128 * 64;        // received partial scores, two buffers
-constexpr int XS_BYTES = 2 * 16 * 32 * 16;       // [2 quarters][16 chunks][32 lanes][16 B]
-constexpr int OFF_P = OFF_XS + 2 * XS_BYTES;     // P of all 128 heads, two buffers
-constexpr int P_BYTES = 128 * 128;               // [128 rows][64 keys] bf16, 128 B swizzle, K-major
-constexpr int PA_BYTES = 128 * 16;               // per row: alpha, l, m (fp32)
-constexpr int PBUF = P_BYTES + PA_BYTES;
-constexpr int OFF_END = OFF_P + 2 * PBUF;
+constexpr int OFF_XS = OFF_QR + 128 * 64;        // the peer's partial scores, two buffers
+constexpr int XS_BYTES = NSOFT * 8 * 32 * 16;    // [softmax warp][8 chunks][32 lanes][16 B]
+constexpr int OFF_BIAS = OFF_XS + 2 * XS_BYTES;  // per stage: 0 / -inf per key
+constexpr int OFF_END = OFF_BIAS + NST * KT * 4;
 constexpr int SMEM_BYTES = OFF_END + 1024;       // + alignment slack
 constexpr uint32_t XS_TX = XS_BYTES;             // partial scores received per tile
-constexpr uint32_t PP_TX = 64 * (128 + 16);      // P rows and (alpha, l, m) received per tile
-constexpr uint32_t GROUP_TX_BYTES = ST_BYTES / 16;  // bytes of one group of four keys
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t T_Q = 0, T_S = 128, T_O = 256;
-constexpr int REGS_WG0 = 152, REGS_REST = 120;
-static_assert(128 * (REGS_WG0 + 3 * REGS_REST) <= 65536, "register split");
+constexpr uint32_t T_Q = 0, T_S = 128, T_P = 192, T_O = 256;
 constexpr float kRescaleThreshold = 8.0f;        // log2 units
-static_assert(ST_BYTES % 1024 == 0 && OFF_QR % 1024 == 0 && OFF_P % 1024 == 0 &&
-                  PBUF % 1024 == 0 && OFF_XS % 16 == 0,
-              "alignment");
+// register split (the launch gives 96 per thread): softmax 112, senders 96,
+// gather / MMA 80: 2 x 112 + 96 + 2 x 80 = 5 x 96
+constexpr int REGS_SOFT = 112, REGS_SEND = 96, REGS_REST = 80;
+static_assert(128 * (2 * REGS_SOFT + REGS_SEND + 2 * REGS_REST) <= NTHREADS * 96, "register split");
+static_assert(ST_BYTES % 1024 == 0 && OFF_QR % 1024 == 0 && OFF_XS % 16 == 0, "alignment");
 static_assert(SMEM_BYTES + 512 <= 232448, "shared memory budget");
-static_assert(T_Q + 128 <= T_S && T_S + 2 * KT <= T_O && T_O + 256 <= TMEM_COLS, "TMEM plan");
-static_assert(KT / 4 == 2 * NGATHER, "two groups of four keys per gather warp and tile");
+static_assert(T_Q + 128 <= T_S && T_S + KT <= T_P && T_P + KT <= T_O && T_O + 256 <= TMEM_COLS,
+              "TMEM plan");
 
 // Schedule: tiles [bnd(c), bnd(c+1)) of the flattened list belong to cluster c.
 struct Sched {
@@ -224,9 +217,6 @@ struct Sched {
 struct Params {
   const __nv_bfloat16* q_tilde;   // [B][128][512]
   const __nv_bfloat16* q_pe;      // [B][128][64]
-  const __nv_bfloat16* ckv;       // latent part of cache row 0 (prefetch addresses)
-  const __nv_bfloat16* kpe;       // rotary part of cache row 0
-  int ckv_rs, kpe_rs;             // row strides in elements
   long long rows_per_b;           // row-index distance between batch rows in the cache maps
   int q_per_row;                  // query rows per cache batch row (query row r reads row r / q_per_row)
   int T;
@@ -245,19 +235,14 @@ struct Params {
 
 struct Bars {
   uint64_t full[NST], empty[NST];  // gather ring
-  uint64_t s_full[2], s_free[2];   // score tile t & 1 in TMEM / read by warps 0-3
+  uint64_t s_full, s_empty;        // score tile in TMEM / read by the softmax and send warps
   uint64_t xs_full[2], xs_free[2]; // peer's partial scores landed / this CTA's buffer read by the peer
-  uint64_t p_own[2];               // this CTA's P rows of tile t & 1 written
-  uint64_t pp_full[2];             // the peer's P rows and (alpha, l, m) landed
-  uint64_t peer_ok[2];             // the peer's rows of O~ rescaled for tile t & 1
-  uint64_t o_done[2];              // this CTA's value product of tile t has completed
-  uint64_t pv_both[2];             // both CTAs' value products of tile t have completed
+  uint64_t p_full[2];              // P of tile t is in TMEM buffer t & 1
+  uint64_t o_done[2];              // the value product of tile t has completed
   uint64_t q_ready;                // the segment's Q~ is in TMEM / shared memory
   uint64_t drain;
-  unsigned long long mask[NST];    // valid keys of the tile in each ring stage
   uint32_t tmem_base;
   int abort;
-  int prog;                        // score products issued (read by the prefetch warp)
 };
 
 DEV bool key_valid(int v, int lim) { return v >= 0 && v < lim; }
@@ -333,12 +318,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     return c;
   };
 
-  const int q4 = warp & 3;                    // TMEM lane quarter of warps 0-7
-  const bool owned = (q4 >> 1) == (int)rank;  // the quarter's heads are this CTA's
-  const int ql = q4 & 1;                      // index of the quarter within its CTA's pair
-  const bool is_gather = warp >= 8 ? warp < 8 + 6 : (warp >= 4 && owned);
-  const int gw = warp >= 8 ? warp - 8 : 6 + ql;  // gather warp index (0..7)
-
   if (warp == MMA_WARP) {
     tmem_alloc(&bars.tmem_base, TMEM_COLS);
     tmem_relinquish();
@@ -348,42 +327,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       mbar_init(&bars.full[s], NGATHER);  // one expect_tx arrival per gather warp + bytes
       mbar_init(&bars.empty[s], 1);       // MMA commit after the tile's value product
     }
+    mbar_init(&bars.s_full, 1);
+    mbar_init(&bars.s_empty, NSOFT + 4);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.s_full[i], 1);
-      mbar_init(&bars.s_free[i], 4);
-      mbar_init(&bars.xs_full[i], 1);   // own expect_tx arrival + the peer's st.async bytes
-      mbar_init(&bars.xs_free[i], 2);   // one arrival per softmax warp of the peer
-      mbar_init(&bars.p_own[i], 2);
-      mbar_init(&bars.pp_full[i], 1);   // own expect_tx arrival + the peer's st.async bytes
-      mbar_init(&bars.peer_ok[i], 2);
+      mbar_init(&bars.xs_full[i], 1);     // own expect_tx arrival + the peer's st.async bytes
+      mbar_init(&bars.xs_free[i], NSOFT); // one arrival per softmax warp of the peer
+      mbar_init(&bars.p_full[i], NSOFT);
       mbar_init(&bars.o_done[i], 1);
-      mbar_init(&bars.pv_both[i], 2);   // this CTA's and the peer's value-product commits
     }
-    mbar_init(&bars.q_ready, 4);
+    mbar_init(&bars.q_ready, NSOFT);
     mbar_init(&bars.drain, 1);
     bars.abort = 0;
-    bars.prog = 0;
     fence_mbarrier_init_cluster();
-    for (int i = 0; i < 2 && i < n; ++i) {
-      mbar_arrive_expect_tx(&bars.xs_full[i], XS_TX);
-      mbar_arrive_expect_tx(&bars.pp_full[i], PP_TX);
-    }
+    for (int i = 0; i < 2 && i < n; ++i) mbar_arrive_expect_tx(&bars.xs_full[i], XS_TX);
   }
   tc_fence_before();
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
-  // Register split (the launch gives 128 per thread): warps 0-3 take
-  // REGS_WG0, every other warp REGS_REST; each role branch below starts with
-  // its warpgroup's setmaxnreg (warps 4-7 mix two roles with the same value).
-#define SHLA_REGS_DEC asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_REST))
-#define SHLA_REGS_INC asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_WG0))
 
-  if (is_gather) {
-    SHLA_REGS_DEC;
+  if (warp >= GATHER_WARP0 && warp < MMA_WARP) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_REST));
     // ---------------- gather (TMA tile::gather4) ----------------
-    // lane l holds the index of key l and key 32 + l of the tile; lanes 0
-    // and 1 each issue the five loads of one group of four keys
+    // lane l holds the index of key l and key 32 + l of the tile; lanes
+    // 0..ng-1 each issue the five loads of one group of four keys
+    const int gw = warp - GATHER_WARP0;
+    const int ng = (16 - gw + NGATHER - 1) / NGATHER;  // groups of this warp
+    constexpr uint32_t GROUP_TX_BYTES = ST_BYTES / 16;
     int bad = 0, issued = 0;
     int base_bb = -1;      // query row whose cache base is in `base`
     long long base = 0;    // first TMA row of that query row's cache batch row
@@ -393,7 +363,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       const int s = i % NST;
       const bool oka = key_valid(cur.ilo, cur.lim), okb = key_valid(cur.ihi, cur.lim);
       if (rank == 0 && gw == 0) bad += (!oka && cur.ilo != -1) + (!okb && cur.ihi != -1);
-      const uint32_t vlo = __ballot_sync(0xffffffffu, oka), vhi = __ballot_sync(0xffffffffu, okb);
       // TMA rows: valid keys map to their cache row, others to row -1 (zero fill)
       if (cur.bb != base_bb) {
         base_bb = cur.bb;
@@ -403,13 +372,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       const int rb = okb ? (int)(base + cur.ihi) : -1;
       if (i + 1 < n) cur = advance(cur);
       if (!warp_wait(&bars.empty[s], ((i / NST) & 1) ^ 1, abort, p.status)) break;
-      if (lane == 0) {
-        if (gw == 0) bars.mask[s] = (unsigned long long)vlo | ((unsigned long long)vhi << 32);
-        mbar_arrive_expect_tx(&bars.full[s], 2 * GROUP_TX_BYTES);
+      if (gw == 0) {
+        // the tile's key biases (0 / -inf), read by the softmax warps
+        const uint32_t bias = sbase + OFF_BIAS + s * (KT * 4);
+        asm volatile("st.shared.f32 [%0], %1;" ::"r"(bias + lane * 4), "f"(oka ? 0.f : -INFINITY)
+                     : "memory");
+        asm volatile("st.shared.f32 [%0], %1;" ::"r"(bias + (32 + lane) * 4),
+                     "f"(okb ? 0.f : -INFINITY)
+                     : "memory");
+        __syncwarp();
       }
+      if (lane == 0) mbar_arrive_expect_tx(&bars.full[s], ng * GROUP_TX_BYTES);
       __syncwarp();
-      const int g = gw + NGATHER * (lane & 1);  // this lane's group (lanes 0 and 1 issue)
-      const int k0 = 4 * g;                     // its first key (0..60)
+      const int g = gw + NGATHER * (lane < ng ? lane : 0);  // this lane's group
+      const int k0 = 4 * g;                                 // its first key (0..60)
       const int src = k0 & 31;
       const int y0 = __shfl_sync(0xffffffffu, ra, src);
       const int y0b = __shfl_sync(0xffffffffu, rb, src);
@@ -419,7 +395,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       const int y2b = __shfl_sync(0xffffffffu, rb, src + 2);
       const int y3 = __shfl_sync(0xffffffffu, ra, src + 3);
       const int y3b = __shfl_sync(0xffffffffu, rb, src + 3);
-      if (lane < 2) {
+      if (lane < ng) {
         const bool hi = k0 >= 32;
         const int r0 = hi ? y0b : y0, r1 = hi ? y1b : y1, r2 = hi ? y2b : y2, r3 = hi ? y3b : y3;
         const uint32_t stage = sbase + OFF_ST + s * ST_BYTES;
@@ -438,52 +414,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);
     if (lane == 0 && bad && p.status) atomicAdd(p.status + 1, bad);
-  } else if (warp == PF_WARP) {
-    SHLA_REGS_DEC;
-    // ---------------- L2 prefetch of the rows PF_AHEAD tiles ahead ----------------
-    // lines of this CTA's part of each valid selected row (latent half and
-    // rotary half); they land in L2 before the gather asks for them
-    TileCur cur = first_cur();
-    const uint64_t t0 = globaltimer_ns();
-#pragma unroll 1
-    for (int i = 0; i < n; ++i) {
-      bool late = false;
-      while (*(volatile int*)&bars.prog < i - PF_AHEAD) {
-        if (*abort || globaltimer_ns() - t0 > kWaitLimitNs) {
-          late = true;
-          break;
-        }
-        __nanosleep(256);
-      }
-      if (late) break;
-      const long long base = (long long)(cur.bb / p.q_per_row) * p.rows_per_b;
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int v = e ? cur.ihi : cur.ilo;
-        if (!key_valid(v, cur.lim)) continue;
-        const long long row = base + v;
-        const char* lat = reinterpret_cast<const char*>(p.ckv + row * p.ckv_rs + rank * 256);
-        const char* rot = reinterpret_cast<const char*>(p.kpe + row * p.kpe_rs + rank * 32);
-#pragma unroll
-        for (int l = 0; l < 4; ++l) prefetch_l2(lat + l * 128);
-        prefetch_l2(lat + 511);
-        prefetch_l2(rot);
-        prefetch_l2(rot + 63);
-      }
-      if (i + 1 < n) cur = advance(cur);
-    }
   } else if (warp == MMA_WARP) {
-    SHLA_REGS_DEC;
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_REST));
     // ---------------- MMA issuer ----------------
-    // Event loop.  A value product (A = P of tile t from shared memory
-    // buffer t & 1) goes first whenever both CTAs' P rows and rescales are
-    // in place; a score product as soon as its keys have landed, its score
-    // buffer has been read and this segment's Q~ is in place.
+    // Event loop.  A value product (A = P of tile t from TMEM buffer t & 1)
+    // goes first whenever its P is ready; a score product as soon as its keys
+    // have landed, the previous score tile has been read and this segment's
+    // Q~ is in place.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, KT, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, 0, 1);
-      // descriptors: a buffer's low word plus a constant per K-step
-      constexpr uint32_t hi_k128 = desc_hi(1024, kSwizzle128B);  // 128 B swizzle, 8-row groups 1 KB apart
+      // descriptors: a stage's low word plus a constant per K-step
+      constexpr uint32_t hi_k128 = desc_hi(1024, kSwizzle128B);  // 128 B swizzle
       constexpr uint32_t hi_k64 = desc_hi(512, kSwizzle64B);     // 64 B swizzle
       const uint32_t lo_qr = desc_lo(sbase + OFF_QR, 16);        // rotary half of Q
       int qk = 0, pv = 0, idle = 0, qseg = -1;
@@ -493,38 +435,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
 #pragma unroll 1
       while (pv < n) {
         bool did = false;
-        if (pv < qk && mbar_test(&bars.p_own[pv & 1], (pv >> 1) & 1) &&
-            mbar_test(&bars.peer_ok[pv & 1], (pv >> 1) & 1)) {
+        if (pv < qk && mbar_test(&bars.p_full[pv & 1], (pv >> 1) & 1)) {
           tc_fence_after();
-          const int b = pv & 1;
-          const uint32_t lo_p = desc_lo(sbase + OFF_P + b * PBUF, 16);              // P, K-major
-          const uint32_t lo_v = desc_lo(sbase + OFF_ST + ps * ST_BYTES, ST_ATOM);  // V, MN-major
+          const int s = ps;
+          const uint32_t lo = desc_lo(sbase + OFF_ST + s * ST_BYTES, ST_ATOM);  // V, MN-major
+          const uint32_t tp = tmem + T_P + (pv & 1) * (KT / 2);
           const bool first = pv == 0 || jp == 0;
           if (first)
-            tc_mma_c<false>(tmem + T_O, desc_join(lo_p, hi_k128), desc_join(lo_v, hi_k128), idesc_pv);
+            tc_mma_tmem_a_c<false>(tmem + T_O, tp, desc_join(lo, hi_k128), idesc_pv);
           else
-            tc_mma_c<true>(tmem + T_O, desc_join(lo_p, hi_k128), desc_join(lo_v, hi_k128), idesc_pv);
+            tc_mma_tmem_a_c<true>(tmem + T_O, tp, desc_join(lo, hi_k128), idesc_pv);
 #pragma unroll
           for (int ks = 1; ks < KT / 16; ++ks)
-            tc_mma_c<true>(tmem + T_O, desc_join(lo_p + ks * 2, hi_k128),
-                           desc_join(lo_v + ks * (2048 >> 4), hi_k128), idesc_pv);
-          tc_commit(&bars.o_done[b]);
-          tc_commit(&bars.empty[ps]);
-          tc_commit_mc(&bars.pv_both[b], 3);
+            tc_mma_tmem_a_c<true>(tmem + T_O, tp + ks * 8, desc_join(lo + ks * (2048 >> 4), hi_k128),
+                                  idesc_pv);
+          tc_commit(&bars.o_done[pv & 1]);
+          tc_commit(&bars.empty[s]);
           ++pv;
           if (++ps == NST) ps = 0;
           if (++jp == nt) jp = 0;
           did = true;
         }
         if (qk < n && mbar_test(&bars.full[qs], qph) &&
-            (qk < 2 || mbar_test(&bars.s_free[qk & 1], ((qk - 2) >> 1) & 1))) {
+            (qk == 0 || mbar_test(&bars.s_empty, (qk - 1) & 1))) {
           const int seg = (qk == 0 || jq == 0) ? qseg + 1 : qseg;
           if (seg == qseg || mbar_test(&bars.q_ready, seg & 1)) {
             qseg = seg;
             tc_fence_after();
             const uint32_t st = sbase + OFF_ST + qs * ST_BYTES;
             const uint32_t lo = desc_lo(st, 16), lo_r = desc_lo(st + ST_KR, 16);
-            const uint32_t ts = tmem + T_S + (qk & 1) * KT;
+            const uint32_t ts = tmem + T_S;
             tc_mma_tmem_a_c<false>(ts, tmem + T_Q, desc_join(lo, hi_k128), idesc_qk);
 #pragma unroll
             for (int ks = 1; ks < 16; ++ks)
@@ -535,9 +475,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
             for (int ks = 0; ks < 2; ++ks)
               tc_mma_c<true>(ts, desc_join(lo_qr + ks * 2, hi_k64), desc_join(lo_r + ks * 2, hi_k64),
                              idesc_qk);
-            tc_commit(&bars.s_full[qk & 1]);
+            tc_commit(&bars.s_full);
             ++qk;
-            *(volatile int*)&bars.prog = qk;
             if (++qs == NST) {
               qs = 0;
               qph ^= 1;
@@ -551,7 +490,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
         if (did) {
           idle = 0;
           t_idle = 0;
-        } else if (++idle >= 64) {
+        } else if (__nanosleep(20), ++idle >= 64) {
+          // (nothing ready: the sleep leaves the issue slots to the softmax warps)
           idle = 0;
           if (*abort) break;
           const uint64_t now = globaltimer_ns();
@@ -567,30 +507,64 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       // everything issued so far has finished before TMEM is released
       tc_commit(&bars.drain);
       mbar_wait(&bars.drain, 0, nullptr, p.status);
-      // the peer's commits of its last value products land on this CTA's
-      // barriers before it leaves (bounded; complete on the normal path)
-      for (int t = max(0, pv - 2); t < pv; ++t)
-        mbar_wait(&bars.pv_both[t & 1], (t >> 1) & 1, nullptr, nullptr);
     }
     __syncwarp();
-  } else {
-    // ---------------- TMEM warps: softmax / sender (0-3), receiver (4-7) ----------------
-    const int h = q4 * 32 + lane;                                // this thread's head row
-    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-    const bool wg0 = warp < 4;
-    const uint32_t xs_off = ql * (XS_BYTES / 2) + lane * 16;    // + buffer + chunk * 512
-    const uint32_t p_peer = mapa_shared(sbase + OFF_P, peer);
-    const uint32_t pp_full_peer = mapa_shared(smem_u32(&bars.pp_full[0]), peer);
+  } else if (warp >= SEND_WARP0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_SEND));
+    // ---------------- send this quarter's partial scores to the peer ----------------
+    // fragments of both 16-lane halves of the quarter, in the register order
+    // of the peer's softmax warps for those rows
+    const int q4 = warp - SEND_WARP0;
+    const uint32_t xs_peer = mapa_shared(sbase + OFF_XS + lane * 16, peer);
     const uint32_t xs_full_peer = mapa_shared(smem_u32(&bars.xs_full[0]), peer);
+#pragma unroll 1
+    for (int i = 0; i < n; ++i) {
+      const int b = i & 1;
+      if (!warp_wait(&bars.s_full, i & 1, abort, p.status)) break;
+      tc_fence_after();
+      uint32_t r0[32], r1[32];
+      tmem_ld_16x256b_x8(tmem + ((uint32_t)(q4 * 32) << 16) + T_S, r0);
+      tmem_ld_16x256b_x8(tmem + ((uint32_t)(q4 * 32 + 16) << 16) + T_S, r1);
+      tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      // relaxed: the tcgen05 loads have completed (waited for above)
+      if (lane == 0) mbar_arrive_relaxed(&bars.s_empty);
+      if (!warp_wait<true>(&bars.xs_free[b], ((i >> 1) & 1) ^ 1, abort, p.status)) break;
+      const uint32_t dst = xs_peer + b * XS_BYTES;
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        st_async_u4(dst + q4 * 4096 + k * 512, r0[4 * k], r0[4 * k + 1], r0[4 * k + 2],
+                    r0[4 * k + 3], xs_full_peer + b * 8);
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        st_async_u4(dst + (q4 + 4) * 4096 + k * 512, r1[4 * k], r1[4 * k + 1], r1[4 * k + 2],
+                    r1[4 * k + 3], xs_full_peer + b * 8);
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFT));
+    // ---------------- softmax: rows [32q + 16h, +16), all keys ----------------
+    // Through the 16x256b TMEM shape thread t holds rows t/4 and t/4 + 8 of
+    // its 16 and, of each 8-key block j, keys 8j + 2(t%4) and 8j + 2(t%4) + 1:
+    // register 4j+e is (row t/4 + 8 (e/2), key 8j + 2(t%4) + e%2).
+    const int q4 = warp & 3, hf = warp >> 2;
+    const int c4 = lane & 3;
+    const int row0 = q4 * 32 + hf * 16 + (lane >> 2), row1 = row0 + 8;
+    const uint32_t frag = (uint32_t)(q4 * 32 + hf * 16) << 16;
+    const uint32_t xs_own = sbase + OFF_XS + warp * 4096 + lane * 16;
     const uint32_t xs_free_peer = mapa_shared(smem_u32(&bars.xs_free[0]), peer);
     bool alive = true;
 
-    // this warp's 32 rows of this CTA's half of Q~ for batch row bb: latent
-    // values into TMEM as bf16 pairs, rotary values into the swizzled shared tile
+    // this warp's share of this CTA's half of Q~ for batch row bb (32x32b
+    // shape, one row per thread): latent values [128 hf, +128) of the CTA's
+    // 256 into TMEM as bf16 pairs, rotary values [16 hf, +16) of its 32 into
+    // the swizzled shared tile; then q_ready
     auto load_q = [&](int bb) {
-      const __nv_bfloat16* qrow = p.q_tilde + ((size_t)bb * kH + h) * kC + rank * 256;
+      const int h = q4 * 32 + lane;
+      const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+      const __nv_bfloat16* qrow = p.q_tilde + ((size_t)bb * kH + h) * kC + rank * 256 + hf * 128;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint4 v[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = ld_global_nc_v4(qrow + c * 64 + i * 8);
@@ -602,13 +576,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
           r[4 * i + 2] = v[i].z;
           r[4 * i + 3] = v[i].w;
         }
-        tmem_st32(tmem + lane_base + T_Q + c * 32, r);
+        tmem_st32(tmem + lane_base + T_Q + hf * 64 + c * 32, r);
       }
-      const __nv_bfloat16* rrow = p.q_pe + ((size_t)bb * kH + h) * kR + rank * 32;
+      const __nv_bfloat16* rrow = p.q_pe + ((size_t)bb * kH + h) * kR + rank * 32 + hf * 16;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         const uint4 v = ld_global_nc_v4(rrow + c * 8);
-        st_shared_v4(sbase + OFF_QR + sw64_off(h, c), v.x, v.y, v.z, v.w);
+        st_shared_v4(sbase + OFF_QR + sw64_off(h, 2 * hf + c), v.x, v.y, v.z, v.w);
       }
       fence_proxy_async_smem();
       tc_wait_st();
@@ -616,238 +590,205 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.q_ready);
     };
-    // the value product of tile t has completed in this CTA
+    // the value product of tile t has completed
     auto wait_pv = [&](int t) -> bool {
       if (!warp_wait(&bars.o_done[t & 1], (t >> 1) & 1, abort, p.status)) return false;
       tc_fence_after();
       return true;
     };
-    // this thread's row of O~ (this CTA's latent half) times a
-    auto rescale_o = [&](float a) {
+    // this thread's two rows of this CTA's half of O~ times a0 / a1
+    auto rescale_o = [&](float a0, float a1) {
 #pragma unroll 1
       for (int cc = 0; cc < 256; cc += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_base + T_O + cc, r);
+        uint32_t r[16];
+        const uint32_t ta = tmem + frag + T_O + cc;
+        tmem_ld_16x256b_x4(ta, r);
         tc_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) r[j] = f2u(u2f(r[j]) * a);
-        tmem_st32(tmem + lane_base + T_O + cc, r);
+        for (int j = 0; j < 4; ++j) {
+          r[4 * j] = f2u(u2f(r[4 * j]) * a0);
+          r[4 * j + 1] = f2u(u2f(r[4 * j + 1]) * a0);
+          r[4 * j + 2] = f2u(u2f(r[4 * j + 2]) * a1);
+          r[4 * j + 3] = f2u(u2f(r[4 * j + 3]) * a1);
+        }
+        tmem_st_16x256b_x4(ta, r);
       }
       tc_wait_st();
     };
-    // epilogue of a segment: this thread's row of this CTA's half of O~ / l
-    // into the row's output (a row held by one cluster) or the segment's slot
-    auto flush = [&](int i_last, int bb, float l, float m, bool write_lse) -> bool {
+    float m0 = -INFINITY, m1 = -INFINITY;  // running maxima of the two rows (log2 units)
+    float l0 = 0.f, l1 = 0.f;              // this thread's parts of their row sums
+    // epilogue of a segment: this thread's rows of this CTA's half of O~ / l
+    // into the row's output (a row held by one cluster) or the segment's slot,
+    // and (rank 0) the segment's log-sum-exps
+    auto flush = [&](int i_last, int bb) -> bool {
+      float t0 = l0 + __shfl_xor_sync(0xffffffffu, l0, 1);
+      t0 += __shfl_xor_sync(0xffffffffu, t0, 2);
+      float t1 = l1 + __shfl_xor_sync(0xffffffffu, l1, 1);
+      t1 += __shfl_xor_sync(0xffffffffu, t1, 2);
       if (!wait_pv(i_last)) return false;
       const int cf = p.sch.c_first(bb);
       const int used = p.sch.c_last(bb) - cf + 1;  // clusters holding a segment of row bb
       const int slot = cid - cf;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* dst = (used == 1 ? p.omerged + ((size_t)bb * kH + h) * kC
-                                      : p.opart + (((size_t)bb * p.slots + slot) * kH + h) * kC) +
-                           rank * 256;
+      const float inv0 = t0 > 0.f ? 1.f / t0 : 0.f;
+      const float inv1 = t1 > 0.f ? 1.f / t1 : 0.f;
+      __nv_bfloat16* dst0 =
+          (used == 1 ? p.omerged + ((size_t)bb * kH + row0) * kC
+                     : p.opart + (((size_t)bb * p.slots + slot) * kH + row0) * kC) +
+          rank * 256 + 2 * c4;
+      __nv_bfloat16* dst1 = dst0 + 8 * kC;
+      uint32_t r[16];
 #pragma unroll 1
       for (int cc = 0; cc < 256; cc += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_base + T_O + cc, r);
+        tmem_ld_16x256b_x4(tmem + frag + T_O + cc, r);
         tc_wait_ld();
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          uint4 o;
-          o.x = pack_bf16x2(u2f(r[8 * j]) * inv, u2f(r[8 * j + 1]) * inv);
-          o.y = pack_bf16x2(u2f(r[8 * j + 2]) * inv, u2f(r[8 * j + 3]) * inv);
-          o.z = pack_bf16x2(u2f(r[8 * j + 4]) * inv, u2f(r[8 * j + 5]) * inv);
-          o.w = pack_bf16x2(u2f(r[8 * j + 6]) * inv, u2f(r[8 * j + 7]) * inv);
-          *reinterpret_cast<uint4*>(dst + cc + 8 * j) = o;
+          *reinterpret_cast<uint32_t*>(dst0 + cc + 8 * j) =
+              pack_bf16x2(u2f(r[4 * j]) * inv0, u2f(r[4 * j + 1]) * inv0);
+          *reinterpret_cast<uint32_t*>(dst1 + cc + 8 * j) =
+              pack_bf16x2(u2f(r[4 * j + 2]) * inv1, u2f(r[4 * j + 3]) * inv1);
         }
       }
       tc_fence_before();
-      if (write_lse && used > 1)
-        p.lse[((size_t)bb * p.slots + slot) * kH + h] = l > 0.f ? m + log2f(l) : -INFINITY;
+      if (used > 1 && rank == 0 && c4 == 0) {
+        float* lse = p.lse + ((size_t)bb * p.slots + slot) * kH;
+        lse[row0] = t0 > 0.f ? m0 + log2f(t0) : -INFINITY;
+        lse[row1] = t1 > 0.f ? m1 + log2f(t1) : -INFINITY;
+      }
+      return true;
+    };
+    // own partial scores of tile t (score tile in TMEM) into x; when tile t
+    // is the last of its batch row and another follows, this warp's share of
+    // the next row's Q~ replaces the current one (the score product just read
+    // was the last that used it)
+    float x[32];
+    auto fetch = [&](int t, const Pos& ct) -> bool {
+      if (!warp_wait(&bars.s_full, t & 1, abort, p.status)) return false;
+      tc_fence_after();
+      uint32_t r[32];
+      tmem_ld_16x256b_x8(tmem + frag + T_S, r);
+      tc_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) x[j] = u2f(r[j]);
+      tc_fence_before();
+      __syncwarp();
+      // relaxed: the tcgen05 loads have completed (waited for above)
+      if (lane == 0) mbar_arrive_relaxed(&bars.s_empty);
+      if (ct.jt == nt - 1 && t + 1 < n) load_q(ct.bb + 1);
       return true;
     };
 
-    if (wg0) {
-      SHLA_REGS_INC;
-      pdl_wait();  // q~ is the fold kernel's output (the other roles read only inputs)
-      load_q(bb0);
-    } else {
-      SHLA_REGS_DEC;
-    }
+    pdl_wait();  // q~ is the fold kernel's output (the other roles read only inputs)
+    load_q(bb0);
     Pos c = {bb0, jt0};
     int prev_bb = bb0;
-    if (wg0 && !owned) {
-      // ---------------- sender of the peer's heads' partial scores ----------------
-      const uint32_t xs_peer = mapa_shared(sbase + OFF_XS + xs_off, peer);
+    int nx = 0;  // next tile whose exchange buffer is consumed
+    alive = fetch(0, c);
 #pragma unroll 1
-      for (int i = 0; i < n; ++i) {
-        const int b = i & 1;
-        if (!warp_wait(&bars.s_full[b], (i >> 1) & 1, abort, p.status)) { alive = false; break; }
-        tc_fence_after();
-        uint32_t s[64];
-        tmem_ld32(tmem + lane_base + T_S + b * KT, *reinterpret_cast<uint32_t(*)[32]>(s));
-        tmem_ld32(tmem + lane_base + T_S + b * KT + 32, *reinterpret_cast<uint32_t(*)[32]>(s + 32));
-        tc_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.s_free[b]);
-        // (the score tile just read was the last product that used this Q~)
-        if (c.jt == nt - 1 && i + 1 < n) load_q(c.bb + 1);
-        if (!warp_wait<true>(&bars.xs_free[b], ((i >> 1) & 1) ^ 1, abort, p.status)) { alive = false; break; }
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-          st_async_u4(xs_peer + b * XS_BYTES + k * 512, s[4 * k], s[4 * k + 1], s[4 * k + 2],
-                      s[4 * k + 3], xs_full_peer + b * 8);
-        c = next_pos(c);
+    for (int i = 0; i < n && alive; ++i) {
+      const int b = i & 1;
+      const bool first = i == 0 || c.jt == 0;
+      // a new segment: write out the previous one and restart the running state
+      if (first && i > 0) {
+        if (!flush(i - 1, prev_bb)) { alive = false; break; }
+        m0 = m1 = -INFINITY;
+        l0 = l1 = 0.f;
       }
-    } else if (wg0) {
-      // ---------------- softmax of this CTA's heads ----------------
-      const uint32_t xs_own = sbase + OFF_XS + xs_off;
-      float m_used = -INFINITY;  // running maximum of the row (log2 units)
-      float l = 0.f;             // running sum of the row
-      int nx = 0;                // next tile whose exchange buffer this warp consumes
-#pragma unroll 1
-      for (int i = 0; i < n; ++i) {
-        const int b = i & 1;
-        const bool first = i == 0 || c.jt == 0;
-        if (!warp_wait(&bars.s_full[b], (i >> 1) & 1, abort, p.status)) { alive = false; break; }
-        tc_fence_after();
-        float s[64];
-        {
-          uint32_t r[64];
-          tmem_ld32(tmem + lane_base + T_S + b * KT, *reinterpret_cast<uint32_t(*)[32]>(r));
-          tmem_ld32(tmem + lane_base + T_S + b * KT + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
-          tc_wait_ld();
+      // key biases of the tile (its stage stays in place until the tile's value product)
+      if (!warp_wait(&bars.full[i % NST], (i / NST) & 1, abort, p.status)) { alive = false; break; }
+      float2 bias[8];
 #pragma unroll
-          for (int j = 0; j < 64; ++j) s[j] = u2f(r[j]);
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.s_free[b]);
-        if (c.jt == nt - 1 && i + 1 < n) load_q(c.bb + 1);
-        // a new segment: write out the previous one and restart the running state
-        if (first && i > 0) {
-          if (!flush(i - 1, prev_bb, l, m_used, true)) { alive = false; break; }
-          m_used = -INFINITY;
-          l = 0.f;
-        }
-        // valid keys of the tile (its stage stays in place until the tile's value product)
-        if (!warp_wait(&bars.full[i % NST], (i / NST) & 1, abort, p.status)) { alive = false; break; }
-        const unsigned long long vmask = *reinterpret_cast<volatile unsigned long long*>(&bars.mask[i % NST]);
-        // the peer's partial scores of these rows (the other latent half)
-        if (!warp_wait<true>(&bars.xs_full[b], (i >> 1) & 1, abort, p.status)) { alive = false; break; }
-        nx = i + 1;
+      for (int j = 0; j < 8; ++j)
+        asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];"
+                     : "=f"(bias[j].x), "=f"(bias[j].y)
+                     : "r"(sbase + OFF_BIAS + (i % NST) * (KT * 4) + (8 * j + 2 * c4) * 4));
+      // the peer's partial scores of these rows (the other latent half): own + peer
+      if (!warp_wait<true>(&bars.xs_full[b], (i >> 1) & 1, abort, p.status)) { alive = false; break; }
+      nx = i + 1;
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const uint4 v = ld_shared_v4(xs_own + b * XS_BYTES + k * 512);
-          s[4 * k] += u2f(v.x);
-          s[4 * k + 1] += u2f(v.y);
-          s[4 * k + 2] += u2f(v.z);
-          s[4 * k + 3] += u2f(v.w);
-        }
-        __syncwarp();
-        if (lane == 0) {
-          // next use of this buffer (tile i + 2): expect the peer's bytes again,
-          // then let the peer write them
-          if (ql == 0 && i + 2 < n) mbar_arrive_expect_tx(&bars.xs_full[b], XS_TX);
-          mbar_arrive_cluster(xs_free_peer + b * 8);
-        }
-        // scale to log2 units, mask, tile maximum (fp32)
-        float mt = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          s[j] = ((vmask >> j) & 1ull) ? s[j] * p.scale_log2 : -INFINITY;
-          mt = fmaxf(mt, s[j]);
-        }
-        const bool resc = mt > m_used + kRescaleThreshold;
-        const float alpha = (resc && !first) ? fast_exp2(m_used - mt) : 1.f;
-        if (!first && __any_sync(0xffffffffu, resc)) {
-          // O~ must hold the value product of tile i - 1 before it is scaled
-          if (!wait_pv(i - 1)) { alive = false; break; }
-          rescale_o(alpha);
-        }
-        if (resc) {
-          l *= alpha;
-          m_used = mt;
-        }
-        // P buffer b was last read by both CTAs' value products of tile i - 2
-        if (i >= 2 && !warp_wait<true>(&bars.pv_both[b], ((i - 2) >> 1) & 1, abort, p.status)) {
-          alive = false;
-          break;
-        }
-        // P = 2^(s - m) in fp32, rounded to bf16 into both CTAs' P buffer b
-        const bool live = m_used != -INFINITY;
-        const uint32_t p_loc = sbase + OFF_P + b * PBUF;
-        const uint32_t p_rem = p_peer + b * PBUF;
-        float ls0 = 0.f, ls1 = 0.f;
-#pragma unroll
-        for (int j8 = 0; j8 < 8; ++j8) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float x0 = live ? fast_exp2(s[8 * j8 + 2 * e] - m_used) : 0.f;
-            const float x1 = live ? fast_exp2(s[8 * j8 + 2 * e + 1] - m_used) : 0.f;
-            ls0 += x0;
-            ls1 += x1;
-            w[e] = pack_bf16x2(x0, x1);
-          }
-          const uint32_t off = sw128_off(h, j8);
-          st_shared_v4(p_loc + off, w[0], w[1], w[2], w[3]);
-          st_async_u4(p_rem + off, w[0], w[1], w[2], w[3], pp_full_peer + b * 8);
-        }
-        l += ls0 + ls1;
-        st_async_u4(p_rem + P_BYTES + h * 16, f2u(alpha), f2u(l), f2u(m_used), 0u,
-                    pp_full_peer + b * 8);
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.p_own[b]);
-        prev_bb = c.bb;
-        c = next_pos(c);
+      for (int k = 0; k < 8; ++k) {
+        const uint4 v = ld_shared_v4(xs_own + b * XS_BYTES + k * 512);
+        x[4 * k] += u2f(v.x);
+        x[4 * k + 1] += u2f(v.y);
+        x[4 * k + 2] += u2f(v.z);
+        x[4 * k + 3] += u2f(v.w);
       }
-      if (__all_sync(0xffffffffu, alive) && !*abort) flush(n - 1, prev_bb, l, m_used, true);
-      // on an abort, partial scores the peer may still be sending land before
-      // the CTA can leave: the armed, unconsumed phases (bounded waits; none
-      // remain on the normal path)
-      for (int t = nx; t < n && t < nx + 2; ++t)
-        warp_wait<true>(&bars.xs_full[t & 1], (t >> 1) & 1, nullptr, nullptr);
-    } else {
-      // ---------------- receiver of the peer's P rows for these heads ----------------
-      float l_r = 0.f, m_r = -INFINITY;  // the owner's running state after the last tile
-      int nx = 0;
-#pragma unroll 1
-      for (int i = 0; i < n; ++i) {
-        const int b = i & 1;
-        const bool first = i == 0 || c.jt == 0;
-        if (first && i > 0) {
-          if (!flush(i - 1, prev_bb, l_r, m_r, false)) { alive = false; break; }
-        }
-        if (!warp_wait<true>(&bars.pp_full[b], (i >> 1) & 1, abort, p.status)) { alive = false; break; }
-        nx = i + 1;
-        const uint4 a = ld_shared_v4(sbase + OFF_P + b * PBUF + P_BYTES + h * 16);
-        // the P rows that landed are read next by the value product (async proxy)
-        fence_proxy_async_smem();
-        __syncwarp();
-        // next use of this buffer (tile i + 2): the peer writes it only after
-        // this CTA's value product of tile i, which waits for this warp
-        if (lane == 0 && ql == 0 && i + 2 < n) mbar_arrive_expect_tx(&bars.pp_full[b], PP_TX);
-        const float alpha = u2f(a.x);
-        if (!first && __any_sync(0xffffffffu, alpha != 1.f)) {
-          if (!wait_pv(i - 1)) { alive = false; break; }
-          rescale_o(alpha);
-        }
-        l_r = u2f(a.y);
-        m_r = u2f(a.z);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.peer_ok[b]);
-        prev_bb = c.bb;
-        c = next_pos(c);
+      __syncwarp();
+      if (lane == 0) {
+        // next use of this buffer (tile i + 2): expect the peer's bytes again,
+        // then let the peer write them.  The arrive is relaxed: the warp's
+        // reads of the buffer have completed (their values are consumed above)
+        if (warp == 0 && i + 2 < n) mbar_arrive_expect_tx_relaxed(&bars.xs_full[b], XS_TX);
+        mbar_arrive_cluster_relaxed(xs_free_peer + b * 8);
       }
-      if (__all_sync(0xffffffffu, alive) && !*abort) flush(n - 1, prev_bb, l_r, m_r, false);
-      for (int t = nx; t < n && t < nx + 2; ++t)
-        warp_wait<true>(&bars.pp_full[t & 1], (t >> 1) & 1, nullptr, nullptr);
+      // scale to log2 units, mask (fp32); row maxima
+      float mt0 = -INFINITY, mt1 = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        x[4 * j] = fmaf(x[4 * j], p.scale_log2, bias[j].x);
+        x[4 * j + 1] = fmaf(x[4 * j + 1], p.scale_log2, bias[j].y);
+        x[4 * j + 2] = fmaf(x[4 * j + 2], p.scale_log2, bias[j].x);
+        x[4 * j + 3] = fmaf(x[4 * j + 3], p.scale_log2, bias[j].y);
+        mt0 = fmaxf(mt0, fmaxf(x[4 * j], x[4 * j + 1]));
+        mt1 = fmaxf(mt1, fmaxf(x[4 * j + 2], x[4 * j + 3]));
+      }
+#pragma unroll
+      for (int o = 1; o < 4; o <<= 1) {
+        mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, o));
+        mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, o));
+      }
+      const bool resc0 = mt0 > m0 + kRescaleThreshold, resc1 = mt1 > m1 + kRescaleThreshold;
+      if (!first && __any_sync(0xffffffffu, resc0 || resc1)) {
+        // O~ must hold the value product of tile i - 1 before it is scaled
+        if (!wait_pv(i - 1)) { alive = false; break; }
+        rescale_o(resc0 ? fast_exp2(m0 - mt0) : 1.f, resc1 ? fast_exp2(m1 - mt1) : 1.f);
+      }
+      if (resc0) {
+        l0 *= first ? 0.f : fast_exp2(m0 - mt0);
+        m0 = mt0;
+      }
+      if (resc1) {
+        l1 *= first ? 0.f : fast_exp2(m1 - mt1);
+        m1 = mt1;
+      }
+      // P buffer b was last read by the value product of tile i - 2
+      if (i >= 2 && !wait_pv(i - 2)) { alive = false; break; }
+      // P = 2^(s - m) in fp32, rounded to bf16 pairs into TMEM buffer b (the
+      // pair of block j lands in P column 4j + c4 of its row)
+      {
+        const bool live0 = m0 != -INFINITY, live1 = m1 != -INFINITY;
+        uint32_t w[16];
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float e0 = live0 ? fast_exp2(x[4 * j] - m0) : 0.f;
+          const float e1 = live0 ? fast_exp2(x[4 * j + 1] - m0) : 0.f;
+          const float e2 = live1 ? fast_exp2(x[4 * j + 2] - m1) : 0.f;
+          const float e3 = live1 ? fast_exp2(x[4 * j + 3] - m1) : 0.f;
+          s0 += e0 + e1;
+          s1 += e2 + e3;
+          w[2 * j] = pack_bf16x2(e0, e1);
+          w[2 * j + 1] = pack_bf16x2(e2, e3);
+        }
+        l0 += s0;
+        l1 += s1;
+        tmem_st_16x128b_x8(tmem + frag + T_P + b * (KT / 2), w);
+      }
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.p_full[b]);
+      prev_bb = c.bb;
+      const Pos cn = next_pos(c);
+      if (i + 1 < n && !fetch(i + 1, cn)) { alive = false; break; }
+      c = cn;
     }
+    if (__all_sync(0xffffffffu, alive) && !*abort) flush(n - 1, prev_bb);
+    // on an abort, partial scores the peer may still be sending land before
+    // the CTA can leave: the armed, unconsumed phases (bounded waits; none
+    // remain on the normal path)
+    for (int t = nx; t < n && t < nx + 2; ++t)
+      warp_wait<true>(&bars.xs_full[t & 1], (t >> 1) & 1, nullptr, nullptr);
   }
 
   tc_fence_before();
@@ -858,8 +799,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
   }
   // neither CTA leaves while its peer may still touch its shared memory
   cluster_sync_all();
-#undef SHLA_REGS_DEC
-#undef SHLA_REGS_INC
 }
 
 // ===========================================================================
@@ -1056,13 +995,17 @@ static int ntiles_of(int k) { return (k + core::KT - 1) / core::KT; }
 // Clusters of the attend kernel that fit on the device at once (cached per
 // device); every cluster is persistent over its range of tiles.
 static int max_clusters() {
-  static int cached[64] = {0};
+  // two host threads that both find the entry empty store the same value
+  static std::atomic<int> cached[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
     cudaGetLastError();
     return 74;
   }
-  if (dev < 64 && cached[dev] > 0) return cached[dev];
+  if (dev < 64) {
+    const int c = cached[dev].load(std::memory_order_acquire);
+    if (c > 0) return c;
+  }
   int n = 0;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -1086,7 +1029,7 @@ static int max_clusters() {
     }
     n = sms / 2;
   }
-  if (dev < 64) cached[dev] = n;
+  if (dev < 64) cached[dev].store(n, std::memory_order_release);
   return n;
 }
 
@@ -1126,7 +1069,7 @@ template <int NB>
 static int launch_fold_nb(const __nv_bfloat16* q_nope, const __nv_bfloat16* wkv_b,
                           __nv_bfloat16* q_tilde, int B, int32_t* status, cudaStream_t st) {
   const int smem = 32768 + NB * 256 + 1024;
-  static unsigned long long attr_done = 0;
+  static std::atomic<unsigned long long> attr_done{0};
   if (int e = ensure_smem_attr(fold_kernel<NB>, smem, &attr_done)) return e;
   dim3 grid(4, kH, (B + NB - 1) / NB);
   fold_kernel<NB><<<grid, 128, smem, st>>>(q_nope, wkv_b, q_tilde, B, status);
@@ -1146,7 +1089,7 @@ template <int NB>
 static int launch_uv_nb(const __nv_bfloat16* wkv_b, const __nv_bfloat16* omerged, int B,
                         __nv_bfloat16* O, int32_t* status, cudaStream_t st, bool pdl) {
   const int smem = 2 * (32768 + NB * 256) + 1024;
-  static unsigned long long attr_done = 0;
+  static std::atomic<unsigned long long> attr_done{0};
   if (int e = ensure_smem_attr(uv_kernel<NB>, smem, &attr_done)) return e;
   dim3 grid(kH, (B + NB - 1) / NB);
   if (pdl) return launch_pdl(uv_kernel<NB>, grid, dim3(128), smem, st, wkv_b, omerged, B, O, status);
@@ -1181,15 +1124,17 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 static EncodeTiledFn encode_tiled() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
+  // looked up once (a function-local static is initialised thread-safely)
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
     void* f = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(f);
-  }
+      return reinterpret_cast<EncodeTiledFn>(f);
+    cudaGetLastError();
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -1290,10 +1235,6 @@ static int decode_impl(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_
   core::Params p;
   p.q_tilde = q_tilde;
   p.q_pe = reinterpret_cast<const __nv_bfloat16*>(q_pe);
-  p.ckv = reinterpret_cast<const __nv_bfloat16*>(c_kv);
-  p.kpe = reinterpret_cast<const __nv_bfloat16*>(k_pe);
-  p.ckv_rs = ckv_rstride;
-  p.kpe_rs = kpe_rstride;
   p.rows_per_b = ckv_bstride / ckv_rstride;
   p.q_per_row = q_per_row;
   p.T = T;
@@ -1316,7 +1257,7 @@ static int decode_impl(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_
       return e;
     if (int e = make_row_map(&map_r, k_pe, kR, rows, kpe_rstride, 32, CU_TENSOR_MAP_SWIZZLE_64B))
       return e;
-    static unsigned long long core_attr = 0;
+    static std::atomic<unsigned long long> core_attr{0};
     if (int e = ensure_smem_attr(core_kernel, core::SMEM_BYTES, &core_attr)) return e;
     // In the full call the fold precedes it: programmatic serialisation lets
     // its set-up and first gathers (which read only the caller's inputs)

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/shla.h"
 
 namespace shla {
@@ -34,15 +36,17 @@ inline int launch_status() {
 }
 
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device).
+// Safe to call from several host threads at once: the mask is atomic, and two
+// threads that both find the bit clear both set the same attribute value.
 template <typename F>
-inline int ensure_smem_attr(F* fn, int bytes, unsigned long long* done_mask) {
+inline int ensure_smem_attr(F* fn, int bytes, std::atomic<unsigned long long>* done_mask) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
   const unsigned long long bit = 1ull << (dev & 63);
-  if (*done_mask & bit) return MLA_OK;
+  if (done_mask->load(std::memory_order_acquire) & bit) return MLA_OK;
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
     return MLA_ERR_CUDA;
-  *done_mask |= bit;
+  done_mask->fetch_or(bit, std::memory_order_acq_rel);
   return MLA_OK;
 }
 

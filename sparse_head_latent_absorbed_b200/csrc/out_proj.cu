@@ -277,15 +277,17 @@ typedef CUresult (*XwtEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, v
                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 static XwtEncodeFn xwt_encode() {
-  static XwtEncodeFn fn = nullptr;
-  if (!fn) {
+  // looked up once (a function-local static is initialised thread-safely)
+  static const XwtEncodeFn fn = []() -> XwtEncodeFn {
     void* f = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<XwtEncodeFn>(f);
-  }
+      return reinterpret_cast<XwtEncodeFn>(f);
+    cudaGetLastError();
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -327,7 +329,7 @@ int xwt_gemm(const void* w, int n_out, int k_in, const void* x, int B, float* pa
   alignas(64) CUtensorMap map_w, map_x;
   if (int e = xwt_map(&map_w, w, n_out, k_in, 128)) return e;
   if (int e = xwt_map(&map_x, x, B, k_in, rows)) return e;
-  static unsigned long long attr_done = 0;
+  static std::atomic<unsigned long long> attr_done{0};
   if (int e = ensure_smem_attr(xwt_kernel, xwt::SMEM_BYTES, &attr_done)) return e;
   const dim3 grid(plan.nc, (B + 127) / 128);
   if (pdl)
