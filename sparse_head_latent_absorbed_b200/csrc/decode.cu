@@ -148,16 +148,21 @@ __global__ void __launch_bounds__(128) fold_kernel(const __nv_bfloat16* __restri
 //   keys to -inf and run the same fp32 online softmax, bit for bit (running
 //   maximum m, raised lazily once the tile maximum exceeds it by more than 8;
 //   P = 2^(s - m) rounded to bf16; row sum l of the fp32 P), so nothing else
-//   crosses between them
+//   crosses between them.  The exchange runs in its own warps, a tile ahead
+//   of the softmax: they free the score tile as soon as they have read it, so
+//   the next score product overlaps the softmax of this one.
 //   O_r += P V_r             M=128, N=256, K=KT, A = P from TMEM
 // V is the same shared-memory tile as K, read MN-major.
 //
 // Warp roles (640 threads):
 //   warps 0-7   softmax: warp w takes the 16 rows [32q + 16h, +16) of lane
 //               quarter q = w % 4, h = w / 4, and all keys of a tile, four
-//               threads per row (16x256b TMEM fragments).  They also load
-//               Q~ at each segment start.
-//   warps 8-11  send the partial scores of lane quarter w - 8 to the peer
+//               threads per row (the 16x256b TMEM fragment order), reading
+//               the tile's full scores from shared memory
+//   warps 8-11  exchange, for lane quarter q = w - 8: read the partial
+//               scores from TMEM, send them to the peer, add the peer's and
+//               store the full scores for the softmax warps; load this CTA's
+//               half of Q~ for the quarter's rows at each segment start
 //   warps 12-18 gather: TMA tile::gather4 of the selected rows
 //   warp 19     TMEM owner and MMA issuer (one thread)
 // TMEM (512 columns): latent half of Q~ [0,128) as bf16 pairs, the score
@@ -181,18 +186,19 @@ constexpr int ST_KR = 4 * ST_ATOM;           // rotary part of a tile (64 B swiz
 constexpr int ST_BYTES = ST_KR + KT * 64;    // 36864
 constexpr int OFF_ST = 0;
 constexpr int OFF_QR = OFF_ST + NST * ST_BYTES;  // rotary half of Q: 128 rows x 64 B, 64 B swizzle
-constexpr int OFF_XS = OFF_QR + 128 * 64;        // the peer's partial scores, two buffers
+constexpr int OFF_XS = OFF_QR + 128 * 64;        // the peer's partial scores of a tile
 constexpr int XS_BYTES = NSOFT * 8 * 32 * 16;    // [softmax warp][8 chunks][32 lanes][16 B]
-constexpr int OFF_BIAS = OFF_XS + 2 * XS_BYTES;  // per stage: 0 / -inf per key
+constexpr int OFF_FS = OFF_XS + XS_BYTES;        // full scores of a tile, the same layout
+constexpr int OFF_BIAS = OFF_FS + XS_BYTES;      // per stage: 0 / -inf per key
 constexpr int OFF_END = OFF_BIAS + NST * KT * 4;
 constexpr int SMEM_BYTES = OFF_END + 1024;       // + alignment slack
 constexpr uint32_t XS_TX = XS_BYTES;             // partial scores received per tile
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t T_Q = 0, T_S = 128, T_P = 192, T_O = 256;
 constexpr float kRescaleThreshold = 8.0f;        // log2 units
-// register split (the launch gives 96 per thread): softmax 112, senders 96,
-// gather / MMA 80: 2 x 112 + 96 + 2 x 80 = 5 x 96
-constexpr int REGS_SOFT = 112, REGS_SEND = 96, REGS_REST = 80;
+// register split (the launch gives 96 per thread): softmax 96, exchange 128,
+// gather / MMA 80: 2 x 96 + 128 + 2 x 80 = 5 x 96
+constexpr int REGS_SOFT = 96, REGS_SEND = 128, REGS_REST = 80;
 static_assert(128 * (2 * REGS_SOFT + REGS_SEND + 2 * REGS_REST) <= NTHREADS * 96, "register split");
 static_assert(ST_BYTES % 1024 == 0 && OFF_QR % 1024 == 0 && OFF_XS % 16 == 0, "alignment");
 static_assert(SMEM_BYTES + 512 <= 232448, "shared memory budget");
@@ -235,8 +241,9 @@ struct Params {
 
 struct Bars {
   uint64_t full[NST], empty[NST];  // gather ring
-  uint64_t s_full, s_empty;        // score tile in TMEM / read by the softmax and send warps
-  uint64_t xs_full[2], xs_free[2]; // peer's partial scores landed / this CTA's buffer read by the peer
+  uint64_t s_full, s_empty;        // score tile in TMEM / read by the exchange warps
+  uint64_t xs_full, xs_free;       // peer's partial scores landed / this CTA's buffer read by the peer
+  uint64_t f_full, f_free;         // full scores of a tile stored / read by the softmax warps
   uint64_t p_full[2];              // P of tile t is in TMEM buffer t & 1
   uint64_t o_done[2];              // the value product of tile t has completed
   uint64_t q_ready;                // the segment's Q~ is in TMEM / shared memory
@@ -328,18 +335,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       mbar_init(&bars.empty[s], 1);       // MMA commit after the tile's value product
     }
     mbar_init(&bars.s_full, 1);
-    mbar_init(&bars.s_empty, NSOFT + 4);
+    mbar_init(&bars.s_empty, 4);
+    mbar_init(&bars.xs_full, 1);     // own expect_tx arrival + the peer's st.async bytes
+    mbar_init(&bars.xs_free, 4);     // one arrival per exchange warp of the peer
+    mbar_init(&bars.f_full, 4);
+    mbar_init(&bars.f_free, NSOFT);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.xs_full[i], 1);     // own expect_tx arrival + the peer's st.async bytes
-      mbar_init(&bars.xs_free[i], NSOFT); // one arrival per softmax warp of the peer
       mbar_init(&bars.p_full[i], NSOFT);
       mbar_init(&bars.o_done[i], 1);
     }
-    mbar_init(&bars.q_ready, NSOFT);
+    mbar_init(&bars.q_ready, 4);
     mbar_init(&bars.drain, 1);
     bars.abort = 0;
     fence_mbarrier_init_cluster();
-    for (int i = 0; i < 2 && i < n; ++i) mbar_arrive_expect_tx(&bars.xs_full[i], XS_TX);
+    mbar_arrive_expect_tx(&bars.xs_full, XS_TX);
   }
   tc_fence_before();
   cluster_sync_all();
@@ -510,61 +519,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     }
     __syncwarp();
   } else if (warp >= SEND_WARP0) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_SEND));
-    // ---------------- send this quarter's partial scores to the peer ----------------
-    // fragments of both 16-lane halves of the quarter, in the register order
-    // of the peer's softmax warps for those rows
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SEND));
+    // ---------------- exchange for lane quarter q ----------------
+    // The two 16-lane halves of the quarter, in the 16x256b fragment order of
+    // the softmax warps q (half 0) and q + 4 (half 1): register 4k+e of half
+    // hf is chunk k of softmax warp q + 4 hf.
     const int q4 = warp - SEND_WARP0;
     const uint32_t xs_peer = mapa_shared(sbase + OFF_XS + lane * 16, peer);
-    const uint32_t xs_full_peer = mapa_shared(smem_u32(&bars.xs_full[0]), peer);
-#pragma unroll 1
-    for (int i = 0; i < n; ++i) {
-      const int b = i & 1;
-      if (!warp_wait(&bars.s_full, i & 1, abort, p.status)) break;
-      tc_fence_after();
-      uint32_t r0[32], r1[32];
-      tmem_ld_16x256b_x8(tmem + ((uint32_t)(q4 * 32) << 16) + T_S, r0);
-      tmem_ld_16x256b_x8(tmem + ((uint32_t)(q4 * 32 + 16) << 16) + T_S, r1);
-      tc_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      // relaxed: the tcgen05 loads have completed (waited for above)
-      if (lane == 0) mbar_arrive_relaxed(&bars.s_empty);
-      if (!warp_wait<true>(&bars.xs_free[b], ((i >> 1) & 1) ^ 1, abort, p.status)) break;
-      const uint32_t dst = xs_peer + b * XS_BYTES;
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        st_async_u4(dst + q4 * 4096 + k * 512, r0[4 * k], r0[4 * k + 1], r0[4 * k + 2],
-                    r0[4 * k + 3], xs_full_peer + b * 8);
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        st_async_u4(dst + (q4 + 4) * 4096 + k * 512, r1[4 * k], r1[4 * k + 1], r1[4 * k + 2],
-                    r1[4 * k + 3], xs_full_peer + b * 8);
-    }
-  } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFT));
-    // ---------------- softmax: rows [32q + 16h, +16), all keys ----------------
-    // Through the 16x256b TMEM shape thread t holds rows t/4 and t/4 + 8 of
-    // its 16 and, of each 8-key block j, keys 8j + 2(t%4) and 8j + 2(t%4) + 1:
-    // register 4j+e is (row t/4 + 8 (e/2), key 8j + 2(t%4) + e%2).
-    const int q4 = warp & 3, hf = warp >> 2;
-    const int c4 = lane & 3;
-    const int row0 = q4 * 32 + hf * 16 + (lane >> 2), row1 = row0 + 8;
-    const uint32_t frag = (uint32_t)(q4 * 32 + hf * 16) << 16;
-    const uint32_t xs_own = sbase + OFF_XS + warp * 4096 + lane * 16;
-    const uint32_t xs_free_peer = mapa_shared(smem_u32(&bars.xs_free[0]), peer);
-    bool alive = true;
-
-    // this warp's share of this CTA's half of Q~ for batch row bb (32x32b
-    // shape, one row per thread): latent values [128 hf, +128) of the CTA's
-    // 256 into TMEM as bf16 pairs, rotary values [16 hf, +16) of its 32 into
-    // the swizzled shared tile; then q_ready
+    const uint32_t xs_full_peer = mapa_shared(smem_u32(&bars.xs_full), peer);
+    const uint32_t xs_free_peer = mapa_shared(smem_u32(&bars.xs_free), peer);
+    const uint32_t own_xs = sbase + OFF_XS + lane * 16;
+    const uint32_t own_fs = sbase + OFF_FS + lane * 16;
+    // the quarter's 32 rows of this CTA's half of Q~ for batch row bb (32x32b
+    // shape, one row per thread): latent values into TMEM as bf16 pairs,
+    // rotary values into the swizzled shared tile; then q_ready
     auto load_q = [&](int bb) {
       const int h = q4 * 32 + lane;
       const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-      const __nv_bfloat16* qrow = p.q_tilde + ((size_t)bb * kH + h) * kC + rank * 256 + hf * 128;
+      const __nv_bfloat16* qrow = p.q_tilde + ((size_t)bb * kH + h) * kC + rank * 256;
 #pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < 4; ++c) {
         uint4 v[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = ld_global_nc_v4(qrow + c * 64 + i * 8);
@@ -576,13 +550,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
           r[4 * i + 2] = v[i].z;
           r[4 * i + 3] = v[i].w;
         }
-        tmem_st32(tmem + lane_base + T_Q + hf * 64 + c * 32, r);
+        tmem_st32(tmem + lane_base + T_Q + c * 32, r);
       }
-      const __nv_bfloat16* rrow = p.q_pe + ((size_t)bb * kH + h) * kR + rank * 32 + hf * 16;
+      const __nv_bfloat16* rrow = p.q_pe + ((size_t)bb * kH + h) * kR + rank * 32;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < 4; ++c) {
         const uint4 v = ld_global_nc_v4(rrow + c * 8);
-        st_shared_v4(sbase + OFF_QR + sw64_off(h, 2 * hf + c), v.x, v.y, v.z, v.w);
+        st_shared_v4(sbase + OFF_QR + sw64_off(h, c), v.x, v.y, v.z, v.w);
       }
       fence_proxy_async_smem();
       tc_wait_st();
@@ -590,6 +564,90 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.q_ready);
     };
+    pdl_wait();  // q~ is the fold kernel's output (the other roles read only inputs)
+    load_q(bb0);
+    Pos c = {bb0, jt0};
+    int nx = 0;  // next tile whose exchange buffer is consumed
+#pragma unroll 1
+    for (int i = 0; i < n; ++i) {
+      if (!warp_wait(&bars.s_full, i & 1, abort, p.status)) break;
+      tc_fence_after();
+      // the score tile just finished was the last product that used this
+      // segment's Q~ when the tile ends its batch row
+      if (c.jt == nt - 1 && i + 1 < n) load_q(c.bb + 1);
+      uint32_t r[2][32];
+      tmem_ld_16x256b_x8(tmem + ((uint32_t)(q4 * 32) << 16) + T_S, r[0]);
+      tmem_ld_16x256b_x8(tmem + ((uint32_t)(q4 * 32 + 16) << 16) + T_S, r[1]);
+      tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      // relaxed: the tcgen05 loads have completed (waited for above)
+      if (lane == 0) mbar_arrive_relaxed(&bars.s_empty);
+      // this CTA's partial scores to the peer (its buffer of tile i - 1 read)
+      if (!warp_wait<true>(&bars.xs_free, (i & 1) ^ 1, abort, p.status)) break;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          st_async_u4(xs_peer + (q4 + 4 * hf) * 4096 + k * 512, r[hf][4 * k], r[hf][4 * k + 1],
+                      r[hf][4 * k + 2], r[hf][4 * k + 3], xs_full_peer);
+      // own + peer, in fp32
+      if (!warp_wait<true>(&bars.xs_full, i & 1, abort, p.status)) break;
+      nx = i + 1;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint4 v = ld_shared_v4(own_xs + (q4 + 4 * hf) * 4096 + k * 512);
+          r[hf][4 * k] = f2u(u2f(r[hf][4 * k]) + u2f(v.x));
+          r[hf][4 * k + 1] = f2u(u2f(r[hf][4 * k + 1]) + u2f(v.y));
+          r[hf][4 * k + 2] = f2u(u2f(r[hf][4 * k + 2]) + u2f(v.z));
+          r[hf][4 * k + 3] = f2u(u2f(r[hf][4 * k + 3]) + u2f(v.w));
+        }
+      // the sums are computed (so the buffer's loads have returned) before
+      // the relaxed arrive below is issued
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+        for (int j = 0; j < 32; ++j) asm volatile("" : "+r"(r[hf][j]));
+      __syncwarp();
+      if (lane == 0) {
+        // next use of the buffer (tile i + 1): expect the peer's bytes again,
+        // then let the peer write them.  Relaxed: the reads have completed
+        // (their values are consumed above), and a release would also wait
+        // for the remote stores just issued.
+        if (q4 == 0 && i + 1 < n) mbar_arrive_expect_tx_relaxed(&bars.xs_full, XS_TX);
+        mbar_arrive_cluster_relaxed(xs_free_peer);
+      }
+      // the full scores for the softmax warps (their buffer of tile i - 1 read)
+      if (!warp_wait(&bars.f_free, (i & 1) ^ 1, abort, p.status)) break;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          st_shared_v4(own_fs + (q4 + 4 * hf) * 4096 + k * 512, r[hf][4 * k], r[hf][4 * k + 1],
+                       r[hf][4 * k + 2], r[hf][4 * k + 3]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.f_full);
+      c = next_pos(c);
+    }
+    // on an abort, partial scores the peer may still be sending land before
+    // the CTA can leave: the armed, unconsumed phase (bounded wait; none
+    // remains on the normal path)
+    if (nx < n) warp_wait<true>(&bars.xs_full, nx & 1, nullptr, nullptr);
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFT));
+    // ---------------- softmax: rows [32q + 16h, +16), all keys ----------------
+    // Through the 16x256b TMEM shape thread t holds rows t/4 and t/4 + 8 of
+    // its 16 and, of each 8-key block j, keys 8j + 2(t%4) and 8j + 2(t%4) + 1:
+    // register 4j+e is (row t/4 + 8 (e/2), key 8j + 2(t%4) + e%2).
+    const int q4 = warp & 3, hf = warp >> 2;
+    const int c4 = lane & 3;
+    const int row0 = q4 * 32 + hf * 16 + (lane >> 2), row1 = row0 + 8;
+    const uint32_t frag = (uint32_t)(q4 * 32 + hf * 16) << 16;
+    const uint32_t fs_own = sbase + OFF_FS + warp * 4096 + lane * 16;
+    bool alive = true;
+
     // the value product of tile t has completed
     auto wait_pv = [&](int t) -> bool {
       if (!warp_wait(&bars.o_done[t & 1], (t >> 1) & 1, abort, p.status)) return false;
@@ -657,33 +715,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       }
       return true;
     };
-    // own partial scores of tile t (score tile in TMEM) into x; when tile t
-    // is the last of its batch row and another follows, this warp's share of
-    // the next row's Q~ replaces the current one (the score product just read
-    // was the last that used it)
     float x[32];
-    auto fetch = [&](int t, const Pos& ct) -> bool {
-      if (!warp_wait(&bars.s_full, t & 1, abort, p.status)) return false;
-      tc_fence_after();
-      uint32_t r[32];
-      tmem_ld_16x256b_x8(tmem + frag + T_S, r);
-      tc_wait_ld();
-#pragma unroll
-      for (int j = 0; j < 32; ++j) x[j] = u2f(r[j]);
-      tc_fence_before();
-      __syncwarp();
-      // relaxed: the tcgen05 loads have completed (waited for above)
-      if (lane == 0) mbar_arrive_relaxed(&bars.s_empty);
-      if (ct.jt == nt - 1 && t + 1 < n) load_q(ct.bb + 1);
-      return true;
-    };
-
-    pdl_wait();  // q~ is the fold kernel's output (the other roles read only inputs)
-    load_q(bb0);
     Pos c = {bb0, jt0};
     int prev_bb = bb0;
-    int nx = 0;  // next tile whose exchange buffer is consumed
-    alive = fetch(0, c);
 #pragma unroll 1
     for (int i = 0; i < n && alive; ++i) {
       const int b = i & 1;
@@ -702,25 +736,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
         asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];"
                      : "=f"(bias[j].x), "=f"(bias[j].y)
                      : "r"(sbase + OFF_BIAS + (i % NST) * (KT * 4) + (8 * j + 2 * c4) * 4));
-      // the peer's partial scores of these rows (the other latent half): own + peer
-      if (!warp_wait<true>(&bars.xs_full[b], (i >> 1) & 1, abort, p.status)) { alive = false; break; }
-      nx = i + 1;
+      // the tile's full scores (exchange warps)
+      if (!warp_wait(&bars.f_full, i & 1, abort, p.status)) { alive = false; break; }
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const uint4 v = ld_shared_v4(xs_own + b * XS_BYTES + k * 512);
-        x[4 * k] += u2f(v.x);
-        x[4 * k + 1] += u2f(v.y);
-        x[4 * k + 2] += u2f(v.z);
-        x[4 * k + 3] += u2f(v.w);
+        const uint4 v = ld_shared_v4(fs_own + k * 512);
+        x[4 * k] = u2f(v.x);
+        x[4 * k + 1] = u2f(v.y);
+        x[4 * k + 2] = u2f(v.z);
+        x[4 * k + 3] = u2f(v.w);
       }
       __syncwarp();
-      if (lane == 0) {
-        // next use of this buffer (tile i + 2): expect the peer's bytes again,
-        // then let the peer write them.  The arrive is relaxed: the warp's
-        // reads of the buffer have completed (their values are consumed above)
-        if (warp == 0 && i + 2 < n) mbar_arrive_expect_tx_relaxed(&bars.xs_full[b], XS_TX);
-        mbar_arrive_cluster_relaxed(xs_free_peer + b * 8);
-      }
+      // release: the exchange warps overwrite the buffer as soon as this arrives
+      if (lane == 0) mbar_arrive(&bars.f_free);
       // scale to log2 units, mask (fp32); row maxima
       float mt0 = -INFINITY, mt1 = -INFINITY;
 #pragma unroll
@@ -779,16 +807,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.p_full[b]);
       prev_bb = c.bb;
-      const Pos cn = next_pos(c);
-      if (i + 1 < n && !fetch(i + 1, cn)) { alive = false; break; }
-      c = cn;
+      c = next_pos(c);
     }
     if (__all_sync(0xffffffffu, alive) && !*abort) flush(n - 1, prev_bb);
-    // on an abort, partial scores the peer may still be sending land before
-    // the CTA can leave: the armed, unconsumed phases (bounded waits; none
-    // remain on the normal path)
-    for (int t = nx; t < n && t < nx + 2; ++t)
-      warp_wait<true>(&bars.xs_full[t & 1], (t >> 1) & 1, nullptr, nullptr);
   }
 
   tc_fence_before();
