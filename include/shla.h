@@ -152,23 +152,35 @@ int mla_cache_write_noalloc(const mla_bf16_t* x, const mla_bf16_t* w_kva,
  *   A          = softmax_t(s)
  *   O~[b,h,:]  = sum_t A[b,h,t] c_KV[b,t,:]
  *   O[b,h,:]   = W_UV[h] O~[b,h,:]                W_UV[h] = wkv_b[h, 128:256, :]
- * The selected set of row b is the set of distinct entries of topk[b, :]
- * inside [0, min(end_pos[b], T)); -1 entries are padding.  Other entries are
- * ignored and counted in status[1].  A row with an empty set gets O = 0.
+ * The selected keys of row b are the entries of topk[b, :] inside
+ * [0, min(end_pos[b], T)); -1 entries are padding.  Other entries are
+ * ignored and counted in status[1].  A row with no valid entry gets O = 0.
+ * The pages' index mask is a set (a position listed twice is selected once);
+ * this call does not look for repeats: each valid entry is one key, so a
+ * position listed twice counts twice.  Callers pass distinct positions (an
+ * indexer's top-k does), and then the two agree.
  *   q_nope  bf16 [B, 128, 128]
  *   q_pe    bf16 [B, 128, 64]   (already rotated)
  *   wkv_b   bf16 [128, 256, 512] ([out, in] storage of the 512 -> 128*256 projection)
  *   c_kv, k_pe, strides, T: cache as in mla_cache_write (read only)
- *   topk    int32 [B, k]   entries of a row must be distinct (besides -1)
+ *   topk    int32 [B, k]   positions, in any order; distinct (see above)
  *   end_pos int32 [B]
  *   scale   softmax scale (192^-0.5 * mscale^2 in the model)
  *   O       bf16 [B, 128, 128]
  *   ws      device workspace of at least mla_decode_workspace_bytes(B, k) bytes,
  *           256-byte aligned; contents need not be initialised
  *   status  optional int32[2] (see top of file), may be NULL
- * Requires 1 <= B <= 65535 and 1 <= k <= 65536; scores, softmax and
- * accumulations are fp32; q~, the softmax weights and per-split partial
- * outputs are rounded to bf16 as tensor-core operands.
+ * Requires 1 <= B <= 65535 and 1 <= k <= 65536.
+ *
+ * Arithmetic: the scores are accumulated in fp32 by the tensor cores (each CTA
+ * of a pair over half of the 576 columns; the two fp32 partial sums are added
+ * in fp32), then scaled, masked, maximised, shifted by the running maximum
+ * and exponentiated in fp32; row sums, the output accumulator and the
+ * rescaling are fp32.  Rounded to bf16, as tensor-core operands: q~ (the
+ * fold's output), the softmax weights P = 2^(s - m) (at most 2^8: the running
+ * maximum is raised once a tile's maximum exceeds it by more than 8 log2
+ * units), and the per-split partial outputs that the merge reads.  O is
+ * rounded to bf16 once, at the end.
  *
  * The call enqueues three or four kernels on `stream`.  The first waits for
  * the stream's earlier work as usual.  The later ones use programmatic

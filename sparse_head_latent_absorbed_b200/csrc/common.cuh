@@ -315,6 +315,23 @@ DEV void tma_gather4(uint32_t dst, const CUtensorMap* map, int x, int y0, int y1
       : "memory");
 }
 
+// TMA tile loads (2-D / 3-D box at the given coordinates, innermost first)
+// into shared memory, completion counted in bytes on the CTA-local mbarrier
+DEV void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+DEV void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // arrive (once) on a CTA-local mbarrier when all previously issued tcgen05
 // operations of this thread have completed
 DEV void tc_commit(uint64_t* bar) {

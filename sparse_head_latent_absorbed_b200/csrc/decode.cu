@@ -31,21 +31,27 @@ DEV T* align1024(T* p) {
 // K1: fold W_UK into the queries.  D^T[c, b] = sum_d W_UK[h][d][c] q_nope[b][h][d]
 //   A = W_UK[h] tile (M = 128 latent columns, K = d), MN-major (c contiguous)
 //   B = q_nope rows  (N = batch rows,        K = d), K-major
-// grid (4 latent tiles, 128 heads, batch blocks of NB); 128 threads.
+// One CTA per (latent half, head, batch block of NB rows); 128 threads.  Both
+// operands arrive by TMA with the 128 B swizzle in one go: the CTA's half of
+// W_UK[h] (two M-tiles of 128 latent columns, 64 KB, each with its own
+// barrier so that the first products start while the second tile lands) and
+// its batch block of q_nope (two 64-wide atoms of d).  The epilogue of M-tile
+// 0 overlaps the products of M-tile 1.
 // ===========================================================================
 template <int NB>
-__global__ void __launch_bounds__(128) fold_kernel(const __nv_bfloat16* __restrict__ q_nope,
-                                                    const __nv_bfloat16* __restrict__ wkv_b,
+__global__ void __launch_bounds__(128) fold_kernel(const __grid_constant__ CUtensorMap map_w,
+                                                    const __grid_constant__ CUtensorMap map_q,
                                                     __nv_bfloat16* __restrict__ q_tilde, int B,
                                                     int32_t* status) {
-  constexpr uint32_t NCOLS = NB <= 32 ? 32 : NB;
+  constexpr uint32_t NCOLS = 2 * NB < 32 ? 32 : 2 * NB;  // two accumulators of NB columns
+  constexpr uint32_t W_TILE = 2 * 16384;                 // one M-tile: 2 atoms x 128 d x 128 B
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  const uint32_t sA = smem_u32(smem);          // [2 atoms][128 d][128 B]  = 32 KB
-  const uint32_t sB = sA + 32768;              // [2 katoms][NB rows][128 B]
-  __shared__ uint64_t bar;
+  const uint32_t sA = smem_u32(smem);    // [2 M-tiles][2 atoms][128 d][128 B]
+  const uint32_t sB = sA + 2 * W_TILE;   // [2 atoms][NB rows][128 B]
+  __shared__ uint64_t bar_q, bar_w[2], bar_mma[2];
   __shared__ uint32_t tmem_base;
-  const int ct = blockIdx.x, h = blockIdx.y, b0 = blockIdx.z * NB;
+  const int half = blockIdx.x, h = blockIdx.y, b0 = blockIdx.z * NB;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_trigger();  // the attend kernel may start its set-up and first gathers
 
@@ -54,72 +60,82 @@ __global__ void __launch_bounds__(128) fold_kernel(const __nv_bfloat16* __restri
     tmem_relinquish();
   }
   if (tid == 0) {
-    mbar_init(&bar, 1);
+    mbar_init(&bar_q, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_w[i], 1);
+      mbar_init(&bar_mma[i], 1);
+    }
     fence_mbarrier_init_cluster();
+    mbar_arrive_expect_tx(&bar_q, 2 * NB * 128);
+    for (int a = 0; a < 2; ++a)
+      tma_load_3d(sB + a * (NB * 128), &map_q, a * 64, h, b0, &bar_q);
+    for (int mt = 0; mt < 2; ++mt) {
+      mbar_arrive_expect_tx(&bar_w[mt], W_TILE);
+      for (int a = 0; a < 2; ++a)
+        tma_load_2d(sA + mt * W_TILE + a * 16384, &map_w, half * 256 + mt * 128 + a * 64, h * 256,
+                    &bar_w[mt]);
+    }
   }
-  for (int q = tid; q < 128 * 16; q += 128) {
-    const int d = q >> 4, ch = q & 15;
-    cp_async_16(sA + (ch >> 3) * 16384 + sw128_off(d, ch & 7),
-                wkv_b + ((size_t)h * 256 + d) * kC + ct * 128 + ch * 8, 16);
-  }
-  for (int q = tid; q < NB * 16; q += 128) {
-    const int n = q >> 4, ch = q & 15, b = b0 + n;
-    const bool in = b < B;
-    cp_async_16(sB + (ch >> 3) * (NB * 128) + sw128_off(n, ch & 7),
-                q_nope + ((size_t)(in ? b : 0) * kH + h) * kDn + ch * 8, in ? 16u : 0u);
-  }
-  cp_async_wait_all();
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
+  bool ok = true;
   if (tid == 0) {
     constexpr uint32_t idesc = idesc_bf16_f32(128, NB, 1, 0);
+    ok = mbar_wait(&bar_q, 0, nullptr, status);
+    for (int mt = 0; mt < 2 && ok; ++mt) {
+      ok = mbar_wait(&bar_w[mt], 0, nullptr, status);
+      if (!ok) break;
+      tc_fence_after();
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const uint64_t ad = smem_desc(sA + ks * 2048, 16384, 1024, kSwizzle128B);
-      const uint64_t bd =
-          smem_desc(sB + (ks >> 2) * (NB * 128) + (ks & 3) * 32, 16, 1024, kSwizzle128B);
-      tc_mma(tmem, ad, bd, idesc, ks > 0);
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint64_t ad = smem_desc(sA + mt * W_TILE + ks * 2048, 16384, 1024, kSwizzle128B);
+        const uint64_t bd =
+            smem_desc(sB + (ks >> 2) * (NB * 128) + (ks & 3) * 32, 16, 1024, kSwizzle128B);
+        tc_mma(tmem + mt * NB, ad, bd, idesc, ks > 0);
+      }
+      tc_commit(&bar_mma[mt]);
     }
-    tc_commit(&bar);
   }
-  __syncwarp();
-  const bool ok = warp_wait(&bar, 0, nullptr, status);
-  tc_fence_after();
-  // epilogue: D^T[c][b] through shared memory (reusing the operand area) as
-  // [b][128 c] bf16 rows, then 16-byte stores of q~[b][h][ct*128 ..]
-  const uint32_t stage = sA;
-  if (ok) {
-    const int cl = warp * 32 + lane;  // this thread's c within the tile
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;  // (only warp 0's lane 0 issued)
+  // epilogue per M-tile: D^T[c][b] through shared memory (the M-tile's own
+  // operand area, free once its products are done) as [b][128 c] bf16 rows,
+  // then 16-byte stores of q~[b][h][256 half + 128 mt ..]
 #pragma unroll 1
-    for (int n0 = 0; n0 < NB; n0 += 16) {
-      uint32_t r[16];
-      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + n0, r);
-      tc_wait_ld();
+  for (int mt = 0; mt < 2; ++mt) {
+    const bool done = warp_wait(&bar_mma[mt], 0, nullptr, status);
+    tc_fence_after();
+    const uint32_t stage = sA + mt * W_TILE;
+    if (done) {
+      const int cl = warp * 32 + lane;  // this thread's c within the tile
+#pragma unroll 1
+      for (int n0 = 0; n0 < NB; n0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + mt * NB + n0, r);
+        tc_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const __nv_bfloat16 v = __float2bfloat16_rn(__uint_as_float(r[j]));
-        asm volatile("st.shared.b16 [%0], %1;" ::"r"(stage + (n0 + j) * 256 + cl * 2),
-                     "h"(*reinterpret_cast<const unsigned short*>(&v))
-                     : "memory");
+        for (int j = 0; j < 16; ++j) {
+          const __nv_bfloat16 v = __float2bfloat16_rn(__uint_as_float(r[j]));
+          asm volatile("st.shared.b16 [%0], %1;" ::"r"(stage + (n0 + j) * 256 + cl * 2),
+                       "h"(*reinterpret_cast<const unsigned short*>(&v))
+                       : "memory");
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (done) {
+      for (int q = tid; q < NB * 16; q += 128) {
+        const int nn = q >> 4, ch = q & 15, b = b0 + nn;
+        if (b >= B) continue;
+        const uint4 v = ld_shared_v4(stage + nn * 256 + ch * 16);
+        *reinterpret_cast<uint4*>(q_tilde + ((size_t)b * kH + h) * kC + half * 256 + mt * 128 +
+                                  ch * 8) = v;
       }
     }
   }
-  tc_fence_before();
-  __syncthreads();
-  if (ok) {
-    for (int q = tid; q < NB * 16; q += 128) {
-      const int nn = q >> 4, ch = q & 15, b = b0 + nn;
-      if (b >= B) continue;
-      uint4 v;
-      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                   : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                   : "r"(stage + nn * 256 + ch * 16));
-      *reinterpret_cast<uint4*>(q_tilde + ((size_t)b * kH + h) * kC + ct * 128 + ch * 8) = v;
-    }
-  }
+  (void)ok;
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
@@ -1086,14 +1102,64 @@ static WsLayout ws_layout(int B, int slots) {
   return w;
 }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled() {
+  // looked up once (a function-local static is initialised thread-safely)
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<EncodeTiledFn>(f);
+    cudaGetLastError();
+    return nullptr;
+  }();
+  return fn;
+}
+
+// tensor map over a bf16 array: dims / byte strides from the innermost
+// dimension, box of `box` elements, 128 B swizzle
+static int make_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+                    const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return MLA_ERR_CUDA;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
+                        strides_bytes, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
 template <int NB>
 static int launch_fold_nb(const __nv_bfloat16* q_nope, const __nv_bfloat16* wkv_b,
                           __nv_bfloat16* q_tilde, int B, int32_t* status, cudaStream_t st) {
-  const int smem = 32768 + NB * 256 + 1024;
+  alignas(64) CUtensorMap map_w, map_q;
+  {
+    // wkv_b as [128 heads x 256 rows][512 latent]: a box is 128 d-rows of one
+    // head by 64 latent columns
+    const cuuint64_t dims[2] = {(cuuint64_t)kC, (cuuint64_t)kH * 256};
+    const cuuint64_t strides[1] = {(cuuint64_t)kC * 2};
+    const cuuint32_t box[2] = {64, 128};
+    if (int e = make_map(&map_w, wkv_b, 2, dims, strides, box)) return e;
+  }
+  {
+    // q_nope as [B][128 heads][128 d]: a box is 64 d of one head for NB rows
+    const cuuint64_t dims[3] = {(cuuint64_t)kDn, (cuuint64_t)kH, (cuuint64_t)B};
+    const cuuint64_t strides[2] = {(cuuint64_t)kDn * 2, (cuuint64_t)kH * kDn * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)NB};
+    if (int e = make_map(&map_q, q_nope, 3, dims, strides, box)) return e;
+  }
+  const int smem = 2 * 32768 + NB * 256 + 1024;
   static std::atomic<unsigned long long> attr_done{0};
   if (int e = ensure_smem_attr(fold_kernel<NB>, smem, &attr_done)) return e;
-  dim3 grid(4, kH, (B + NB - 1) / NB);
-  fold_kernel<NB><<<grid, 128, smem, st>>>(q_nope, wkv_b, q_tilde, B, status);
+  dim3 grid(2, kH, (B + NB - 1) / NB);
+  fold_kernel<NB><<<grid, 128, smem, st>>>(map_w, map_q, q_tilde, B, status);
   return launch_status();
 }
 
@@ -1102,8 +1168,7 @@ static int launch_fold(const __nv_bfloat16* q_nope, const __nv_bfloat16* wkv_b,
   if (B <= 16) return launch_fold_nb<16>(q_nope, wkv_b, q_tilde, B, status, st);
   if (B <= 32) return launch_fold_nb<32>(q_nope, wkv_b, q_tilde, B, status, st);
   if (B <= 64) return launch_fold_nb<64>(q_nope, wkv_b, q_tilde, B, status, st);
-  if (B <= 128) return launch_fold_nb<128>(q_nope, wkv_b, q_tilde, B, status, st);
-  return launch_fold_nb<256>(q_nope, wkv_b, q_tilde, B, status, st);
+  return launch_fold_nb<128>(q_nope, wkv_b, q_tilde, B, status, st);
 }
 
 template <int NB>
@@ -1139,26 +1204,6 @@ static core::Sched schedule_for(int B, int k) {
 
 // 2-D tensor map over cache rows: dims {cols, rows}, row pitch rstride
 // elements, box {box_cols, 1} (one row high, as tile::gather4 requires).
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_tiled() {
-  // looked up once (a function-local static is initialised thread-safely)
-  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      return reinterpret_cast<EncodeTiledFn>(f);
-    cudaGetLastError();
-    return nullptr;
-  }();
-  return fn;
-}
-
 static int make_row_map(CUtensorMap* map, const void* base, int cols, unsigned long long rows,
                         int rstride, int box_cols, CUtensorMapSwizzle swz) {
   EncodeTiledFn fn = encode_tiled();

@@ -285,3 +285,27 @@ def test_cache_write(shla, rows, S, norm_ones):
     assert np.all(np.abs(got - exact) <= np.abs(exact) * 2.0 ** -7 + 1e-4)
     untouched = torch.cat([cache[:, :start], cache[:, start + S:]], 1)
     assert torch.all(untouched == 3.0)
+
+
+def test_decode_repeated_entries_count_per_listing(shla):
+    """The decode call takes each valid top-k entry as one key and does not
+    look for repeats (the header says so).  With positions listed twice, its
+    output is the attention over the list with repeats (the oracle over the
+    repeated rows), not over the set (the oracle's reading of the pages'
+    scatter mask), which differs measurably."""
+    wl = mi.make_small(B=3, T=400, k=120, seed=21, dup=20, device="cuda")
+    out = shla.mla_decode(wl.q_nope, wl.q_pe, wl.wkv_b, wl.cache, wl.topk, wl.end_pos, wl.scale)
+    g = out.double().cpu().numpy()
+    as_set = _oracle_decode(wl)
+    cache = wl.cache.cpu()
+    for b in range(wl.B):
+        ep = int(wl.end_pos[b])
+        listed = [v for v in wl.topk[b].tolist() if 0 <= v < min(ep, wl.T)]
+        assert len(listed) > len(set(listed))  # the row really repeats positions
+        r = mi.f64(cache[b, listed])
+        n = len(listed)
+        as_list = orc.decode_absorbed(mi.f64(wl.q_nope[b:b + 1]), mi.f64(wl.q_pe[b:b + 1]),
+                                      mi.f64(wl.wkv_b), r[None, :, :512], r[None, :, 512:],
+                                      np.arange(n)[None], np.array([n]), wl.scale)[0]
+        _check_O(out[b:b + 1], as_list[None], f"row {b} with repeats")
+        assert _rel(g[b], as_set[b]) > 3 * _rel(g[b], as_list)
