@@ -77,12 +77,6 @@ DEV void mbar_arrive(uint64_t* bar) {
                : "memory");
 }
 
-// arrive on a barrier in another CTA of the cluster (address from mapa)
-DEV void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-
 // relaxed remote arrive: orders nothing; used only where every access it
 // must follow has already completed (loaded values consumed)
 DEV void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
@@ -196,22 +190,6 @@ DEV uint32_t mapa_shared(uint32_t local_addr, uint32_t rank) {
   return r;
 }
 
-// 16-byte store into another CTA's shared memory that counts its bytes
-// against that CTA's mbarrier (complete_tx); no fence needed on either side
-DEV void st_async_v4(uint32_t addr, float a, float b, float c, float d, uint32_t remote_bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::
-          "r"(addr),
-      "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
-      : "memory");
-}
-
-DEV void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
-
 // ---------------------------------------------------------------------------
 // async-proxy fences and cp.async
 // ---------------------------------------------------------------------------
@@ -227,12 +205,6 @@ DEV void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
                : "memory");
 }
 DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-// arrive on ``bar`` once all cp.async copies issued so far by this thread
-// have landed (counts as one of the barrier's expected arrivals)
-DEV void cp_async_arrive_noinc(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
 DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 DEV void cp_async_wait() {
@@ -270,19 +242,8 @@ DEV void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
       : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16; A is M x 16 bf16 in TMEM
-// (row m in lane m, elements 2c and 2c+1 packed in column c)
-DEV void tc_mma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// The two MMA forms above with the accumulate flag fixed at compile time
+// The MMA above with the accumulate flag fixed at compile time, and its form
+// with A in TMEM (row m in lane m, elements 2c and 2c+1 packed in column c)
 template <bool kAccumulate>
 DEV void tc_mma_c(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc) {
   asm volatile(
@@ -356,16 +317,6 @@ DEV void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 
-DEV void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15])
-      : "memory");
-}
-
 // 16 lanes x 256 bit shape, N repetitions along the columns: thread t holds,
 // for repetition j, (lane t/4, columns 8j + 2(t%4), +1) in registers 4j, 4j+1
 // and (lane t/4 + 8, the same columns) in registers 4j+2, 4j+3; the lane
@@ -413,21 +364,6 @@ DEV void tmem_st_16x128b_x8(uint32_t taddr, const uint32_t (&r)[16]) {
       : "memory");
 }
 
-// 32 lanes x 32 bit, 32 / 64 consecutive columns (thread i: lane quarter
-// base + i); loads complete at tc_wait_ld
-DEV void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-        "=r"(r[31])
-      : "r"(taddr));
-}
 DEV void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -438,17 +374,6 @@ DEV void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
       "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
       "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
       "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
-
-// arrive (once) on the mbarrier at the same shared-memory offset in every
-// CTA of ``cta_mask`` when all previously issued tcgen05 operations of this
-// thread have completed
-DEV void tc_commit_mc(uint64_t* bar, uint16_t cta_mask) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], %1;" ::"r"(smem_u32(bar)),
-      "h"(cta_mask)
       : "memory");
 }
 
@@ -463,6 +388,15 @@ DEV void st_async_u4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t
       : "memory");
 }
 
+// bring the 128-byte line holding p into L2 (no register result)
+DEV void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
+DEV uint32_t ld_shared_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
 DEV uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
@@ -470,8 +404,6 @@ DEV uint4 ld_shared_v4(uint32_t addr) {
                : "r"(addr));
   return v;
 }
-
-DEV void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 
 // ---------------------------------------------------------------------------
 // descriptors

@@ -6,10 +6,10 @@
 //                    (batch row, key tile) list: TMA gather of the selected
 //                    cache rows, S = Q~ K^T with the 128 heads as M, fp32
 //                    online softmax, O~ += P V.  CTA r of the pair holds latent
-//                    columns [256r, 256r+256) and rotary columns [32r, 32r+32)
-//                    and runs the softmax of half of the heads; partial scores
-//                    and P cross between the two through distributed shared
-//                    memory.
+//                    columns [256r, 256r+256) and rotary columns [32r, 32r+32);
+//                    the two exchange their fp32 partial scores through
+//                    distributed shared memory and both run the same softmax
+//                    over all heads.
 //   combine_kernel   log-sum-exp merge of the rows split across clusters
 //   uv_kernel        O = O~ W_UV^T per head on the merged O~ (tcgen05, value
 //                    dim as M, batch as N)
@@ -206,7 +206,8 @@ constexpr int OFF_XS = OFF_QR + 128 * 64;        // the peer's partial scores of
 constexpr int XS_BYTES = NSOFT * 8 * 32 * 16;    // [softmax warp][8 chunks][32 lanes][16 B]
 constexpr int OFF_FS = OFF_XS + XS_BYTES;        // full scores of a tile, the same layout
 constexpr int OFF_BIAS = OFF_FS + XS_BYTES;      // per stage: 0 / -inf per key
-constexpr int OFF_END = OFF_BIAS + NST * KT * 4;
+constexpr int OFF_ROWSTART = OFF_BIAS + NST * KT * 4;  // per stage: the tile starts its row
+constexpr int OFF_END = OFF_ROWSTART + NST * 4;
 constexpr int SMEM_BYTES = OFF_END + 1024;       // + alignment slack
 constexpr uint32_t XS_TX = XS_BYTES;             // partial scores received per tile
 constexpr uint32_t TMEM_COLS = 512;
@@ -222,19 +223,42 @@ static_assert(T_Q + 128 <= T_S && T_S + KT <= T_P && T_P + KT <= T_O && T_O + 25
               "TMEM plan");
 
 // Schedule: tiles [bnd(c), bnd(c+1)) of the flattened list belong to cluster c.
+// Uniform: every row has nt tiles and the ranges are equal.  Ragged: row b
+// has tstart[b + 1] - tstart[b] >= 1 tiles (its list up to the last tile that
+// holds an entry other than -1), and the range boundaries tb[] balance the
+// tiles plus a fixed cost per row (each row a cluster starts loads its
+// queries and writes its output), computed on the device.
 struct Sched {
-  int nt;    // tiles per batch row
-  int tot;   // B * nt
-  int nc;    // clusters
-  __host__ __device__ long long bnd(int c) const { return (long long)c * tot / nc; }
-  // first / last cluster whose range meets batch row b
+  int nt;                  // tiles per row (uniform)
+  int tot;                 // tiles in all (uniform)
+  int nc;                  // clusters (uniform: never more than tot)
+  const int32_t* tstart;   // ragged: first tile of each row, B + 1 entries; null: uniform
+  const int32_t* tb;       // ragged: first tile of each cluster's range, nc + 1 entries
+  __host__ __device__ long long bnd(int c) const {
+    return tb ? (long long)tb[c] : (long long)c * tot / nc;
+  }
+  __host__ __device__ long long row_start(int b) const {
+    return tstart ? (long long)tstart[b] : (long long)b * nt;
+  }
+  __device__ int row_tiles(int b) const { return tstart ? tstart[b + 1] - tstart[b] : nt; }
+  // uniform: first / last cluster whose range meets row b
   __host__ __device__ int c_first(int b) const {
-    return (int)(((long long)b * nt + 1) * nc + tot - 1) / tot - 1;
+    return (int)(((row_start(b) + 1) * nc + tot - 1) / tot) - 1;
   }
   __host__ __device__ int c_last(int b) const {
-    return (int)(((long long)(b + 1) * nt) * nc + tot - 1) / tot - 1;
+    return (int)((row_start(b + 1) * nc + tot - 1) / tot) - 1;
   }
+  // Partial-output slot (0 or 1) of cluster c for row b.  A cluster holds at
+  // most two segments that are not whole rows: its first (the row began at
+  // or before the range's start: slot 0) and its last (the row began inside
+  // the range and runs past its end: slot 1).
+  __host__ __device__ int slot(int c, int b) const { return row_start(b) > bnd(c) ? 1 : 0; }
 };
+// fixed cost of a row, in tiles, in the ragged schedule's balance: the
+// query load and output flush a row costs its cluster (measured on B200
+// prefill: 1 prompt x 4096 tokens and 4 x 1024, top-k 2048 and 512, the
+// total time is flat between 4 and 6 and rises on either side)
+constexpr int kRowCostTiles = 5;
 
 struct Params {
   const __nv_bfloat16* q_tilde;   // [B][128][512]
@@ -247,10 +271,10 @@ struct Params {
   const int32_t* end_pos;
   int B;
   Sched sch;
-  int slots;                      // partial-output slots per batch row
+  const int32_t* crow;            // ragged: the row that holds tile bnd(c), per cluster
   float scale_log2;               // softmax scale * log2(e)
-  __nv_bfloat16* opart;           // [B][slots][128][512], normalised per segment
-  float* lse;                     // [B][slots][128], log2 units of scaled scores
+  __nv_bfloat16* opart;           // [clusters][2 slots][128][512], normalised per segment
+  float* lse;                     // [clusters][2 slots][128], log2 units of scaled scores
   __nv_bfloat16* omerged;         // [B][128][512]: O~ of rows held by a single cluster
   int32_t* status;
 };
@@ -272,13 +296,14 @@ DEV bool key_valid(int v, int lim) { return v >= 0 && v < lim; }
 
 // Position of a tile in the flattened list, advanced one tile at a time
 // (no division in the loops): batch row, tile within the row, the row's
-// valid-position limit and the tile's indices (lane l: keys l and 32 + l).
+// tile count and valid-position limit, and the tile's indices (lane l: keys
+// l and 32 + l).
 struct TileCur {
-  int bb, jt, lim, ilo, ihi;
+  int bb, jt, nr, lim, ilo, ihi;
 };
-// The same position without the indices.
+// The same position without the limit and the indices.
 struct Pos {
-  int bb, jt;
+  int bb, jt, nr;
 };
 
 }  // namespace core
@@ -296,24 +321,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
   const uint32_t peer = rank ^ 1u;
   const int cid = blockIdx.x >> 1;
   const int t_begin = (int)p.sch.bnd(cid), t_end = (int)p.sch.bnd(cid + 1);
-  const int n = t_end - t_begin;  // tiles of this cluster (>= 1)
-  const int nt = p.sch.nt;
+  const int n = t_end - t_begin;  // tiles of this cluster (ragged rows: possibly none)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // the merge / W_UV kernels may be scheduled; they take an SM only once
   // this kernel's CTA has left it (it holds the whole register file)
   pdl_trigger();
   const uint32_t sbase = smem_u32(smem);
-  const int bb0 = t_begin / nt, jt0 = t_begin - bb0 * nt;  // row / tile-in-row of tile 0
+  // row / tile-in-row of tile 0
+  const int bb0 = p.sch.tstart ? ld_global_nc_s32_early(p.crow + cid) : t_begin / p.sch.nt;
+  const int jt0 = t_begin - (int)p.sch.row_start(bb0);
+  auto tiles_of = [&](int bb) { return bb < p.B ? p.sch.row_tiles(bb) : 1; };
   auto lim_of = [&](int bb) { return min(ld_global_nc_s32_early(p.end_pos + bb), p.T); };
   // the tile after `c` (indices and limit loaded, not yet consumed)
   auto advance = [&](const TileCur& c) {
     TileCur d;
     d.bb = c.bb;
     d.jt = c.jt + 1;
+    d.nr = c.nr;
     d.lim = c.lim;
-    if (d.jt == nt) {
+    if (d.jt == d.nr) {
       d.jt = 0;
       ++d.bb;
+      d.nr = tiles_of(d.bb);
       d.lim = d.bb < p.B ? lim_of(d.bb) : 0;
     }
     d.ilo = d.ihi = -1;
@@ -329,14 +358,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     TileCur c;
     c.bb = bb0;
     c.jt = jt0 - 1;  // advance() from the tile before
+    c.nr = tiles_of(bb0);
     c.lim = lim_of(bb0);
     c.ilo = c.ihi = -1;
     return advance(c);
   };
   auto next_pos = [&](Pos c) {
-    if (++c.jt == nt) {
+    if (++c.jt == c.nr) {
       c.jt = 0;
       ++c.bb;
+      c.nr = tiles_of(c.bb);
     }
     return c;
   };
@@ -371,7 +402,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
 
-  if (warp >= GATHER_WARP0 && warp < MMA_WARP) {
+  if (n == 0) {
+    // an empty range (ragged rows, fewer tiles than clusters): nothing to do
+  } else if (warp >= GATHER_WARP0 && warp < MMA_WARP) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_REST));
     // ---------------- gather (TMA tile::gather4) ----------------
     // lane l holds the index of key l and key 32 + l of the tile; lanes
@@ -395,6 +428,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       }
       const int ra = oka ? (int)(base + cur.ilo) : -1;
       const int rb = okb ? (int)(base + cur.ihi) : -1;
+      const bool row_start = cur.jt == 0;
       if (i + 1 < n) cur = advance(cur);
       if (!warp_wait(&bars.empty[s], ((i / NST) & 1) ^ 1, abort, p.status)) break;
       if (gw == 0) {
@@ -405,6 +439,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
         asm volatile("st.shared.f32 [%0], %1;" ::"r"(bias + (32 + lane) * 4),
                      "f"(okb ? 0.f : -INFINITY)
                      : "memory");
+        if (lane == 0)
+          asm volatile("st.shared.u32 [%0], %1;" ::"r"(sbase + OFF_ROWSTART + s * 4),
+                       "r"(i == 0 || row_start ? 1u : 0u)
+                       : "memory");
         __syncwarp();
       }
       if (lane == 0) mbar_arrive_expect_tx(&bars.full[s], ng * GROUP_TX_BYTES);
@@ -455,7 +493,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       const uint32_t lo_qr = desc_lo(sbase + OFF_QR, 16);        // rotary half of Q
       int qk = 0, pv = 0, idle = 0, qseg = -1;
       int qs = 0, qph = 0, ps = 0;  // stage of the next score product (and its phase), value product
-      int jq = jt0, jp = jt0;  // tile-in-row of the next score / value product
       uint64_t t_idle = 0;  // when the current idle stretch was first checked (0: not yet)
 #pragma unroll 1
       while (pv < n) {
@@ -465,7 +502,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
           const int s = ps;
           const uint32_t lo = desc_lo(sbase + OFF_ST + s * ST_BYTES, ST_ATOM);  // V, MN-major
           const uint32_t tp = tmem + T_P + (pv & 1) * (KT / 2);
-          const bool first = pv == 0 || jp == 0;
+          // the tile starts a segment: its row's first tile, or the range's
+          const bool first = ld_shared_u32(sbase + OFF_ROWSTART + s * 4) != 0;
           if (first)
             tc_mma_tmem_a_c<false>(tmem + T_O, tp, desc_join(lo, hi_k128), idesc_pv);
           else
@@ -478,12 +516,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
           tc_commit(&bars.empty[s]);
           ++pv;
           if (++ps == NST) ps = 0;
-          if (++jp == nt) jp = 0;
           did = true;
         }
         if (qk < n && mbar_test(&bars.full[qs], qph) &&
             (qk == 0 || mbar_test(&bars.s_empty, (qk - 1) & 1))) {
-          const int seg = (qk == 0 || jq == 0) ? qseg + 1 : qseg;
+          const int seg = ld_shared_u32(sbase + OFF_ROWSTART + qs * 4) ? qseg + 1 : qseg;
           if (seg == qseg || mbar_test(&bars.q_ready, seg & 1)) {
             qseg = seg;
             tc_fence_after();
@@ -506,7 +543,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
               qs = 0;
               qph ^= 1;
             }
-            if (++jq == nt) jq = 0;
             did = true;
           }
         }
@@ -553,20 +589,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       const int h = q4 * 32 + lane;
       const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
       const __nv_bfloat16* qrow = p.q_tilde + ((size_t)bb * kH + h) * kC + rank * 256;
+      // two rounds of 16 loads in flight per thread (the row's load is on
+      // the path to its first score product)
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint4 v[8];
+      for (int c = 0; c < 4; c += 2) {
+        uint4 v[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = ld_global_nc_v4(qrow + c * 64 + i * 8);
-        uint32_t r[32];
+        for (int i = 0; i < 16; ++i) v[i] = ld_global_nc_v4(qrow + c * 64 + i * 8);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          r[4 * i] = v[i].x;
-          r[4 * i + 1] = v[i].y;
-          r[4 * i + 2] = v[i].z;
-          r[4 * i + 3] = v[i].w;
+        for (int hc = 0; hc < 2; ++hc) {
+          uint32_t r[32];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            r[4 * i] = v[8 * hc + i].x;
+            r[4 * i + 1] = v[8 * hc + i].y;
+            r[4 * i + 2] = v[8 * hc + i].z;
+            r[4 * i + 3] = v[8 * hc + i].w;
+          }
+          tmem_st32(tmem + lane_base + T_Q + (c + hc) * 32, r);
         }
-        tmem_st32(tmem + lane_base + T_Q + c * 32, r);
       }
       const __nv_bfloat16* rrow = p.q_pe + ((size_t)bb * kH + h) * kR + rank * 32;
 #pragma unroll
@@ -580,17 +621,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.q_ready);
     };
+    // this thread's part of the next row's queries into L2, a row ahead of
+    // its load (the next row starts inside this cluster's range)
+    auto prefetch_q = [&](int i, const Pos& c) {
+      if (i + c.nr - c.jt >= n) return;
+      const int h = q4 * 32 + lane;
+      const __nv_bfloat16* qrow = p.q_tilde + ((size_t)(c.bb + 1) * kH + h) * kC + rank * 256;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) prefetch_l2(qrow + j * 64);
+      prefetch_l2(p.q_pe + ((size_t)(c.bb + 1) * kH + h) * kR + rank * 32);
+    };
     pdl_wait();  // q~ is the fold kernel's output (the other roles read only inputs)
     load_q(bb0);
-    Pos c = {bb0, jt0};
+    Pos c = {bb0, jt0, tiles_of(bb0)};
     int nx = 0;  // next tile whose exchange buffer is consumed
 #pragma unroll 1
     for (int i = 0; i < n; ++i) {
+      if (i == 0 || c.jt == 0) prefetch_q(i, c);
       if (!warp_wait(&bars.s_full, i & 1, abort, p.status)) break;
       tc_fence_after();
       // the score tile just finished was the last product that used this
       // segment's Q~ when the tile ends its batch row
-      if (c.jt == nt - 1 && i + 1 < n) load_q(c.bb + 1);
+      if (c.jt == c.nr - 1 && i + 1 < n) load_q(c.bb + 1);
       uint32_t r[2][32];
       tmem_ld_16x256b_x8(tmem + ((uint32_t)(q4 * 32) << 16) + T_S, r[0]);
       tmem_ld_16x256b_x8(tmem + ((uint32_t)(q4 * 32 + 16) << 16) + T_S, r[1]);
@@ -694,20 +746,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
     // epilogue of a segment: this thread's rows of this CTA's half of O~ / l
     // into the row's output (a row held by one cluster) or the segment's slot,
     // and (rank 0) the segment's log-sum-exps
-    auto flush = [&](int i_last, int bb) -> bool {
+    // `partial`: the segment is not its whole row (it began mid-row at the
+    // range's start, or its row runs past the range's end); such a segment
+    // goes to slot 0 of this cluster when it is the range's first, else to
+    // slot 1 (the rule of Sched::slot)
+    auto flush = [&](int i_last, int bb, bool partial, int slot1) -> bool {
       float t0 = l0 + __shfl_xor_sync(0xffffffffu, l0, 1);
       t0 += __shfl_xor_sync(0xffffffffu, t0, 2);
       float t1 = l1 + __shfl_xor_sync(0xffffffffu, l1, 1);
       t1 += __shfl_xor_sync(0xffffffffu, t1, 2);
       if (!wait_pv(i_last)) return false;
-      const int cf = p.sch.c_first(bb);
-      const int used = p.sch.c_last(bb) - cf + 1;  // clusters holding a segment of row bb
-      const int slot = cid - cf;
+      const int slot = 2 * cid + slot1;
       const float inv0 = t0 > 0.f ? 1.f / t0 : 0.f;
       const float inv1 = t1 > 0.f ? 1.f / t1 : 0.f;
       __nv_bfloat16* dst0 =
-          (used == 1 ? p.omerged + ((size_t)bb * kH + row0) * kC
-                     : p.opart + (((size_t)bb * p.slots + slot) * kH + row0) * kC) +
+          (!partial ? p.omerged + ((size_t)bb * kH + row0) * kC
+                    : p.opart + ((size_t)slot * kH + row0) * kC) +
           rank * 256 + 2 * c4;
       __nv_bfloat16* dst1 = dst0 + 8 * kC;
       uint32_t r[16];
@@ -724,23 +778,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
         }
       }
       tc_fence_before();
-      if (used > 1 && rank == 0 && c4 == 0) {
-        float* lse = p.lse + ((size_t)bb * p.slots + slot) * kH;
+      if (partial && rank == 0 && c4 == 0) {
+        float* lse = p.lse + (size_t)slot * kH;
         lse[row0] = t0 > 0.f ? m0 + log2f(t0) : -INFINITY;
         lse[row1] = t1 > 0.f ? m1 + log2f(t1) : -INFINITY;
       }
       return true;
     };
     float x[32];
-    Pos c = {bb0, jt0};
+    Pos c = {bb0, jt0, tiles_of(bb0)};
     int prev_bb = bb0;
+    bool open = false;  // the last tile processed is not its row's last
+    int nseg = 0;       // segments written out
 #pragma unroll 1
     for (int i = 0; i < n && alive; ++i) {
       const int b = i & 1;
       const bool first = i == 0 || c.jt == 0;
-      // a new segment: write out the previous one and restart the running state
+      // a new segment: write out the previous one (which ended its row) and
+      // restart the running state
       if (first && i > 0) {
-        if (!flush(i - 1, prev_bb)) { alive = false; break; }
+        if (!flush(i - 1, prev_bb, nseg == 0 && jt0 > 0, 0)) { alive = false; break; }
+        ++nseg;
         m0 = m1 = -INFINITY;
         l0 = l1 = 0.f;
       }
@@ -823,9 +881,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.p_full[b]);
       prev_bb = c.bb;
+      open = c.jt != c.nr - 1;
       c = next_pos(c);
     }
-    if (__all_sync(0xffffffffu, alive) && !*abort) flush(n - 1, prev_bb);
+    if (__all_sync(0xffffffffu, alive) && !*abort)
+      flush(n - 1, prev_bb, (nseg == 0 && jt0 > 0) || open, nseg == 0 ? 0 : 1);
   }
 
   tc_fence_before();
@@ -841,37 +901,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
 // ===========================================================================
 // K3a: merge the segments of the rows that more than one cluster held
 //   O~[b,h,:] = sum_s 2^(lse_s - max) O~_s / sum_s 2^(lse_s - max)
-// grid (B rows, 8 groups of 16 heads); 256 threads, 4 x 16 bytes each per
-// segment; rows held by one cluster were written final by the attend kernel.
+// grid (cluster boundaries 1 .. clusters-1, 8 groups of 16 heads); 256
+// threads, 4 x 16 bytes each per segment.  Boundary c merges the row that
+// holds tile bnd(c) when the boundary falls inside that row and is the row's
+// first one; rows held by one cluster were written final by the attend
+// kernel.
 // ===========================================================================
 __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ opart,
                                                        const float* __restrict__ lse,
-                                                       core::Sched sch, int slots,
+                                                       const core::Sched sch,
+                                                       const int32_t* __restrict__ crow,
                                                        __nv_bfloat16* __restrict__ omerged) {
-  const int b = blockIdx.x;
-  const int used = sch.c_last(b) - sch.c_first(b) + 1;
+  const int cb = blockIdx.x + 1;
   pdl_trigger();
-  if (used <= 1) return;
-  pdl_wait();  // partial outputs of the attend kernel
+  // every block waits for the attend kernel, those with nothing to merge
+  // too: the W_UV kernel after this one relies on this grid's completion
+  // implying the attend kernel's (it reads the rows written final there)
+  pdl_wait();
+  const long long t = sch.bnd(cb);
+  const int b = sch.tb ? ld_global_nc_s32_early(crow + cb) : (int)(t / sch.nt);
+  const long long rs = sch.row_start(b), re = sch.row_start(b + 1);
+  // the boundary is inside the row, and the one before it is not: cluster
+  // cb - 1 holds the row's first tile
+  if (rs == t || sch.bnd(cb - 1) > rs) return;
+  const int cf = cb - 1;
   const int h = blockIdx.y * 16 + (threadIdx.x >> 4);
   const int c0 = (threadIdx.x & 15) * 8;  // chunks c0, c0 + 128, c0 + 256, c0 + 384
-  const float* lse_b = lse + (size_t)b * slots * kH + h;
+  // the row's segments, in cluster order: slot 1 of cluster cf (slot 0 when
+  // the row starts its range), slot 0 of every later cluster whose range
+  // starts inside the row and is not empty
+  auto holds = [&](int c) { return c == cf || sch.bnd(c) != sch.bnd(c + 1); };
+  const int s0 = 2 * cf + sch.slot(cf, b);
+  const float* lse_h = lse + h;
   float mx = -INFINITY;
-  for (int s = 0; s < used; ++s) mx = fmaxf(mx, lse_b[(size_t)s * kH]);
+  for (int c = cf; c < sch.nc && (c == cf || sch.bnd(c) < re); ++c)
+    if (holds(c)) mx = fmaxf(mx, lse_h[(size_t)(c == cf ? s0 : 2 * c) * kH]);
   float acc[4][8];
 #pragma unroll
   for (int j = 0; j < 4; ++j)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
   float wsum = 0.f;
-  const __nv_bfloat16* src = opart + ((size_t)b * slots * kH + h) * kC + c0;
+  const __nv_bfloat16* src = opart + (size_t)h * kC + c0;
 #pragma unroll 1
-  for (int s = 0; s < used; ++s) {
-    const float w = mx == -INFINITY ? 0.f : exp2f(lse_b[(size_t)s * kH] - mx);
+  for (int c = cf; c < sch.nc && (c == cf || sch.bnd(c) < re); ++c) {
+    if (!holds(c)) continue;
+    const size_t sl = (size_t)(c == cf ? s0 : 2 * c);
+    const float w = mx == -INFINITY ? 0.f : exp2f(lse_h[sl * kH] - mx);
     wsum += w;
     uint4 v[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) v[j] = ld_global_nc_v4(src + (size_t)s * kH * kC + j * 128);
+    for (int j = 0; j < 4; ++j) v[j] = ld_global_nc_v4(src + sl * kH * kC + j * 128);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&v[j]);
@@ -893,6 +973,82 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
     o.z = pack_bf16x2(acc[j][4] * inv, acc[j][5] * inv);
     o.w = pack_bf16x2(acc[j][6] * inv, acc[j][7] * inv);
     *reinterpret_cast<uint4*>(out + j * 128) = o;
+  }
+}
+
+// ===========================================================================
+// Ragged rows (several query rows per cache row: prefill and multi-query
+// decode, whose lists end in -1 padding).  Row r needs the tiles up to and
+// including the last one that holds an entry other than -1, and at least
+// one, so that a row with nothing listed still gets its zero output; the
+// tiles after it hold only padding and are not scheduled.
+//   row_tiles_kernel   one warp per row, scanning its list from the end
+//   tile_scan_kernel   one block: tstart = exclusive prefix sum of the
+//                      counts (B + 1 entries) and, per cluster c, the row
+//                      that holds tile bnd(c)
+// ===========================================================================
+__global__ void __launch_bounds__(256) row_tiles_kernel(const int32_t* __restrict__ topk, int k,
+                                                         int B, int32_t* __restrict__ cnt) {
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (r >= B) return;
+  const int32_t* row = topk + (size_t)r * k;
+  int t = (k + core::KT - 1) / core::KT;
+#pragma unroll 1
+  for (; t > 1; --t) {
+    const int j0 = (t - 1) * core::KT + lane, j1 = j0 + 32;
+    const bool listed = (j0 < k && ld_global_nc_s32_early(row + j0) != -1) ||
+                        (j1 < k && ld_global_nc_s32_early(row + j1) != -1);
+    if (__any_sync(0xffffffffu, listed)) break;
+  }
+  if (lane == 0) cnt[r] = t;
+}
+
+__global__ void __launch_bounds__(1024) tile_scan_kernel(const int32_t* __restrict__ cnt, int B,
+                                                          int nc, int32_t* __restrict__ tstart,
+                                                          int32_t* __restrict__ tb,
+                                                          int32_t* __restrict__ crow) {
+  __shared__ int part[1024];
+  const int tid = threadIdx.x;
+  const int per = (B + 1023) / 1024;
+  const int lo = min(B, tid * per), hi = min(B, lo + per);
+  int sum = 0;
+  for (int r = lo; r < hi; ++r) sum += cnt[r];
+  part[tid] = sum;
+  __syncthreads();
+  for (int o = 1; o < 1024; o <<= 1) {
+    const int v = tid >= o ? part[tid - o] : 0;
+    __syncthreads();
+    part[tid] += v;
+    __syncthreads();
+  }
+  int run = part[tid] - sum;
+  for (int r = lo; r < hi; ++r) {
+    tstart[r] = run;
+    run += cnt[r];
+  }
+  const int tot = part[1023];
+  if (tid == 0) tstart[B] = tot;
+  __syncthreads();  // tstart written by the block is visible to it
+  // Cost units: row r spans core::kRowCostTiles units of its own cost, then one
+  // unit per tile, from u(r) = tstart[r] + r * core::kRowCostTiles.  Cluster c
+  // takes the units [c * U / nc, (c + 1) * U / nc); a range that starts in a
+  // row's own units starts at the row's first tile.
+  const long long U = (long long)tot + (long long)B * core::kRowCostTiles;
+  for (int c = tid; c <= nc; c += 1024) {
+    if (c == nc) {
+      tb[c] = tot;
+      crow[c] = B;
+      continue;
+    }
+    const long long u = (long long)c * U / nc;
+    int a = 0, e = B;  // u(a) <= u < u(e)
+    while (e - a > 1) {
+      const int m = (a + e) >> 1;
+      if ((long long)tstart[m] + (long long)m * core::kRowCostTiles <= u) a = m; else e = m;
+    }
+    const long long into = u - ((long long)tstart[a] + (long long)a * core::kRowCostTiles);
+    tb[c] = tstart[a] + (into > core::kRowCostTiles ? (int)(into - core::kRowCostTiles) : 0);
+    crow[c] = a;
   }
 }
 
@@ -1075,6 +1231,8 @@ static core::Sched make_sched(int B, int k, int clusters) {
   s.nt = ntiles_of(k);
   s.tot = B * s.nt;
   s.nc = clusters < s.tot ? clusters : s.tot;
+  s.tstart = nullptr;
+  s.tb = nullptr;
   return s;
 }
 
@@ -1089,16 +1247,22 @@ static int slots_of(const core::Sched& s, int B) {
 }
 
 struct WsLayout {
-  size_t q_tilde, opart, lse, omerged, total;
+  size_t q_tilde, opart, lse, omerged, cnt, tstart, tb, crow, total;
 };
 
-static WsLayout ws_layout(int B, int slots) {
+// Partial outputs are held per cluster (two slots each), so their size
+// depends on the cluster count, not on B or on how the rows are split.
+static WsLayout ws_layout(int B, int clusters) {
   WsLayout w;
   w.q_tilde = 0;
   w.opart = round_up(w.q_tilde + (size_t)B * kH * kC * 2, 256);
-  w.lse = round_up(w.opart + (size_t)B * slots * kH * kC * 2, 256);
-  w.omerged = round_up(w.lse + (size_t)B * slots * kH * 4, 256);
-  w.total = round_up(w.omerged + (size_t)B * kH * kC * 2, 256);
+  w.lse = round_up(w.opart + (size_t)clusters * 2 * kH * kC * 2, 256);
+  w.omerged = round_up(w.lse + (size_t)clusters * 2 * kH * 4, 256);
+  w.cnt = round_up(w.omerged + (size_t)B * kH * kC * 2, 256);
+  w.tstart = round_up(w.cnt + (size_t)B * 4, 256);
+  w.tb = round_up(w.tstart + (size_t)(B + 1) * 4, 256);
+  w.crow = round_up(w.tb + (size_t)(clusters + 1) * 4, 256);
+  w.total = round_up(w.crow + (size_t)(clusters + 1) * 4, 256);
   return w;
 }
 
@@ -1202,6 +1366,17 @@ static core::Sched schedule_for(int B, int k) {
   return s;
 }
 
+// Ragged rows: the cluster count of the uniform schedule of the same B and
+// k; the ranges come from the tile counts on the device (tile_scan_kernel),
+// and with fewer tiles than clusters some of them are empty.
+static core::Sched ragged_schedule_for(int B, int k, const int32_t* tstart, const int32_t* tb) {
+  core::Sched s = schedule_for(B, k);
+  s.tot = 0;  // (the ranges come from tb)
+  s.tstart = tstart;
+  s.tb = tb;
+  return s;
+}
+
 // 2-D tensor map over cache rows: dims {cols, rows}, row pitch rstride
 // elements, box {box_cols, 1} (one row high, as tile::gather4 requires).
 static int make_row_map(CUtensorMap* map, const void* base, int cols, unsigned long long rows,
@@ -1245,8 +1420,7 @@ extern "C" int mla_decode_num_splits(int B, int k) {
 
 extern "C" size_t mla_decode_workspace_bytes(int B, int k) {
   if (B < 1 || k < 1) return 0;
-  const core::Sched s = schedule_for(B, k);
-  return ws_layout(B, slots_of(s, B)).total;
+  return ws_layout(B, max_clusters()).total;
 }
 
 extern "C" int mla_fold_wuk(const mla_bf16_t* q_nope, const mla_bf16_t* wkv_b, int B,
@@ -1265,9 +1439,10 @@ static int decode_impl(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_
                        const mla_bf16_t* wkv_b, const mla_bf16_t* c_kv, int64_t ckv_bstride,
                        int ckv_rstride, const mla_bf16_t* k_pe, int64_t kpe_bstride,
                        int kpe_rstride, int T, const int32_t* topk, int k,
-                       const int32_t* end_pos, int B, int q_per_row, float scale, mla_bf16_t* O,
-                       void* ws, size_t ws_bytes, int32_t* status, void* stream) {
-  if (phase < 0 || phase > 3) return MLA_ERR_SHAPE;
+                       const int32_t* end_pos, int B, int q_per_row, bool ragged, float scale,
+                       mla_bf16_t* O, void* ws, size_t ws_bytes, int32_t* status,
+                       void* stream) {
+  if (phase < 0 || phase > 3 || (ragged && phase != 0)) return MLA_ERR_SHAPE;
   if (q_per_row < 1 || B % q_per_row != 0) return MLA_ERR_SHAPE;
   if (!q_nope || !q_pe || !wkv_b || !topk || !end_pos || !O) return MLA_ERR_NULL;
   if (int e = check_cache_args(c_kv, ckv_bstride, ckv_rstride, k_pe, kpe_bstride, kpe_rstride, T))
@@ -1280,9 +1455,7 @@ static int decode_impl(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_
     return MLA_ERR_ALIGN;
   if (!ws || !aligned256(ws)) return MLA_ERR_WORKSPACE;
   if (int e = check_device()) return e;
-  const core::Sched sch = schedule_for(B, k);
-  const int slots = slots_of(sch, B);
-  const WsLayout L = ws_layout(B, slots);
+  const WsLayout L = ws_layout(B, max_clusters());
   if (ws_bytes < L.total) return MLA_ERR_WORKSPACE;
   cudaStream_t st = as_stream(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
@@ -1290,7 +1463,22 @@ static int decode_impl(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_
   __nv_bfloat16* opart = reinterpret_cast<__nv_bfloat16*>(wsb + L.opart);
   float* lse = reinterpret_cast<float*>(wsb + L.lse);
   __nv_bfloat16* omerged = reinterpret_cast<__nv_bfloat16*>(wsb + L.omerged);
+  int32_t* cnt = reinterpret_cast<int32_t*>(wsb + L.cnt);
+  int32_t* tstart = reinterpret_cast<int32_t*>(wsb + L.tstart);
+  int32_t* tb = reinterpret_cast<int32_t*>(wsb + L.tb);
+  int32_t* crow = reinterpret_cast<int32_t*>(wsb + L.crow);
+  const core::Sched sch = ragged ? ragged_schedule_for(B, k, tstart, tb) : schedule_for(B, k);
+  // whether any row can be split across clusters (ragged: decided on the device)
+  const bool merge = ragged ? sch.nc > 1 : slots_of(sch, B) > 1;
 
+  if (ragged) {
+    // plain launches: they complete before the fold starts, so the attend
+    // kernel (which may start during the fold) finds the tile counts
+    row_tiles_kernel<<<(B + 7) / 8, 256, 0, st>>>(topk, k, B, cnt);
+    if (int e = launch_status()) return e;
+    tile_scan_kernel<<<1, 1024, 0, st>>>(cnt, B, sch.nc, tstart, tb, crow);
+    if (int e = launch_status()) return e;
+  }
   if (phase == 0 || phase == 1) {
     if (int e = launch_fold(reinterpret_cast<const __nv_bfloat16*>(q_nope),
                             reinterpret_cast<const __nv_bfloat16*>(wkv_b), q_tilde, B, status,
@@ -1309,7 +1497,7 @@ static int decode_impl(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_
   p.end_pos = end_pos;
   p.B = B;
   p.sch = sch;
-  p.slots = slots;
+  p.crow = crow;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.opart = opart;
   p.lse = lse;
@@ -1338,18 +1526,19 @@ static int decode_impl(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_
     }
   }
   if (phase == 0 || phase == 3) {
-    if (slots > 1) {
+    if (merge) {
+      const dim3 grid(sch.nc - 1, kH / 16);
       if (phase == 0) {
-        if (int e = launch_pdl(combine_kernel, dim3(B, kH / 16), dim3(256), 0, st, opart, lse,
-                               sch, slots, omerged))
+        if (int e = launch_pdl(combine_kernel, grid, dim3(256), 0, st, opart, lse, sch,
+                               (const int32_t*)crow, omerged))
           return e;
       } else {
-        combine_kernel<<<dim3(B, kH / 16), 256, 0, st>>>(opart, lse, sch, slots, omerged);
+        combine_kernel<<<grid, 256, 0, st>>>(opart, lse, sch, crow, omerged);
         if (int e = launch_status()) return e;
       }
     }
     return launch_uv(reinterpret_cast<const __nv_bfloat16*>(wkv_b), omerged, B,
-                     reinterpret_cast<__nv_bfloat16*>(O), status, st, phase == 0 || slots > 1);
+                     reinterpret_cast<__nv_bfloat16*>(O), status, st, phase == 0 || merge);
   }
   return MLA_OK;
 }
@@ -1361,7 +1550,8 @@ extern "C" int mla_decode(const mla_bf16_t* q_nope, const mla_bf16_t* q_pe,
                           const int32_t* end_pos, int B, float scale, mla_bf16_t* O, void* ws,
                           size_t ws_bytes, int32_t* status, void* stream) {
   return decode_impl(0, q_nope, q_pe, wkv_b, c_kv, ckv_bstride, ckv_rstride, k_pe, kpe_bstride,
-                     kpe_rstride, T, topk, k, end_pos, B, 1, scale, O, ws, ws_bytes, status, stream);
+                     kpe_rstride, T, topk, k, end_pos, B, 1, false, scale, O, ws, ws_bytes, status,
+                     stream);
 }
 
 extern "C" int mla_decode_mq(const mla_bf16_t* q_nope, const mla_bf16_t* q_pe,
@@ -1372,8 +1562,8 @@ extern "C" int mla_decode_mq(const mla_bf16_t* q_nope, const mla_bf16_t* q_pe,
                              mla_bf16_t* O, void* ws, size_t ws_bytes, int32_t* status,
                              void* stream) {
   return decode_impl(0, q_nope, q_pe, wkv_b, c_kv, ckv_bstride, ckv_rstride, k_pe, kpe_bstride,
-                     kpe_rstride, T, topk, k, end_pos, B, queries_per_row, scale, O, ws, ws_bytes,
-                     status, stream);
+                     kpe_rstride, T, topk, k, end_pos, B, queries_per_row, true, scale, O, ws,
+                     ws_bytes, status, stream);
 }
 
 extern "C" int mla_decode_phase(int phase, const mla_bf16_t* q_nope, const mla_bf16_t* q_pe,
@@ -1383,6 +1573,6 @@ extern "C" int mla_decode_phase(int phase, const mla_bf16_t* q_nope, const mla_b
                                 int k, const int32_t* end_pos, int B, float scale, mla_bf16_t* O,
                                 void* ws, size_t ws_bytes, int32_t* status, void* stream) {
   return decode_impl(phase, q_nope, q_pe, wkv_b, c_kv, ckv_bstride, ckv_rstride, k_pe,
-                     kpe_bstride, kpe_rstride, T, topk, k, end_pos, B, 1, scale, O, ws, ws_bytes,
-                     status, stream);
+                     kpe_bstride, kpe_rstride, T, topk, k, end_pos, B, 1, false, scale, O, ws,
+                     ws_bytes, status, stream);
 }

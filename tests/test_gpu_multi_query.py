@@ -60,24 +60,110 @@ def test_multi_query_matches_oracle():
     assert np.abs(got - want).max() <= MAX_ABS
 
 
-def test_shared_cache_rows_equal_decode_on_a_repeated_cache():
-    """Reading cache row r // S gives bit for bit what mla_decode gives on a
-    cache with each row repeated S times (same rows, same schedule)."""
+def test_shared_cache_rows_equal_one_query_per_row_on_a_repeated_cache():
+    """Reading cache row r // S gives bit for bit what one query per row
+    gives on a cache with each row repeated S times (same rows, same lists,
+    so the same schedule)."""
     import sparse_head_latent_absorbed_b200 as shla
     wl = mi.make_multi_query(B=4, S=3, T=500, k=150, seed=3, device="cuda")
     a = shla.mla_decode_mq(wl.q_nope, wl.q_pe, wl.wkv_b, wl.cache, wl.topk, wl.end_pos, wl.scale,
                            3)
     rep = wl.cache.repeat_interleave(3, dim=0).contiguous()
-    b = shla.mla_decode(wl.q_nope, wl.q_pe, wl.wkv_b, rep, wl.topk, wl.end_pos, wl.scale)
+    b = shla.mla_decode_mq(wl.q_nope, wl.q_pe, wl.wkv_b, rep, wl.topk, wl.end_pos, wl.scale, 1)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
 
 
-def test_one_query_per_row_is_mla_decode():
+def test_one_query_per_row_matches_mla_decode():
+    """One query per row is mla_decode's operation; the two may cut the rows
+    at different tiles (mla_decode_mq balances a per-row cost as well), so
+    they agree within the workload tolerance, and each with the oracle."""
     import sparse_head_latent_absorbed_b200 as shla
     wl = mi.make_small(B=3, T=300, k=130, seed=4, device="cuda")
     a = shla.mla_decode_mq(wl.q_nope, wl.q_pe, wl.wkv_b, wl.cache, wl.topk, wl.end_pos, wl.scale,
                            1)
     b = shla.mla_decode(wl.q_nope, wl.q_pe, wl.wkv_b, wl.cache, wl.topk, wl.end_pos, wl.scale)
     torch.cuda.synchronize()
+    a64 = a.double().cpu().numpy()
+    b64 = b.double().cpu().numpy()
+    cache = mi.f64(wl.cache)
+    want = orc.decode_absorbed(mi.f64(wl.q_nope), mi.f64(wl.q_pe), mi.f64(wl.wkv_b),
+                               cache[..., :512], cache[..., 512:], wl.topk.cpu().numpy(),
+                               wl.end_pos.cpu().numpy(), wl.scale)
+    assert _rel(a64, b64) <= REL_L2
+    assert _rel(a64, want) <= REL_L2
+    assert np.abs(a64 - want).max() <= MAX_ABS
+
+
+def test_prefill_1024_token_prompt_sampled_tokens():
+    """One prompt of 1024 tokens, top-k 256 (four 64-key tiles per token).
+    Tokens before position 255 list fewer positions and pad with -1; the
+    tiles that hold only padding are not scheduled, so the rows have 1 to 4
+    tiles and the cluster ranges cut them unevenly.  The whole prompt runs on
+    the GPU; 40 tokens (the tile edges, both ends and a seeded draw) are
+    checked against the oracle's absorbed decode at their causal limits
+    (pinned equal to the prefill branch on the CPU)."""
+    S, k = 1024, 256
+    wl = mi.make_prefill(B=1, S=S, k=k, seed=5, device="cuda")
+    got = _run(wl)
+    rng = np.random.default_rng(11)
+    fixed = [0, 1, 2, 62, 63, 64, 65, 127, 128, 191, 192, 254, 255, 256, 257, 511, 512, 1022, 1023]
+    rows = sorted(set(fixed) | set(rng.choice(S, 40 - len(fixed), replace=False).tolist()))
+    sel = torch.tensor(rows, device="cuda")
+    cache = mi.f64(wl.cache)
+    c = np.broadcast_to(cache, (len(rows),) + cache.shape[1:])
+    want = orc.decode_absorbed(mi.f64(wl.q_nope[sel]), mi.f64(wl.q_pe[sel]), mi.f64(wl.wkv_b),
+                               c[..., :512], c[..., 512:], wl.topk[sel].cpu().numpy(),
+                               wl.end_pos[sel].cpu().numpy(), wl.scale)
+    g = got[rows]
+    assert np.isfinite(got).all()
+    assert _rel(g, want) <= REL_L2
+    assert np.abs(g - want).max() <= MAX_ABS * max(1.0, float(np.abs(want).max()))
+
+
+def test_trailing_padding_tiles_are_skipped():
+    """Four query rows with room for 640 entries (10 tiles each) but at most
+    40 listed: each row needs one tile, so the 4 tiles in all fall to 4 of
+    the clusters and the others get an empty range; one row lists nothing.
+    The result is bit for bit mla_decode on the same lists cut to 40 entries
+    (one tile per row, each row held whole by one cluster in both), which
+    also shows that the padding tiles were not run: a padding tile changes
+    no value, but a row cut in two would be merged in another order."""
+    import sparse_head_latent_absorbed_b200 as shla
+    wl = mi.make_small(B=4, T=300, k=40, seed=6, device="cuda")
+    wl.topk[2] = -1
+    padded = torch.full((4, 640), -1, dtype=torch.int32, device="cuda")
+    padded[:, :40] = wl.topk
+    status = torch.zeros(2, dtype=torch.int32, device="cuda")
+    a = shla.mla_decode_mq(wl.q_nope, wl.q_pe, wl.wkv_b, wl.cache, padded, wl.end_pos, wl.scale,
+                           1, status=status)
+    b = shla.mla_decode(wl.q_nope, wl.q_pe, wl.wkv_b, wl.cache, wl.topk, wl.end_pos, wl.scale)
+    torch.cuda.synchronize()
+    assert status.tolist() == [0, 0]
     assert torch.equal(a, b)
+    assert float(a[2].abs().max()) == 0.0
+    cache = mi.f64(wl.cache)
+    want = orc.decode_absorbed(mi.f64(wl.q_nope), mi.f64(wl.q_pe), mi.f64(wl.wkv_b),
+                               cache[..., :512], cache[..., 512:], padded.cpu().numpy(),
+                               wl.end_pos.cpu().numpy(), wl.scale)
+    assert _rel(a.double().cpu().numpy(), want) <= REL_L2
+
+
+def test_ragged_rows_split_across_clusters():
+    """Multi-query rows whose lists end in padding of different lengths, with
+    enough tiles in all that rows are split across clusters at uneven
+    points: every split row is merged from the right clusters' slots."""
+    wl = mi.make_multi_query(B=24, S=2, T=3000, k=1024, seed=7, device="cuda")
+    # cut each row's list to a different length (padding at the end)
+    g = torch.Generator().manual_seed(8)
+    keep = torch.randint(1, 1025, (wl.B,), generator=g)
+    keep[::5] = 1024
+    for r in range(wl.B):
+        wl.topk[r, int(keep[r]):] = -1
+    got = _run(wl)
+    cache = mi.f64(wl.cache)
+    want = orc.decode_multi_query(mi.f64(wl.q_nope), mi.f64(wl.q_pe), mi.f64(wl.wkv_b),
+                                  cache[..., :512], cache[..., 512:], wl.topk.cpu().numpy(),
+                                  wl.end_pos.cpu().numpy(), wl.scale, 2)
+    assert _rel(got, want) <= REL_L2
+    assert np.abs(got - want).max() <= MAX_ABS * max(1.0, float(np.abs(want).max()))
