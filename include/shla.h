@@ -182,6 +182,13 @@ int mla_cache_write_noalloc(const mla_bf16_t* x, const mla_bf16_t* w_kva,
  * units), and the per-split partial outputs that the merge reads.  O is
  * rounded to bf16 once, at the end.
  *
+ * Work split: the flattened list of (row, 64-key tile) is cut into equal
+ * contiguous ranges, one per SM pair; a row cut between two ranges is merged
+ * from their partial results by log-sum-exp.  The ranges depend on the
+ * number of SM pairs the device runs the kernel on, so on devices with
+ * different SM counts the split rows (and the last bits of their outputs)
+ * may differ; on one device the result is the same on every call.
+ *
  * The call enqueues three or four kernels on `stream`.  The first waits for
  * the stream's earlier work as usual.  The later ones use programmatic
  * dependent launch: each may start its set-up while its predecessor drains,
@@ -220,6 +227,15 @@ int mla_decode(const mla_bf16_t* q_nope, const mla_bf16_t* q_pe, const mla_bf16_
  *   q_nope, q_pe, topk, end_pos, O: B query rows, layouts as mla_decode
  *   c_kv, k_pe, strides, T: B / queries_per_row cache batch rows
  *   ws: mla_decode_workspace_bytes(B, k) bytes
+ *
+ * Ragged lists: the lists of prefill tokens and new tokens end in -1 padding
+ * of different lengths.  Two small kernels run first: one counts, per query
+ * row, the 64-entry tiles up to the last one that holds an entry other than
+ * -1 (at least one), and one prefix-sums the counts and cuts the work into
+ * ranges that balance the tiles plus a fixed cost per row; the tiles after a
+ * row's last listed entry are not run.  The split points therefore differ
+ * from mla_decode's, and with one query per row the two calls agree within
+ * rounding, not bit for bit.
  * Requires queries_per_row >= 1 dividing B, and every cache row in use
  * addressable as a 32-bit row index: (B / queries_per_row - 1) *
  * (ckv_bstride / ckv_rstride) + T <= 2^31 - 1 (else MLA_ERR_SHAPE).
@@ -279,7 +295,8 @@ int mla_gather_rows(const mla_bf16_t* c_kv, int64_t ckv_bstride, int ckv_rstride
                     const int32_t* topk, int B, int k, const int32_t* end_pos,
                     mla_bf16_t* rows, int32_t* status, void* stream);
 
-/* Number of key splits mla_decode uses for (B, k) on the current device. */
+/* The most ranges (SM pairs) that share one row in mla_decode's work split
+ * for (B, k) on the current device (1: no row is split). */
 int mla_decode_num_splits(int B, int k);
 
 /*
