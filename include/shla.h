@@ -295,6 +295,19 @@ int mla_gather_rows(const mla_bf16_t* c_kv, int64_t ckv_bstride, int ckv_rstride
                     const int32_t* topk, int B, int k, const int32_t* end_pos,
                     mla_bf16_t* rows, int32_t* status, void* stream);
 
+/*
+ * Test hook: the expiry path of the bounded waits.  Every wait in the
+ * library's kernels (mbarrier phases, the MMA issuer's event loop) gives up
+ * after 1 s, sets MLA_STATUS_TIMEOUT in status[0] and lets its kernel wind
+ * down, so that a lost arrival ends as an error the host can read instead of
+ * a hung GPU.  This call launches one block of two warps that wait, through
+ * the same code, on an mbarrier that nothing arrives on; it returns after the
+ * limit with status[0] |= MLA_STATUS_TIMEOUT and gave_up[0] += 2 (one per
+ * warp).  The GPU context stays usable.
+ *   status  int32[2] device (status[1] untouched); gave_up int32[1] device
+ */
+int mla_wait_limit_check(int32_t* status, int32_t* gave_up, void* stream);
+
 /* The most ranges (SM pairs) that share one row in mla_decode's work split
  * for (B, k) on the current device (1: no row is split). */
 int mla_decode_num_splits(int B, int k);

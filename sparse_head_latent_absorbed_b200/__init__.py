@@ -27,6 +27,7 @@ _EXPORTS = (
     "mla_query_proj",
     "mla_query_proj_workspace_bytes",
     "mla_rope",
+    "mla_wait_limit_check",
     "status_string",
 )
 

@@ -30,6 +30,7 @@ _SIGS = {
                                          _vp, _c_i64, _c_int, _vp, _c_i64, _c_int, _c_int, _vp]),
     "mla_decode_workspace_bytes": (_c_size, [_c_int, _c_int]),
     "mla_decode_num_splits": (_c_int, [_c_int, _c_int]),
+    "mla_wait_limit_check": (_c_int, [_vp, _vp, _vp]),
     "mla_decode": (_c_int, [_vp, _vp, _vp, _vp, _c_i64, _c_int, _vp, _c_i64, _c_int, _c_int,
                             _vp, _c_int, _vp, _c_int, _c_float, _vp, _vp, _c_size, _vp, _vp]),
     "mla_decode_mq": (_c_int, [_vp, _vp, _vp, _vp, _c_i64, _c_int, _vp, _c_i64, _c_int, _c_int,
@@ -307,6 +308,14 @@ def mla_fold_wuk(q_nope: torch.Tensor, wkv_b: torch.Tensor,
     _check(LIB.mla_fold_wuk(_p(q_nope), _p(wkv_b), B, _p(out), _stream(q_nope.device)),
            "mla_fold_wuk")
     return out
+
+
+def mla_wait_limit_check(status: torch.Tensor, gave_up: torch.Tensor) -> None:
+    """Launches the bounded-wait expiry check (see include/shla.h)."""
+    _need(status, torch.int32, "status")
+    _need(gave_up, torch.int32, "gave_up")
+    _check(LIB.mla_wait_limit_check(_p(status), _p(gave_up), _stream(status.device)),
+           "mla_wait_limit_check")
 
 
 def mla_index_mask(topk: torch.Tensor, end_pos: torch.Tensor, T: int,

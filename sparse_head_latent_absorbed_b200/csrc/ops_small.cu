@@ -124,6 +124,34 @@ extern "C" int mla_rope(const mla_bf16_t* x, const float* rope, int B, int S, in
   return launch_status();
 }
 
+// ---------------------------------------------------------------------------
+// the bounded wait's expiry path
+// ---------------------------------------------------------------------------
+
+// Two warps wait, through the waits every kernel of the library uses, on an
+// mbarrier that nothing arrives on: each gives up after the limit, flags the
+// CTA's abort word and the status word, and the kernel returns.  The second
+// warp may also leave through the abort word the first one set.
+__global__ void __launch_bounds__(64) wait_limit_kernel(int32_t* status, int32_t* gave_up) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_word;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_word = 0;
+    fence_mbarrier_init_cluster();
+  }
+  __syncthreads();
+  const bool ok = warp_wait(&bar, 0, &abort_word, status);
+  if (!ok && (threadIdx.x & 31) == 0) atomicAdd(gave_up, 1);
+}
+
+extern "C" int mla_wait_limit_check(int32_t* status, int32_t* gave_up, void* stream) {
+  if (!status || !gave_up) return MLA_ERR_NULL;
+  if (int e = check_device()) return e;
+  wait_limit_kernel<<<1, 64, 0, as_stream(stream)>>>(status, gave_up);
+  return launch_status();
+}
+
 extern "C" int mla_index_mask(const int32_t* topk, int B, int k, const int32_t* end_pos, int T,
                               uint8_t* mask, int32_t* status, void* stream) {
   if (!topk || !end_pos || !mask) return MLA_ERR_NULL;
