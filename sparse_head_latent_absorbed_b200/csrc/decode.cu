@@ -931,27 +931,24 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
   // the row starts its range), slot 0 of every later cluster whose range
   // starts inside the row and is not empty
   auto holds = [&](int c) { return c == cf || sch.bnd(c) != sch.bnd(c + 1); };
+  auto in_row = [&](int c) { return c < sch.nc && (c == cf || sch.bnd(c) < re); };
+  auto next_held = [&](int from) {  // the next cluster from `from` on holding a segment, or -1
+    int x = from;
+    while (in_row(x) && !holds(x)) ++x;
+    return in_row(x) ? x : -1;
+  };
   const int s0 = 2 * cf + sch.slot(cf, b);
+  auto slot_of = [&](int c) { return (size_t)(c == cf ? s0 : 2 * c); };
   const float* lse_h = lse + h;
-  float mx = -INFINITY;
-  for (int c = cf; c < sch.nc && (c == cf || sch.bnd(c) < re); ++c)
-    if (holds(c)) mx = fmaxf(mx, lse_h[(size_t)(c == cf ? s0 : 2 * c) * kH]);
+  const __nv_bfloat16* src = opart + (size_t)h * kC + c0;
   float acc[4][8];
 #pragma unroll
   for (int j = 0; j < 4; ++j)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
   float wsum = 0.f;
-  const __nv_bfloat16* src = opart + (size_t)h * kC + c0;
-#pragma unroll 1
-  for (int c = cf; c < sch.nc && (c == cf || sch.bnd(c) < re); ++c) {
-    if (!holds(c)) continue;
-    const size_t sl = (size_t)(c == cf ? s0 : 2 * c);
-    const float w = mx == -INFINITY ? 0.f : exp2f(lse_h[sl * kH] - mx);
+  auto add = [&](const uint4 (&v)[4], float w) {
     wsum += w;
-    uint4 v[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) v[j] = ld_global_nc_v4(src + sl * kH * kC + j * 128);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&v[j]);
@@ -961,6 +958,32 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
         acc[j][2 * e] += w * f.x;
         acc[j][2 * e + 1] += w * f.y;
       }
+    }
+  };
+  const int c1 = next_held(cf + 1);
+  if (c1 >= 0 && next_held(c1 + 1) < 0) {
+    // two segments (the usual split): every load in flight together
+    const size_t sa = slot_of(cf), sb = slot_of(c1);
+    uint4 va[4], vb[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) va[j] = ld_global_nc_v4(src + sa * kH * kC + j * 128);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) vb[j] = ld_global_nc_v4(src + sb * kH * kC + j * 128);
+    const float la = lse_h[sa * kH], lb = lse_h[sb * kH];
+    const float mx = fmaxf(la, lb);
+    add(va, mx == -INFINITY ? 0.f : exp2f(la - mx));
+    add(vb, mx == -INFINITY ? 0.f : exp2f(lb - mx));
+  } else {
+    // the segments in cluster order
+    float mx = -INFINITY;
+    for (int c = cf; c >= 0; c = next_held(c + 1)) mx = fmaxf(mx, lse_h[slot_of(c) * kH]);
+#pragma unroll 1
+    for (int c = cf; c >= 0; c = next_held(c + 1)) {
+      const size_t sl = slot_of(c);
+      uint4 v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[j] = ld_global_nc_v4(src + sl * kH * kC + j * 128);
+      add(v, mx == -INFINITY ? 0.f : exp2f(lse_h[sl * kH] - mx));
     }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
