@@ -640,9 +640,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
       if (i == 0 || c.jt == 0) prefetch_q(i, c);
       if (!warp_wait(&bars.s_full, i & 1, abort, p.status)) break;
       tc_fence_after();
-      // the score tile just finished was the last product that used this
-      // segment's Q~ when the tile ends its batch row
-      if (c.jt == c.nr - 1 && i + 1 < n) load_q(c.bb + 1);
       uint32_t r[2][32];
       tmem_ld_16x256b_x8(tmem + ((uint32_t)(q4 * 32) << 16) + T_S, r[0]);
       tmem_ld_16x256b_x8(tmem + ((uint32_t)(q4 * 32 + 16) << 16) + T_S, r[1]);
@@ -697,6 +694,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(core::NTHREADS, 1)
                        r[hf][4 * k + 2], r[hf][4 * k + 3]);
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.f_full);
+      // the score tile just finished was the last product that used this
+      // segment's Q~ when the tile ends its batch row: load the next row's,
+      // after this tile's full scores are out (the softmax and the segment's
+      // flush proceed meanwhile)
+      if (c.jt == c.nr - 1 && i + 1 < n) load_q(c.bb + 1);
       c = next_pos(c);
     }
     // on an abort, partial scores the peer may still be sending land before
