@@ -1085,8 +1085,6 @@ __global__ void __launch_bounds__(1024) tile_scan_kernel(const int32_t* __restri
 // grid (128 heads, batch blocks of NB); 128 threads; K in 4 chunks of 128,
 // double-buffered (cp.async for chunk k+2 while the MMAs of chunk k run).
 // ===========================================================================
-constexpr int kMaxSlots = 32;
-
 template <int NB>
 __global__ void __launch_bounds__(128) uv_kernel(const __nv_bfloat16* __restrict__ wkv_b,
                                                   const __nv_bfloat16* __restrict__ omerged,
@@ -1383,7 +1381,10 @@ static int launch_uv(const __nv_bfloat16* wkv_b, const __nv_bfloat16* omerged, i
 }
 
 // The number of clusters is capped so that no batch row meets more than
-// kMaxSlots of them (only matters for very small B x k).
+// kMaxSlots of them, which bounds the segments the merge of one row reads
+// (only matters for very small B x k).
+constexpr int kMaxSlots = 32;
+
 static core::Sched schedule_for(int B, int k) {
   int nc = max_clusters();
   core::Sched s = make_sched(B, k, nc);

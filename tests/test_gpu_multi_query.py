@@ -167,3 +167,57 @@ def test_ragged_rows_split_across_clusters():
                                   wl.end_pos.cpu().numpy(), wl.scale, 2)
     assert _rel(got, want) <= REL_L2
     assert np.abs(got - want).max() <= MAX_ABS * max(1.0, float(np.abs(want).max()))
+
+
+def test_ragged_row_split_across_many_clusters():
+    """Two query rows of 32 tiles each: with so few tiles the ranges are one
+    tile or none, so each row is merged from about 30 clusters' segments
+    (the merge's general path), with trailing padding on one row."""
+    wl = mi.make_multi_query(B=2, S=1, T=3000, k=2048, seed=9, device="cuda")
+    wl.topk[1, 1500:] = -1
+    got = _run(wl)
+    cache = mi.f64(wl.cache)
+    want = orc.decode_multi_query(mi.f64(wl.q_nope), mi.f64(wl.q_pe), mi.f64(wl.wkv_b),
+                                  cache[..., :512], cache[..., 512:], wl.topk.cpu().numpy(),
+                                  wl.end_pos.cpu().numpy(), wl.scale, 1)
+    assert _rel(got, want) <= REL_L2
+    assert np.abs(got - want).max() <= MAX_ABS * max(1.0, float(np.abs(want).max()))
+
+
+@pytest.mark.parametrize("case", range(6))
+def test_ragged_seeded_sweep(case):
+    """Seeded random shapes for the ragged schedule: sequences, new tokens
+    per sequence (1, 2 or 4), list length, trailing padding per row (from
+    none to all of it), and a few invalid entries; each checked against the
+    oracle, with the invalid entries counted in status[1]."""
+    import sparse_head_latent_absorbed_b200 as shla
+    rng = np.random.default_rng(1000 + case)
+    S = int(rng.choice([1, 2, 4]))
+    B = int(rng.integers(1, 12))
+    k = int(rng.choice([40, 64, 130, 700, 1500]))
+    T = int(rng.integers(k + 10, 3 * k + 100))
+    wl = mi.make_multi_query(B=B, S=S, T=T, k=k, seed=500 + case, device="cuda")
+    topk = wl.topk.cpu()
+    ep = wl.end_pos.cpu()
+    n_bad = 0
+    for r in range(wl.B):
+        keep = int(rng.integers(0, k + 1))
+        topk[r, keep:] = -1
+        if keep > 2 and rng.random() < 0.5:
+            topk[r, 1] = int(ep[r]) + 5  # out of range: masked and counted
+            n_bad += 1
+    wl.topk.copy_(topk)
+    status = torch.zeros(2, dtype=torch.int32, device="cuda")
+    out = shla.mla_decode_mq(wl.q_nope, wl.q_pe, wl.wkv_b, wl.cache, wl.topk, wl.end_pos,
+                             wl.scale, S, status=status)
+    torch.cuda.synchronize()
+    assert status.tolist() == [0, n_bad]
+    got = out.double().cpu().numpy()
+    cache = mi.f64(wl.cache)
+    want = orc.decode_multi_query(mi.f64(wl.q_nope), mi.f64(wl.q_pe), mi.f64(wl.wkv_b),
+                                  cache[..., :512], cache[..., 512:], topk.numpy(),
+                                  ep.numpy(), wl.scale, S)
+    assert np.isfinite(got).all()
+    if np.linalg.norm(want) > 0:
+        assert _rel(got, want) <= REL_L2
+    assert np.abs(got - want).max() <= MAX_ABS * max(1.0, float(np.abs(want).max()))
