@@ -77,12 +77,32 @@ def load_peaks(path=os.path.join(ROOT, "MEASURED_PEAKS.json")):
                 "source": "fallback"}
 
 
-def kernel_source_sha():
+def code_only(text):
+    """C++/CUDA source without // comments, trailing blanks and empty lines:
+    what the compiler sees of it, so that editing a comment does not
+    invalidate a profile taken on the same code.  (The sources use no block
+    comments, and no string literal in them holds //.)"""
+    out = []
+    for line in text.splitlines():
+        code = line.split("//", 1)[0].rstrip()
+        if code:
+            out.append(code)
+    return "\n".join(out) + "\n"
+
+
+def kernel_source_sha(texts=None):
+    """sha256 of the attend kernel's code (decode.cu and common.cuh, comments
+    removed); `texts` may give the two files' contents instead of reading them."""
     h = hashlib.sha256()
-    for rel in ("sparse_head_latent_absorbed_b200/csrc/decode.cu",
-                "sparse_head_latent_absorbed_b200/csrc/common.cuh"):
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+    rels = ("sparse_head_latent_absorbed_b200/csrc/decode.cu",
+            "sparse_head_latent_absorbed_b200/csrc/common.cuh")
+    for i, rel in enumerate(rels):
+        if texts is not None:
+            text = texts[i]
+        else:
+            with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+                text = f.read()
+        h.update(code_only(text).encode())
     return h.hexdigest()
 
 

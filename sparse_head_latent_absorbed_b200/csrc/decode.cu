@@ -1,5 +1,7 @@
 // Absorbed sparse MLA decode for sm_100a ("Mix and project" page, the decode
-// ("MQA decode") code excerpt).  Three kernels on the caller's stream:
+// ("MQA decode") code excerpt).  Up to four kernels on the caller's stream
+// (mla_decode_mq first runs two small ones that schedule ragged lists,
+// row_tiles_kernel and tile_scan_kernel):
 //
 //   fold_kernel      q~ = q_nope W_UK per head (tcgen05, latent as M, batch as N)
 //   core_kernel      persistent 2-CTA clusters over equal ranges of the
@@ -11,6 +13,7 @@
 //                    distributed shared memory and both run the same softmax
 //                    over all heads.
 //   combine_kernel   log-sum-exp merge of the rows split across clusters
+//                    (launched only when some row is split)
 //   uv_kernel        O = O~ W_UV^T per head on the merged O~ (tcgen05, value
 //                    dim as M, batch as N)
 #include <math.h>

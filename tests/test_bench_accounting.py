@@ -55,3 +55,19 @@ def test_fewer_than_three_warmup_steps_are_rejected():
     r = subprocess.run([sys.executable, "bench.py", "--warmup", "2"], cwd=ROOT,
                        capture_output=True, text=True, timeout=120)
     assert r.returncode == 2 and "warmup" in r.stderr
+
+
+def test_kernel_hash_ignores_comments_only():
+    """The profiled-traffic key changes with the attend kernel's code, not
+    with its comments."""
+    import bench
+    rels = ("sparse_head_latent_absorbed_b200/csrc/decode.cu",
+            "sparse_head_latent_absorbed_b200/csrc/common.cuh")
+    texts = [open(os.path.join(bench.ROOT, r), encoding="utf-8").read() for r in rels]
+    base = bench.kernel_source_sha(texts)
+    assert base == bench.kernel_source_sha()
+    commented = [texts[0] + "\n// a note\n\n", texts[1].replace("\n", "  // x\n", 1)]
+    assert bench.kernel_source_sha(commented) == base
+    changed = [texts[0].replace("kRescaleThreshold = 8.0f", "kRescaleThreshold = 7.0f"), texts[1]]
+    assert changed[0] != texts[0]
+    assert bench.kernel_source_sha(changed) != base
