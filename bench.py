@@ -573,6 +573,30 @@ def run_ours(args):
                 for ph in (1, 2, 3):
                     phase_ms[ph].append(ev[ph - 1].elapsed_time(ev[ph]))
     peaks = load_peaks()
+    cache_write = None
+    if write:
+        # the cache write alone (kv = x W_KVa, RMSNorm, RoPE, row store), each
+        # call after an L2 flush: bound by streaming W_KVa once
+        n_rep = max(3, min(args.steps, 200))
+        cw_ms = []
+        for i in range(n_rep + 3):
+            flush_l2()
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            shla.mla_cache_write(wl.x, wl.w_kva, wl.norm_w, wl.eps, tab, wl.write_pos, wl.cache,
+                                 ws=cw_ws)
+            b_.record(stream)
+            torch.cuda.synchronize()
+            if i >= 3:
+                cw_ms.append(a.elapsed_time(b_))
+        cw = reduce_max(statistics.mean(cw_ms), world, dev)
+        cw_bytes = 7168 * 576 * 2 + B * (7168 * 2 + 576 * 2)
+        cache_write = {"what": "cache write of B rows: kv = x W_KVa (split-K tcgen05) + RMSNorm + "
+                               "RoPE + bf16 store (cw_gemm_kernel + cw_finalize_kernel)",
+                       "us": cw * 1e3, "bound": "hbm", "algorithmic_bytes": cw_bytes,
+                       "achieved": cw_bytes / (cw * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                       "unit": "GB/s",
+                       "frac": cw_bytes / (cw * 1e-3) / 1e9 / peaks["hbm_gbs"]}
     roofline = None
     if phase_ms[2]:
         core_ms = reduce_max(statistics.mean(phase_ms[2]), world, dev)
@@ -651,6 +675,7 @@ def run_ours(args):
         "data": "synthetic (seeded, distributions of the workload; no public dataset involved)",
         "config": workload_config(args.config, world),
         "roofline": roofline,
+        **({"cache_write": cache_write} if cache_write else {}),
         "e2e": {"value": world * units / (e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
                 "what": "H2D of q_nope, q_pe, top-k, end_pos from pinned host memory, "

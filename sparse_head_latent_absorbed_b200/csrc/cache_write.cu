@@ -46,6 +46,7 @@ __global__ void __launch_bounds__(128) cw_gemm_kernel(const __nv_bfloat16* __res
   __shared__ uint32_t tmem_base;
   const int mt = blockIdx.x, kc = blockIdx.y, r0 = blockIdx.z * NB;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_trigger();  // the finalize kernel may be scheduled (it waits for this grid)
 
   if (warp == 0) {
     tmem_alloc(&tmem_base, NCOLS);
@@ -126,10 +127,16 @@ __global__ void __launch_bounds__(256) cw_finalize_kernel(
   const int b = r / S, s = r - b * S;
   const int pos = start_pos + s;
   const int tid = threadIdx.x;
+  pdl_wait();  // the GEMM's partials (a no-op when launched without programmatic dependence)
   float ss = 0.f;
   for (int f = tid; f < kOut; f += 256) {
+    // the chunks in order; all their loads in flight together
+    float v[NKCH];
+#pragma unroll
+    for (int c = 0; c < NKCH; ++c) v[c] = part[((size_t)c * rows + r) * kOut + f];
     float acc = 0.f;
-    for (int c = 0; c < NKCH; ++c) acc += part[((size_t)c * rows + r) * kOut + f];
+#pragma unroll
+    for (int c = 0; c < NKCH; ++c) acc += v[c];
     kv[f] = acc;
     if (f < kLat) ss += acc * acc;
   }
@@ -201,11 +208,12 @@ extern "C" int mla_cache_write(const mla_bf16_t* x, const mla_bf16_t* w_kva,
   else if (rows <= 128) e = launch_cw_gemm<128>(xb, wb, rows, part, st);
   else e = launch_cw_gemm<256>(xb, wb, rows, part, st);
   if (e) return e;
-  cw_finalize_kernel<<<rows, 256, 0, st>>>(
-      part, rows, reinterpret_cast<const __nv_bfloat16*>(norm_w), eps, rope, S, start_pos,
-      reinterpret_cast<__nv_bfloat16*>(c_kv), ckv_bstride, ckv_rstride,
-      reinterpret_cast<__nv_bfloat16*>(k_pe), kpe_bstride, kpe_rstride);
-  return launch_status();
+  // programmatic serialisation: the finalize kernel is scheduled while the
+  // GEMM drains and waits for it before reading the partials
+  return launch_pdl(cw_finalize_kernel, dim3(rows), dim3(256), 0, st, (const float*)part, rows,
+                    reinterpret_cast<const __nv_bfloat16*>(norm_w), eps, rope, S, start_pos,
+                    reinterpret_cast<__nv_bfloat16*>(c_kv), (long long)ckv_bstride, ckv_rstride,
+                    reinterpret_cast<__nv_bfloat16*>(k_pe), (long long)kpe_bstride, kpe_rstride);
 }
 
 // ---------------------------------------------------------------------------
