@@ -103,6 +103,10 @@ int mla_rope(const mla_bf16_t* x, const float* rope, int B, int S, int Hx, int i
  *   ws      device workspace of at least mla_cache_write_workspace_bytes(B*S)
  *           bytes, 256-byte aligned; contents need not be initialised
  * Requires 1 <= B*S <= 4096.
+ * Two kernels are enqueued on `stream`: a split-K GEMM, then the finalize
+ * kernel under programmatic dependent launch (it waits for the GEMM before
+ * reading its partials).  For the caller nothing changes: work enqueued
+ * after the call starts when the finalize kernel has finished.
  */
 size_t mla_cache_write_workspace_bytes(int rows);
 int mla_cache_write(const mla_bf16_t* x, const mla_bf16_t* w_kva, const mla_bf16_t* norm_w,
