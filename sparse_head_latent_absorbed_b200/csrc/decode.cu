@@ -965,26 +965,47 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
       }
     }
   };
-  const int c1 = next_held(cf + 1);
-  if (c1 >= 0 && next_held(c1 + 1) < 0) {
-    // two segments (the usual split): every load in flight together
-    const size_t sa = slot_of(cf), sb = slot_of(c1);
-    uint4 va[4], vb[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) va[j] = ld_global_nc_v4(src + sa * kH * kC + j * 128);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) vb[j] = ld_global_nc_v4(src + sb * kH * kC + j * 128);
-    const float la = lse_h[sa * kH], lb = lse_h[sb * kH];
-    const float mx = fmaxf(la, lb);
-    add(va, mx == -INFINITY ? 0.f : exp2f(la - mx));
-    add(vb, mx == -INFINITY ? 0.f : exp2f(lb - mx));
-  } else {
-    // the segments in cluster order
+  // the row's segments in cluster order; up to four (every split row of the
+  // workloads here) two at a time, each pair's loads in flight together
+  constexpr int kFast = 4;
+  int cl[kFast];
+  cl[0] = cf;
+  cl[1] = next_held(cf + 1);
+  cl[2] = cl[1] >= 0 ? next_held(cl[1] + 1) : -1;
+  cl[3] = cl[2] >= 0 ? next_held(cl[2] + 1) : -1;
+  const int more = cl[3] >= 0 ? next_held(cl[3] + 1) : -1;
+  const int np = cl[1] < 0 ? 1 : cl[2] < 0 ? 2 : cl[3] < 0 ? 3 : 4;
+  if (more < 0) {
+    float l[kFast];
     float mx = -INFINITY;
-    for (int c = cf; c >= 0; c = next_held(c + 1)) mx = fmaxf(mx, lse_h[slot_of(c) * kH]);
+#pragma unroll
+    for (int q = 0; q < kFast; ++q)
+      if (q < np) {
+        l[q] = lse_h[slot_of(cl[q]) * kH];
+        mx = fmaxf(mx, l[q]);
+      }
+    // two segments at a time, both segments' loads in flight together
+#pragma unroll
+    for (int q = 0; q < kFast; q += 2) {
+      if (q < np) {
+        uint4 va[4], vb[4];
+        const size_t sa = slot_of(cl[q]);
+        const size_t sb = slot_of(q + 1 < np ? cl[q + 1] : cl[q]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) va[j] = ld_global_nc_v4(src + sa * kH * kC + j * 128);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) vb[j] = ld_global_nc_v4(src + sb * kH * kC + j * 128);
+        add(va, mx == -INFINITY ? 0.f : exp2f(l[q] - mx));
+        if (q + 1 < np) add(vb, mx == -INFINITY ? 0.f : exp2f(l[q + 1] - mx));
+      }
+    }
+  } else {
+    // more segments (very small B x k): in cluster order, one after another
+    float mx = -INFINITY;
+    for (int c2 = cf; c2 >= 0; c2 = next_held(c2 + 1)) mx = fmaxf(mx, lse_h[slot_of(c2) * kH]);
 #pragma unroll 1
-    for (int c = cf; c >= 0; c = next_held(c + 1)) {
-      const size_t sl = slot_of(c);
+    for (int c2 = cf; c2 >= 0; c2 = next_held(c2 + 1)) {
+      const size_t sl = slot_of(c2);
       uint4 v[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) v[j] = ld_global_nc_v4(src + sl * kH * kC + j * 128);
