@@ -246,20 +246,7 @@ __global__ void __launch_bounds__(128) xwt_finish_bf16(const float* __restrict__
   const int used = sch.c_last(m) - sch.c_first(m) + 1;
   pdl_wait();  // the partials of the GEMM before this kernel
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-  for (int s = 0; s < used; ++s) {
-    const float4* src =
-        reinterpret_cast<const float4*>(part + ((size_t)(m * sch.slots + s) * B + b) * 128 + nl);
-    const float4 v0 = src[0], v1 = src[1];
-    acc[0] += v0.x;
-    acc[1] += v0.y;
-    acc[2] += v0.z;
-    acc[3] += v0.w;
-    acc[4] += v1.x;
-    acc[5] += v1.y;
-    acc[6] += v1.z;
-    acc[7] += v1.w;
-  }
+  xwt_sum_slots<4>(part, sch, m, nl, b, B, 0, 1, used, acc);
   uint4 o;
   o.x = pack_bf16x2(acc[0], acc[1]);
   o.y = pack_bf16x2(acc[2], acc[3]);

@@ -48,20 +48,7 @@ __global__ void __launch_bounds__(QA_THREADS) qa_finish(const float* __restrict_
   pdl_trigger();  // the second GEMM may set up and prefetch its weight now
   pdl_wait();     // the partials of the first GEMM
   float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-  for (int s = g; s < used; s += QA_GROUPS) {
-    const float4* src =
-        reinterpret_cast<const float4*>(part + ((size_t)(m * sch.slots + s) * B + b) * 128 + nl);
-    const float4 a = src[0], c = src[1];
-    v[0] += a.x;
-    v[1] += a.y;
-    v[2] += a.z;
-    v[3] += a.w;
-    v[4] += c.x;
-    v[5] += c.y;
-    v[6] += c.z;
-    v[7] += c.w;
-  }
+  xwt_sum_slots<4>(part, sch, m, nl, b, B, g, QA_GROUPS, used, v);
   if (g > 0) {
     float4* dst = reinterpret_cast<float4*>(&gsum[g - 1][n0]);
     dst[0] = make_float4(v[0], v[1], v[2], v[3]);
@@ -126,20 +113,7 @@ __global__ void __launch_bounds__(128) qb_finish(const float* __restrict__ part,
   const int used = sch.c_last(m) - sch.c_first(m) + 1;
   pdl_wait();  // the partials of the second GEMM
   float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-  for (int s = 0; s < used; ++s) {
-    const float4* src =
-        reinterpret_cast<const float4*>(part + ((size_t)(m * sch.slots + s) * B + b) * 128 + nl);
-    const float4 a = src[0], c = src[1];
-    v[0] += a.x;
-    v[1] += a.y;
-    v[2] += a.z;
-    v[3] += a.w;
-    v[4] += c.x;
-    v[5] += c.y;
-    v[6] += c.z;
-    v[7] += c.w;
-  }
+  xwt_sum_slots<2>(part, sch, m, nl, b, B, 0, 1, used, v);
   uint4 o;
   uint32_t* op = reinterpret_cast<uint32_t*>(&o);
   if (e < DN) {

@@ -32,6 +32,42 @@ struct XwtSched {
   }
 };
 
+// acc[0..7] += the partials of outputs nl .. nl + 7 of row tile m, batch row
+// b, in slots s0, s0 + step, s0 + 2 step, ... below `used`, added in slot
+// order; the loads of kBatch slots are in flight together.
+template <int kBatch>
+__device__ __forceinline__ void xwt_sum_slots(const float* __restrict__ part, const XwtSched& sch,
+                                              int m, int nl, int b, int B, int s0, int step,
+                                              int used, float (&acc)[8]) {
+#pragma unroll 1
+  for (int base = s0; base < used; base += kBatch * step) {
+    float4 v[kBatch][2];
+#pragma unroll
+    for (int t = 0; t < kBatch; ++t) {
+      const int s = base + t * step;
+      if (s < used) {
+        const float4* src =
+            reinterpret_cast<const float4*>(part + ((size_t)(m * sch.slots + s) * B + b) * 128 + nl);
+        v[t][0] = src[0];
+        v[t][1] = src[1];
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kBatch; ++t) {
+      if (base + t * step < used) {
+        acc[0] += v[t][0].x;
+        acc[1] += v[t][0].y;
+        acc[2] += v[t][0].z;
+        acc[3] += v[t][0].w;
+        acc[4] += v[t][1].x;
+        acc[5] += v[t][1].y;
+        acc[6] += v[t][1].z;
+        acc[7] += v[t][1].w;
+      }
+    }
+  }
+}
+
 // CTAs per block of batch rows: min(148, units), the same on every device,
 // so the summation order (and with it every result bit) does not depend on
 // the device
